@@ -1,0 +1,2 @@
+"""fp64 CPU oracle (test infrastructure only; see svg_oracle.py)."""
+from .svg_oracle import *  # noqa: F401,F403

@@ -1,0 +1,324 @@
+"""Pins of the fp64 oracle to facts the pages and the mathematics fix.
+
+Every check here is independent of the oracle's own code path: hand-derived
+fixtures, closed forms, brute force with scalar loops, a library routine for
+the textbook special case, and invariants.  A plausible slip in the oracle (a
+dropped mask, a wrong index or sign, a transposed operand, a wrong
+normalisation, an inverted label) fails at least one of them.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_video_profile_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "masks_small_cases.txt")
+
+
+# ---------------------------------------------------------------- fixtures
+
+def _read_golden():
+    cases, cur, sec = [], None, None
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("case"):
+            kv = dict(t.split("=") for t in line.split()[1:])
+            cur = {k: int(v) for k, v in kv.items()}
+            cases.append(cur)
+        elif line.startswith("["):
+            sec = line.strip("[]")
+            cur[sec] = []
+        else:
+            cur[sec].append(line)
+    for c in cases:
+        for sec in ("spatial", "temporal", "temporal_token_major"):
+            c[sec] = np.array([[ch == "1" for ch in row] for row in c[sec]])
+        c["pi"] = np.array([int(t) for t in c["pi"][0].split()])
+    return cases
+
+
+@pytest.mark.parametrize("case", _read_golden(), ids=lambda c: f"N{c['N']}F{c['F']}")
+def test_masks_match_hand_derived_fixture(case):
+    N, F, a1, a2 = case["N"], case["F"], case["a1"], case["a2"]
+    np.testing.assert_array_equal(oracle.spatial_mask(N, F, a1), case["spatial"])
+    np.testing.assert_array_equal(oracle.temporal_mask(N, F, a2), case["temporal"])
+    np.testing.assert_array_equal(oracle.token_major_index(N, F), case["pi"])
+    # permuted temporal mask: entry (x', y') of the token-major view
+    pi = oracle.token_major_index(N, F)
+    inv = np.argsort(pi)
+    mt = oracle.temporal_mask(N, F, a2)
+    np.testing.assert_array_equal(mt[np.ix_(inv, inv)], case["temporal_token_major"])
+    np.testing.assert_array_equal(oracle.banded_mask(N * F, N, a2), case["temporal_token_major"])
+
+
+# ------------------------------------------------------------- mask pins
+
+def _masks_by_definition(N, F, a1, a2):
+    """Scalar loops over token pairs (i1, j1), (i2, j2) straight from the
+    (i, j) definitions."""
+    L = N * F
+    ms = np.zeros((L, L), dtype=bool)
+    mt = np.zeros((L, L), dtype=bool)
+    for i1, j1, i2, j2 in itertools.product(range(N), range(F), range(N), range(F)):
+        x1, x2 = i1 * F + j1, i2 * F + j2
+        ms[x1, x2] = abs(i1 - i2) < a1
+        mt[x1, x2] = abs(j1 - j2) < a2
+    return ms, mt
+
+
+@pytest.mark.parametrize("N,F,a1,a2", [(3, 5, 1, 1), (4, 6, 2, 3), (5, 4, 5, 4), (2, 7, 3, 9), (6, 3, 2, 2)])
+def test_masks_match_ij_definition(N, F, a1, a2):
+    ms, mt = _masks_by_definition(N, F, a1, a2)
+    np.testing.assert_array_equal(oracle.spatial_mask(N, F, a1), ms)
+    np.testing.assert_array_equal(oracle.temporal_mask(N, F, a2), mt)
+    # rows= restriction selects the same rows
+    rows = np.array([0, N * F - 1, F // 2 + F])
+    rows = rows[rows < N * F]
+    np.testing.assert_array_equal(oracle.spatial_mask(N, F, a1, rows), ms[rows])
+    np.testing.assert_array_equal(oracle.temporal_mask(N, F, a2, rows), mt[rows])
+
+
+def _closed_count(n, a):
+    # pairs (u, v) in [0, n) with |u - v| < a: the diagonal plus 2 * sum_{t=1}^{a-1} (n - t)
+    a = min(a, n)
+    return n + 2 * sum(n - t for t in range(1, a))
+
+
+@pytest.mark.parametrize("N,F,a1,a2", [(4, 64, 1, 4), (8, 256, 2, 16), (5, 7, 5, 7), (3, 11, 2, 20)])
+def test_mask_density_closed_form_explicit(N, F, a1, a2):
+    ms = oracle.spatial_mask(N, F, a1)
+    mt = oracle.temporal_mask(N, F, a2)
+    assert ms.sum() == F * F * _closed_count(N, a1)
+    assert mt.sum() == N * N * _closed_count(F, a2)
+    # the algebraic form n(2a-1) - a(a-1) of the same count (a <= n)
+    for n, a in ((N, min(a1, N)), (F, min(a2, F))):
+        assert _closed_count(n, a) == n * (2 * a - 1) - a * (a - 1)
+
+
+@pytest.mark.parametrize("name,sp_density,tp_density", [
+    ("tiny", 0.2500, 0.1064), ("small", 0.3438, 0.1174),
+    ("cogvideox", 0.3491, 0.2495), ("hunyuan", 0.1460, 0.1498)])
+def test_mask_density_large_configs_by_row_counting(name, sp_density, tp_density):
+    """Row counts of the oracle's masks (one row per frame for the spatial
+    mask, one row per in-frame position for the temporal one; every other row
+    is a copy by symmetry) against the closed form and the densities the band
+    widths were chosen for."""
+    wl = synth.WORKLOADS[name]
+    N, F, L = wl.N, wl.F, wl.L
+    sp_rows = np.arange(N) * F
+    tp_rows = np.arange(F)
+    sp = oracle.spatial_mask(N, F, wl.a1, sp_rows).sum() * F
+    tp = sum(int(oracle.temporal_mask(N, F, wl.a2, tp_rows[c:c + 64]).sum())
+             for c in range(0, F, 64)) * N
+    assert sp == F * F * _closed_count(N, wl.a1)
+    assert tp == N * N * _closed_count(F, wl.a2)
+    assert abs(sp / L ** 2 - sp_density) < 5e-5
+    assert abs(tp / L ** 2 - tp_density) < 5e-5
+
+
+@pytest.mark.parametrize("N,F,a1,a2", [(4, 6, 2, 3), (5, 24, 3, 4), (3, 10, 1, 10), (7, 5, 4, 1)])
+def test_spatial_is_block_banded_and_permuted_temporal_is_block_banded(N, F, a1, a2):
+    L = N * F
+    np.testing.assert_array_equal(oracle.spatial_mask(N, F, a1), oracle.banded_mask(L, F, a1))
+    pi = oracle.token_major_index(N, F)
+    assert sorted(pi.tolist()) == list(range(L))  # a bijection
+    inv = np.argsort(pi)
+    mt = oracle.temporal_mask(N, F, a2)
+    np.testing.assert_array_equal(mt[np.ix_(inv, inv)], oracle.banded_mask(L, N, a2))
+
+
+@pytest.mark.parametrize("N,F,a2", [(4, 9, 2), (5, 6, 1), (3, 8, 8)])
+def test_temporal_mask_has_2N_minus_1_slashes(N, F, a2):
+    """The unmasked pairs fall on exactly 2N-1 slashes, one per frame offset
+    k = i1 - i2, each holding the pairs |j1 - j2| < a2 ("Sparse Video-Gen",
+    Temporal Head)."""
+    mt = oracle.temporal_mask(N, F, a2)
+    x1, x2 = np.nonzero(mt)
+    k = x1 // F - x2 // F
+    assert sorted(set(k.tolist())) == list(range(-(N - 1), N))
+    for kk in range(-(N - 1), N):
+        assert (k == kk).sum() == (N - abs(kk)) * _closed_count(F, a2)
+
+
+# ------------------------------------------------------------ attention pins
+
+def _brute_attention(q, k, v, mask, scale):
+    """Scalar loops with math.exp: the softmax-weighted average of value rows."""
+    R, d = len(q), len(q[0])
+    out = []
+    for r in range(R):
+        scores = []
+        for y in range(len(k)):
+            if mask is None or mask[r][y]:
+                scores.append((y, scale * sum(q[r][c] * k[y][c] for c in range(d))))
+        mx = max(s for _, s in scores)
+        w = [(y, math.exp(s - mx)) for y, s in scores]
+        z = sum(e for _, e in w)
+        out.append([sum(e * v[y][c] for y, e in w) / z for c in range(len(v[0]))])
+    return np.array(out)
+
+
+def test_attention_matches_bruteforce_with_masks():
+    rng = np.random.default_rng(3)
+    N, F, d = 3, 4, 3
+    L = N * F
+    q, k, v = (rng.standard_normal((L, d)) for _ in range(3))
+    v = rng.standard_normal((L, 5))  # value width differs from d: catches a transposed operand
+    for mask in (None, oracle.spatial_mask(N, F, 2), oracle.temporal_mask(N, F, 2)):
+        got = oracle.attention(q, k, v, mask)
+        ref = _brute_attention(q.tolist(), k.tolist(), v.tolist(),
+                               None if mask is None else mask.tolist(), 1 / math.sqrt(d))
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_dense_attention_matches_library_sdpa():
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((1, 2, 40, 16)) for _ in range(3))
+    got = oracle.dense_attention(q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(t) for t in (q, k, v))).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_invariants():
+    rng = np.random.default_rng(7)
+    q, k = rng.standard_normal((6, 4)), rng.standard_normal((9, 4))
+    mask = rng.random((6, 9)) < 0.5
+    mask[:, 0] = True
+    p = oracle.attention_probs(q, k, mask)
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-14)
+    assert np.all(p[~mask] == 0)
+    # a per-row constant added to the scores changes nothing: append a column
+    # c_r / scale to q and a column of ones to k
+    scale = 0.5
+    c = rng.standard_normal(6) * 10
+    q2 = np.concatenate([q, (c / scale)[:, None]], axis=1)
+    k2 = np.concatenate([k, np.ones((9, 1))], axis=1)
+    np.testing.assert_allclose(oracle.attention_probs(q2, k2, mask, scale),
+                               oracle.attention_probs(q, k, mask, scale), rtol=1e-12, atol=1e-15)
+
+
+def _rand_qkv(B, H, L, d, seed):
+    rng = np.random.default_rng(seed)
+    return tuple(rng.standard_normal((B, H, L, d)) for _ in range(3))
+
+
+def test_full_bands_equal_dense():
+    N, F, d = 4, 6, 8
+    q, k, v = _rand_qkv(1, 2, N * F, d, 11)
+    dense = oracle.dense_attention(q, k, v)
+    for label in (np.array([[0, 0]]), np.array([[1, 1]])):
+        np.testing.assert_allclose(oracle.sparse_attention(q, k, v, label, N, F, N, F), dense,
+                                   rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(oracle.sparse_attention_via_layout(q, k, v, label, N, F, N, F),
+                                   dense, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("N,F,a1,a2", [(4, 6, 2, 2), (5, 8, 1, 3), (3, 12, 3, 5)])
+def test_layout_transformation_is_equivalent(N, F, a1, a2):
+    """permute -> block-banded attention -> unpermute equals attention under
+    the temporal mask in the original layout (SVG2 explainer, 2.A)."""
+    q, k, v = _rand_qkv(1, 2, N * F, 6, 13)
+    label = np.array([[0, 1]])
+    np.testing.assert_allclose(oracle.sparse_attention_via_layout(q, k, v, label, N, F, a1, a2),
+                               oracle.sparse_attention(q, k, v, label, N, F, a1, a2),
+                               rtol=1e-12, atol=1e-13)
+    x = q[0, 0]
+    np.testing.assert_array_equal(oracle.unpermute(oracle.permute(x, N, F), N, F), x)
+    # the token (i, j) lands at row j*N + i
+    xp = oracle.permute(x, N, F)
+    for i, j in itertools.product(range(N), range(F)):
+        np.testing.assert_array_equal(xp[j * N + i], x[i * F + j])
+
+
+def test_rows_subset_matches_full():
+    N, F = 3, 8
+    q, k, v = _rand_qkv(1, 2, N * F, 4, 17)
+    label = np.array([[1, 0]])
+    rows = np.array([0, 5, 9, 23])
+    full = oracle.sparse_attention(q, k, v, label, N, F, 2, 3)
+    part = oracle.sparse_attention(q, k, v, label, N, F, 2, 3, rows=rows)
+    np.testing.assert_allclose(part, full[:, :, rows], rtol=1e-13, atol=1e-14)
+
+
+# ------------------------------------------------------------ profiling pins
+
+def _brute_profile(q, k, v, N, F, a1, a2, rows):
+    d = len(q[0])
+    sc = 1 / math.sqrt(d)
+    ms = [[abs(x // F - y // F) < a1 for y in range(N * F)] for x in rows]
+    mt = [[abs(x % F - y % F) < a2 for y in range(N * F)] for x in rows]
+    qr = [q[x] for x in rows]
+    od = _brute_attention(qr, k, v, None, sc)
+    os_ = _brute_attention(qr, k, v, ms, sc)
+    ot = _brute_attention(qr, k, v, mt, sc)
+    n = len(rows) * len(v[0])
+    mse_s = sum((os_[r][c] - od[r][c]) ** 2 for r in range(len(rows)) for c in range(len(v[0]))) / n
+    mse_t = sum((ot[r][c] - od[r][c]) ** 2 for r in range(len(rows)) for c in range(len(v[0]))) / n
+    return mse_s, mse_t
+
+
+def test_profile_matches_bruteforce():
+    N, F, d = 3, 5, 4
+    q, k, v = _rand_qkv(1, 3, N * F, d, 19)
+    q[0, 1] *= 3.0  # sharpen one head
+    rows = np.array([1, 7, 8, 14])
+    mse, label = oracle.profile_heads(q, k, v, N, F, 2, 2, rows)
+    for h in range(3):
+        ms, mt = _brute_profile(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), N, F, 2, 2, rows)
+        np.testing.assert_allclose(mse[0, h], [ms, mt], rtol=1e-10, atol=1e-15)
+        assert label[0, h] == (1 if mt < ms else 0)
+
+
+def test_profile_special_cases():
+    N, F = 4, 6
+    q, k, v = _rand_qkv(1, 2, N * F, 8, 23)
+    rows = np.array([0, 3, 10, 17, 23])
+    mse, label = oracle.profile_heads(q, k, v, N, F, N, 2, rows)  # spatial band covers all
+    assert np.all(mse[..., 0] == 0) and np.all(mse[..., 1] > 0) and np.all(label == 0)
+    mse, label = oracle.profile_heads(q, k, v, N, F, 1, F, rows)  # temporal band covers all
+    assert np.all(mse[..., 1] == 0) and np.all(mse[..., 0] > 0) and np.all(label == 1)
+    mse, label = oracle.profile_heads(q, k, v, N, F, N, F, rows)  # tie -> spatial
+    assert np.all(mse == 0) and np.all(label == 0)
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_synthetic_heads_get_their_constructed_labels(name):
+    wl = synth.WORKLOADS[name]
+    q, k, v = (synth.round_bf16_to_f64(t) for t in synth.make_qkv(wl, seed=0))
+    rows = synth.sample_rows(wl.L, wl.S, 0)
+    mse, label = oracle.profile_heads(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows)
+    np.testing.assert_array_equal(label, synth.head_kinds(wl, 0))
+    gap = np.abs(mse[..., 0] - mse[..., 1]) / mse.max(-1)
+    assert np.all(gap > 0.2)
+
+
+# ------------------------------------------------------------ block list pin
+
+def _banded_tile_ranges(L, G, a, Bq, Bk, qb):
+    q0, q1 = qb * Bq, min(L, (qb + 1) * Bq)
+    g_lo, g_hi = q0 // G, (q1 - 1) // G
+    lo, hi = max(0, (g_lo - a + 1) * G), min(L, (g_hi + a) * G)
+    f_lo, f_hi = max(0, (g_hi - a + 1) * G), min(L, (g_lo + a) * G)
+    active = set(range(lo // Bk, -(-hi // Bk)))
+    full = {kb for kb in range(-(-L // Bk)) if kb * Bk >= f_lo and min(L, (kb + 1) * Bk) <= f_hi}
+    return active, full
+
+
+@pytest.mark.parametrize("L,G,a,Bq,Bk", [(256, 64, 1, 128, 128), (2048, 8, 16, 128, 128),
+                                         (700, 33, 3, 128, 64), (517, 50, 2, 64, 128),
+                                         (300, 7, 100, 128, 128), (129, 129, 1, 128, 128)])
+def test_block_list_bruteforce_matches_closed_form(L, G, a, Bq, Bk):
+    active, full = oracle.block_list(oracle.banded_mask(L, G, a), Bq, Bk)
+    for qb in range(active.shape[0]):
+        act, ful = _banded_tile_ranges(L, G, a, Bq, Bk, qb)
+        assert set(np.nonzero(active[qb])[0].tolist()) == act
+        assert set(np.nonzero(full[qb])[0].tolist()) == ful
+

@@ -1,0 +1,248 @@
+/*
+ * svg.h -- C ABI of libsvg: spatial/temporal sparse 3D attention for video
+ * diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * The method (Sparse VideoGen) runs four steps right before each 3D attention
+ * call:
+ *   1. online profiling labels every head spatial or temporal
+ *      (svg_profile_heads);
+ *   2. the layout transformation moves temporal heads' Q/K/V from frame-major
+ *      to token-major order (svg_permute / svg_permute_qkv);
+ *   3. block-sparse attention over each head's block-banded pattern
+ *      (svg_block_sparse_attn);
+ *   4. the inverse layout transformation of the output (svg_unpermute).
+ * svg_sparse_3d_attn runs all four.  svg_dense_attn is the unmasked reference.
+ *
+ * Sources, cited by page title and section:
+ *   "Sparse Video-Gen" author rebuttal (paperhub.cn): Weakness 1 answer
+ *     (token indexing x = i*F + j; Spatial Head mask |i1-i2| < a1; Temporal
+ *     Head mask |j1-j2| < a2) and the later Weakness 1 answer on online
+ *     profiling (per step and layer, right before attention; labels -1/+1).
+ *   "Sparse VideoGen: Accelerating Video Diffusion Transformers with
+ *     Spatial-Temporal Sparsity" (newx.sg): Abstract (online profiling,
+ *     hardware-efficient layout transformation, custom kernels).
+ *   SVG2 explainer (gist.science), 2.A "Semantic-Aware Permutation": a token
+ *     permutation applied before attention and undone after it leaves the
+ *     output unchanged.
+ *
+ * Conventions shared by every entry point
+ *   Shapes.   B batch, H heads, N frames, F tokens per frame, L = N*F tokens,
+ *             d head dim.  Token (i, j) (frame i, in-frame position j) sits at
+ *             row x = i*F + j of the frame-major layout.
+ *   Layout.   Every Q/K/V/O tensor is contiguous [B, H, L, d], row-major, d
+ *             fastest, in the element type of shape->dtype (bf16 or fp32).
+ *             Token-major ("permuted") tensors have the same shape with
+ *             token (i, j) at row x' = j*N + i.
+ *   Labels.   int8 per (b, h), [B, H]: SVG_SPATIAL (0) or SVG_TEMPORAL (1),
+ *             standing for the pages' -1 and +1.
+ *   Memory.   The caller allocates and owns every buffer.  Pointers named
+ *             *_dev or described as device memory are CUDA device pointers;
+ *             tensor pointers must be 16-byte aligned.  No entry point
+ *             allocates or frees memory or synchronises the stream.
+ *   Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *             device work is enqueued asynchronously on it.
+ *   Errors.   The return value reports argument errors (SVG_ERR_INVALID_ARG,
+ *             SVG_ERR_UNSUPPORTED, SVG_ERR_WORKSPACE) before anything is
+ *             enqueued, and launch errors (SVG_ERR_CUDA) after.  Errors that
+ *             happen on the device (a bounded wait that ran out) are OR-ed
+ *             into the optional device word `status_dev` as SVG_DEV_* bits;
+ *             read it after the stream has synchronised.  svg_last_error()
+ *             gives a message for the last failing call on this host thread.
+ *   Support.  bf16: d in {64, 128}.  fp32: d in {32, 64, 128}.  a1 >= 1,
+ *             a2 >= 1 (a1 >= N or a2 >= F keep every pair of that kind).
+ */
+#ifndef SVG_H_
+#define SVG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVG_API __attribute__((visibility("default")))
+#else
+#define SVG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svg_status {
+  SVG_OK = 0,
+  SVG_ERR_INVALID_ARG = 1, /* null pointer, bad size or band, misalignment */
+  SVG_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d = 96)      */
+  SVG_ERR_CUDA = 3,        /* a CUDA call or launch failed                */
+  SVG_ERR_TIMEOUT = 4,     /* reserved for host-side reporting of SVG_DEV_TIMEOUT */
+  SVG_ERR_WORKSPACE = 5    /* workspace smaller than the size query says   */
+} svg_status;
+
+typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
+
+#define SVG_SPATIAL 0
+#define SVG_TEMPORAL 1
+
+/* Bits of the device status word. */
+#define SVG_DEV_TIMEOUT 0x1u  /* a pipeline wait exceeded its bound; outputs invalid */
+
+typedef struct svg_shape {
+  int32_t B, H, N, F, d;
+  int32_t dtype; /* svg_dtype */
+  float scale;   /* softmax scale on q.k; 0 selects 1/sqrt(d) */
+} svg_shape;
+
+/* ABI version of this header (bumped on any signature change). */
+#define SVG_ABI_VERSION 1
+SVG_API int32_t svg_abi_version(void);
+
+/* Static text for a status code; never NULL. */
+SVG_API const char* svg_status_string(int32_t status);
+
+/* Message for the last non-OK status returned on the calling host thread. */
+SVG_API const char* svg_last_error(void);
+
+/*
+ * svg_attn_tile -- query/key tile sizes (rows) of the attention kernel for a
+ * given dtype and head dim, i.e. the Bq x Bk tiling its block list refers to.
+ * Host only.
+ */
+SVG_API svg_status svg_attn_tile(int32_t dtype, int32_t d, int32_t* Bq, int32_t* Bk);
+
+/*
+ * svg_block_list -- the block schedule of a block-banded mask, host only.
+ *
+ * Mask: keep (x, y) iff |floor(x/G) - floor(y/G)| < a over L tokens.  With
+ * G = F, a = a1 this is the spatial mask ("Sparse Video-Gen", Spatial Head:
+ * block-banded with the main and +-(a1-1) neighbouring block diagonals); with
+ * G = N, a = a2 it is the temporal mask after the token-major layout
+ * transformation.  For each query tile qb (rows [qb*Bq, min(L,(qb+1)*Bq))),
+ * writes the key-tile ranges [kb_lo[qb], kb_hi[qb]) of tiles with any kept
+ * element and [full_lo[qb], full_hi[qb]) of tiles with every element kept
+ * (an empty range has lo == hi).  These are the tiles the attention kernel
+ * visits and the ones it visits without an elementwise mask.
+ * Arrays: host memory, ceil(L/Bq) int32 each, owned by the caller.
+ * Errors: SVG_ERR_INVALID_ARG if L, G, a, Bq or Bk < 1 or a pointer is NULL.
+ */
+SVG_API svg_status svg_block_list(int32_t L, int32_t G, int32_t a, int32_t Bq, int32_t Bk,
+                          int32_t* kb_lo, int32_t* kb_hi, int32_t* full_lo, int32_t* full_hi);
+
+/*
+ * svg_profile_workspace_size -- bytes of device workspace svg_profile_heads
+ * needs for this shape and sample count (0 on invalid arguments).
+ */
+SVG_API size_t svg_profile_workspace_size(const svg_shape* shape, int32_t S);
+
+/*
+ * svg_profile_heads -- online profiling ("Sparse Video-Gen", Weakness 1
+ * answer on online profiling; "Sparse VideoGen ...", Abstract).
+ *
+ * For every head (b, h) and every sampled query row x = rows[s], computes
+ * the exact attention output of that row with no mask (O_dense), under the
+ * spatial mask |i_x - i_y| < a1 (O_s) and under the temporal mask
+ * |j_x - j_y| < a2 (O_t), in fp32 from the given inputs, then
+ *   mse[b,h,0] = mean over S*d of (O_s - O_dense)^2,
+ *   mse[b,h,1] = mean over S*d of (O_t - O_dense)^2,
+ *   label[b,h] = SVG_TEMPORAL if mse[b,h,1] < mse[b,h,0] else SVG_SPATIAL.
+ * The reduction order is fixed, so repeated calls give identical bits.
+ *
+ * q, k, v   device, [B,H,L,d] frame-major, dtype of shape.
+ * rows      device, int32 [S], each in [0, L) (duplicates allowed), shared by
+ *           every head.  1 <= S <= 128.
+ * mse       device, float [B,H,2] (written).
+ * label     device, int8 [B,H] (written).
+ * workspace device, >= svg_profile_workspace_size(shape, S) bytes, 256-byte
+ *           aligned; contents on entry do not matter.
+ * Errors: SVG_ERR_INVALID_ARG (null pointer, S out of range, a1/a2 < 1),
+ *         SVG_ERR_UNSUPPORTED (dtype/d), SVG_ERR_WORKSPACE, SVG_ERR_CUDA.
+ */
+SVG_API svg_status svg_profile_heads(const svg_shape* shape, const void* q, const void* k, const void* v,
+                             int32_t a1, int32_t a2, const int32_t* rows, int32_t S, float* mse,
+                             int8_t* label, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * svg_permute -- the layout transformation ("Sparse VideoGen ...", Abstract;
+ * SVG2 explainer 2.A) of one tensor: for every head with label[b,h] ==
+ * SVG_TEMPORAL, xp[b,h, j*N+i, :] = x[b,h, i*F+j, :].  Rows of spatial heads
+ * in xp are not written.  label == NULL permutes every head.
+ * x, xp: device [B,H,L,d], distinct, 16-byte aligned.  label: device or NULL.
+ */
+SVG_API svg_status svg_permute(const svg_shape* shape, const void* x, void* xp, const int8_t* label,
+                       void* stream);
+
+/* svg_permute_qkv -- svg_permute of q, k and v in one launch. */
+SVG_API svg_status svg_permute_qkv(const svg_shape* shape, const void* q, const void* k, const void* v,
+                           void* qp, void* kp, void* vp, const int8_t* label, void* stream);
+
+/*
+ * svg_unpermute -- inverse layout transformation: for every head with
+ * label[b,h] == SVG_TEMPORAL, x[b,h, i*F+j, :] = xp[b,h, j*N+i, :].  Rows of
+ * spatial heads in x are not written.  label == NULL unpermutes every head.
+ */
+SVG_API svg_status svg_unpermute(const svg_shape* shape, const void* xp, void* x, const int8_t* label,
+                         void* stream);
+
+/*
+ * svg_block_sparse_attn -- block-sparse attention over each head's banded
+ * pattern (the "customized kernel" of "Sparse VideoGen ...", Abstract; masks
+ * from "Sparse Video-Gen", Spatial Head / Temporal Head).
+ *
+ *   spatial head:  O = softmax(scale*QK^T + M)V on q,k,v -> o, with M = 0 iff
+ *                  |floor(x/F) - floor(y/F)| < a1 (frame-major rows);
+ *   temporal head: the same on qp,kp,vp -> op with G = N, a = a2, i.e.
+ *                  |floor(x'/N) - floor(y'/N)| < a2 on token-major rows, which
+ *                  is the temporal mask |j1-j2| < a2 after the layout
+ *                  transformation.
+ * All heads run in one launch; the key range of each query tile is computed
+ * on the fly from (G, a); no mask tensor is read.  Rows of temporal heads in
+ * o and of spatial heads in op are not written.
+ *
+ * q,k,v,o      device [B,H,L,d] frame-major.
+ * qp,kp,vp,op  device [B,H,L,d] token-major (temporal heads' slices are used);
+ *              may be NULL when no head is temporal.
+ * label        device int8 [B,H].
+ * status_dev   device int32 or NULL (SVG_DEV_* bits OR-ed in).
+ */
+SVG_API svg_status svg_block_sparse_attn(const svg_shape* shape, const void* q, const void* k,
+                                 const void* v, const void* qp, const void* kp, const void* vp,
+                                 void* o, void* op, const int8_t* label, int32_t a1, int32_t a2,
+                                 int32_t* status_dev, void* stream);
+
+/*
+ * svg_banded_attn -- the same kernel with one band for every head:
+ * keep (x, y) iff |floor(x/G) - floor(y/G)| < a, on q,k,v -> o as given
+ * (no label, no permutation).  G >= L or a large gives dense attention.
+ */
+SVG_API svg_status svg_banded_attn(const svg_shape* shape, const void* q, const void* k, const void* v,
+                           void* o, int32_t G, int32_t a, int32_t* status_dev, void* stream);
+
+/*
+ * svg_dense_attn -- unmasked attention softmax(scale*QK^T)V of every head,
+ * the reference the sparse call is compared with.  Same kernel, one band
+ * covering all L tokens.
+ */
+SVG_API svg_status svg_dense_attn(const svg_shape* shape, const void* q, const void* k, const void* v,
+                          void* o, int32_t* status_dev, void* stream);
+
+/*
+ * svg_sparse_3d_attn_workspace_size -- bytes of device workspace the fused
+ * call needs: token-major copies of q, k, v and o plus the profiling
+ * workspace (0 on invalid arguments).
+ */
+SVG_API size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t S);
+
+/*
+ * svg_sparse_3d_attn -- one whole sparse 3D-attention call: profile ->
+ * permute temporal heads -> block-sparse attention -> unpermute, all
+ * enqueued on `stream` with no host synchronisation.  Outputs o (frame-major
+ * [B,H,L,d]) plus the profiling results mse [B,H,2] and label [B,H] (device).
+ * Arguments as in the four calls above.
+ */
+SVG_API svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v,
+                              void* o, int32_t a1, int32_t a2, const int32_t* rows, int32_t S,
+                              float* mse, int8_t* label, void* workspace, size_t workspace_bytes,
+                              int32_t* status_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVG_H_ */

@@ -1,0 +1,444 @@
+// attn_sm100.cu -- block-sparse (banded) attention on B200 tensor cores.
+//
+// Computes, per head, O = softmax(scale * Q K^T + M) V with
+//   M[x, y] = 0 iff |floor(x/G) - floor(y/G)| < a, else -inf,
+// the block-banded form of the spatial mask ("Sparse Video-Gen", Spatial
+// Head: G = F, a = a1) and of the temporal mask after the token-major layout
+// transformation ("Sparse VideoGen ...", Abstract; G = N, a = a2).  These are
+// the "customized kernel implementations" the pages name without giving a
+// design; the design here is B200-native.
+//
+// Because the band is contiguous in the key index, a query tile [q0, q1)
+// only needs keys [max(0, (g(q0)-a+1) G), min(L, (g(q1-1)+a) G)).  The kernel
+// derives that range from (G, a) on the fly -- no mask tensor, no block list
+// in memory -- and masks elementwise only in tiles a row's band does not
+// fully cover.
+//
+// One CTA = 256 query rows = two 128-row Q tiles sharing every K/V tile:
+//   warp 8      TMA producer: Q tiles once, then K_k / V_k into a ring of
+//               128-key slots (128-byte swizzle, OOB rows zero-filled);
+//   warp 9      one thread issues tcgen05.mma: S_i = Q_i K^T into TMEM, and
+//               O_i += P_i V with P_i read straight from TMEM;
+//   warps 0-3   softmax of Q tile 0, warps 4-7 softmax of Q tile 1: one thread
+//               per query row reads its S row from TMEM, applies the band
+//               mask on edge tiles, keeps the running max / sum, writes P as
+//               bf16 back into the S columns, and rescales its O row in TMEM
+//               only when the max grew by more than 2^8 (lazy rescaling).
+// The MMA order S_0, S_1, then per key tile {P_0 V, S_0 <- next}, {P_1 V,
+// S_1 <- next} lets the tensor core work on one Q tile while the other's
+// softmax runs.
+// TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D,256+2D).
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace svg {
+namespace {
+
+struct AttnParams {
+  CUtensorMap tm_q, tm_k, tm_v;     // frame-major [BH, L, D] bf16
+  CUtensorMap tm_qp, tm_kp, tm_vp;  // token-major [BH, L, D] bf16
+  __nv_bfloat16* o;
+  __nv_bfloat16* op;
+  const int8_t* label;
+  int BH, L, n_ctiles;
+  int G0, a0, G1, a1;
+  float sl2;      // scale * log2(e)
+  float lazy_th;  // rescale threshold in raw score units (8 / sl2)
+  int* status;
+  uint64_t wait_ns;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int BQ = 128;          // rows per Q tile (MMA M)
+  static constexpr int BK = 128;          // keys per K/V tile
+  static constexpr int HALVES = D / 64;   // 128-byte swizzle rows hold 64 bf16
+  static constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = BK * D * 2;
+  static constexpr int NS = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int SMEM_Q = 2 * TILE_BYTES;
+  static constexpr int SMEM_BAR = SMEM_Q + NS * TILE_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;  // barriers + alignment slack
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t col_s(int i) { return 128u * i; }
+  static constexpr uint32_t col_o(int i) { return 256u + D * i; }
+};
+
+__device__ __forceinline__ void record_timeout(const AttnParams& p, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
+}
+
+// Warp-uniform bounded wait.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit) {
+  const bool ok = mbar_wait(bar, parity, limit);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constant__ AttnParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sRing = smem + C::SMEM_Q;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_full = bars + 1;
+  uint64_t* bar_empty = bars + 1 + C::NS;
+  uint64_t* bar_s = bars + 1 + 2 * C::NS;  // [2] S_i ready
+  uint64_t* bar_p = bar_s + 2;             // [2] P_i written (128 arrivals)
+  uint64_t* bar_o = bar_p + 2;             // [2] P_i V done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_o + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = (*reinterpret_cast<volatile int*>(p.status) & SVG_DEV_TIMEOUT) ? 1 : 0;
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], 128);
+      mbar_init(&bar_o[i], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- work item: (head, 256-row query slab)
+  const int ct = blockIdx.x % p.n_ctiles;
+  const int bh = blockIdx.x / p.n_ctiles;
+  const int lab = p.label ? static_cast<int>(p.label[bh]) : 0;
+  const int G = lab ? p.G1 : p.G0;
+  const int a = lab ? p.a1 : p.a0;
+  const int L = p.L;
+  const int q0 = ct * 256;
+  const int q_last = min(q0 + 255, L - 1);
+  const long long g_first = q0 / G, g_last = q_last / G;
+  const int lo_cta = static_cast<int>(max(0LL, (g_first - a + 1) * G));
+  const int hi_cta = static_cast<int>(min(static_cast<long long>(L), (g_last + a) * G));
+  const int kt0 = lo_cta / C::BK;
+  const int nk = (hi_cta + C::BK - 1) / C::BK - kt0;
+  const bool run = (*abort_flag == 0);
+
+  if (run && warp == 8) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const CUtensorMap* tq = lab ? &p.tm_qp : &p.tm_q;
+      const CUtensorMap* tk = lab ? &p.tm_kp : &p.tm_k;
+      const CUtensorMap* tv = lab ? &p.tm_vp : &p.tm_v;
+      tma_prefetch_desc(tq);
+      tma_prefetch_desc(tk);
+      tma_prefetch_desc(tv);
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_3d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, tq, bar_q, h * 64, q0 + i * C::BQ, bh);
+      for (int n = 0; n < 2 * nk; ++n) {
+        const int slot = n % C::NS;
+        const uint32_t ph = (n / C::NS) & 1;
+        if (!mbar_wait(&bar_empty[slot], ph ^ 1, p.wait_ns)) {
+          record_timeout(p, abort_flag);
+          break;
+        }
+        const CUtensorMap* tm = (n & 1) ? tv : tk;
+        const int row = (kt0 + (n >> 1)) * C::BK;
+        mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, row, bh);
+      }
+    }
+  } else if (run && warp == 9) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t ring_base = smem_u32(sRing);
+      auto issue_qk = [&](int i, int slot) {
+        const uint32_t a0 = q_base + i * C::TILE_BYTES;
+        const uint32_t b0 = ring_base + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::HALF_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + C::col_s(i), smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024),
+                  idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_s[i]);
+      };
+      auto issue_pv = [&](int i, int slot, bool acc) {
+        const uint32_t b0 = ring_base + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          umma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
+                  smem_desc_sw128(b0 + kk * 16 * 128, C::HALF_BYTES, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        umma_commit(&bar_o[i]);
+      };
+      bool ok = mbar_wait(bar_q, 0, p.wait_ns) && mbar_wait(&bar_full[0], 0, p.wait_ns);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        issue_qk(1, 0);
+        umma_commit(&bar_empty[0]);
+      }
+      for (int k = 0; ok && k < nk; ++k) {
+        const int nV = 2 * k + 1, nK = 2 * k + 2;
+        const int slotV = nV % C::NS, slotK = nK % C::NS;
+        const bool has_next = k + 1 < nk;
+        ok = mbar_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
+        for (int i = 0; ok && i < 2; ++i) {
+          ok = mbar_wait(&bar_p[i], k & 1, p.wait_ns);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(i, slotV, k > 0);
+          if (has_next) {
+            if (i == 0) {
+              ok = mbar_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_qk(i, slotK);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&bar_empty[slotV]);
+        if (has_next) umma_commit(&bar_empty[slotK]);
+      }
+      if (!ok) record_timeout(p, abort_flag);
+    }
+  } else if (run && warp < 8) {
+    // ------------------------------------------------ softmax / epilogue
+    const int i = warp >> 2;
+    const int quad = warp & 3;
+    const int r = q0 + i * C::BQ + quad * 32 + lane;  // query row in the head's layout
+    const bool row_ok = r < L;
+    int lo_r = 0, hi_r = 0;
+    if (row_ok) {
+      const long long g = r / G;
+      lo_r = static_cast<int>(max(0LL, (g - a + 1) * G));
+      hi_r = static_cast<int>(min(static_cast<long long>(L), (g + a) * G));
+    }
+    const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + C::col_s(i);
+    const uint32_t tO = tmem + lane_bits + C::col_o(i);
+    const float sl2 = p.sl2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int k = 0; k < nk; ++k) {
+      if (!warp_wait(&bar_s[i], k & 1, p.wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(sr[c][e]);
+
+      const int kbase = (kt0 + k) * C::BK;
+      if (kbase < lo_r || kbase + C::BK > hi_r) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int y = kbase + c;
+          if (y < lo_r || y >= hi_r) s[c] = -INFINITY;
+        }
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float m_new = fmaxf(fmaxf(m_used, fmaxf(mx0, mx1)), fmaxf(mx2, mx3));
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_new > m_used + p.lazy_th) {  // false while both are -inf
+        alpha = ex2_approx((m_used - m_new) * sl2);  // 0 when m_used is -inf
+        m_used = m_new;
+        resc = true;
+      }
+      l *= alpha;
+      const float nb = (m_used == -INFINITY) ? 0.f : -m_used * sl2;
+      uint32_t pk[2][32];
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, nb));
+        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, nb));
+        ls0 += p0;
+        ls1 += p1;
+        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+      }
+      l += ls0 + ls1;
+      __syncwarp();
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+      if (k > 0 && __any_sync(0xffffffffu, resc)) {
+        // O_i must hold P_i(k-1) V before it is rescaled.
+        if (!warp_wait(&bar_o[i], (k - 1) & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tmem_wait_ld();
+          reg_fence32(ov);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tO + c * 32, ov);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_p[i]);
+    }
+    if (ok && warp_wait(&bar_o[i], (nk - 1) & 1, p.wait_ns)) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* out = (lab ? p.op : p.o) + (static_cast<size_t>(bh) * L + (row_ok ? r : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        __syncwarp();
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+        reg_fence32(ov);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    } else {
+      record_timeout(p, abort_flag);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [BH, L, D] bf16, box = 64 elements x 128 rows x 1 head, 128-byte swizzle.
+svg_status make_map(CUtensorMap* map, const void* base, int BH, int L, int D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SVG_OK;
+}
+
+template <int D>
+svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
+  using C = Cfg<D>;
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  const int BH = a.B * a.H;
+  svg_status st;
+  if ((st = make_map(&p.tm_q, a.q, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_map(&p.tm_k, a.k, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_map(&p.tm_v, a.v, BH, a.L, D)) != SVG_OK) return st;
+  const bool perm = a.label != nullptr;
+  if ((st = make_map(&p.tm_qp, perm ? a.qp : a.q, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_map(&p.tm_kp, perm ? a.kp : a.k, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_map(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.op = static_cast<__nv_bfloat16*>(perm ? a.op : a.o);
+  p.label = a.label;
+  p.BH = BH;
+  p.L = a.L;
+  p.n_ctiles = (a.L + 255) / 256;
+  p.G0 = a.G0;
+  p.a0 = a.a0;
+  p.G1 = a.G1;
+  p.a1 = a.a1;
+  p.sl2 = a.scale * 1.4426950408889634f;
+  p.lazy_th = 8.0f / p.sl2;
+  p.status = a.status;
+  p.wait_ns = a.wait_ns;
+  const long long grid = static_cast<long long>(BH) * p.n_ctiles;
+  if (grid > 0x7fffffffLL) return fail(SVG_ERR_UNSUPPORTED, "grid too large");
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(attention smem)");
+    attr_set = true;
+  }
+  attn_sm100_kernel<D><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cuda_check(cudaGetLastError(), "attention launch");
+}
+
+}  // namespace
+
+svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream) {
+  switch (a.d) {
+    case 64: return launch_d<64>(a, stream);
+    case 128: return launch_d<128>(a, stream);
+    default: return fail(SVG_ERR_UNSUPPORTED, "bf16 attention supports d in {64, 128}, got %d", a.d);
+  }
+}
+
+}  // namespace svg

@@ -1,0 +1,73 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "svg.h"
+
+namespace svg {
+
+// Upper bound on any single pipeline wait inside a kernel.  Waits in a
+// healthy run last microseconds; the bound only turns a stall into an error.
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+
+// Records a message for svg_last_error() and returns `st`.
+svg_status fail(svg_status st, const char* fmt, ...);
+// Maps a CUDA error to SVG_ERR_CUDA with a message; SVG_OK if e == cudaSuccess.
+svg_status cuda_check(cudaError_t e, const char* what);
+
+// ------------------------------------------------------------- permute
+
+// Moves rows between frame-major (x = i*F + j) and token-major (x' = j*N + i)
+// order for up to three tensors.  to_token_major: src frame-major -> dst
+// token-major; otherwise the inverse.  label == nullptr: every head.
+svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F,
+                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream);
+
+// ------------------------------------------------------------- attention
+
+struct BandAttnArgs {
+  int B, H, L, d;
+  int dtype;  // svg_dtype
+  float scale;
+  // frame-major tensors (spatial heads, or all heads when label == nullptr)
+  const void *q, *k, *v;
+  void* o;
+  // token-major tensors (temporal heads)
+  const void *qp, *kp, *vp;
+  void* op;
+  const int8_t* label;  // nullptr -> every head uses band 0 on (q, k, v, o)
+  int G0, a0;           // band of label-0 heads
+  int G1, a1;           // band of label-1 heads
+  int* status;          // device status word (never null here)
+  uint64_t wait_ns;
+};
+
+svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);
+svg_status launch_attn_simt(const BandAttnArgs& a, cudaStream_t stream);
+// Tile shape of the tcgen05 kernel (rows of Q per tile, keys per tile).
+constexpr int kAttnBq = 128;
+constexpr int kAttnBk = 128;
+
+// ------------------------------------------------------------- profiling
+
+struct ProfileLayout {
+  int S_pad;      // sampled rows rounded up to the row-block of the kernel
+  int n_chunks;   // key chunks per head
+  int chunk;      // keys per chunk (multiple of 64)
+  size_t o_bytes;   // partial outputs  [BH][n_chunks][3][S_pad][d] f32
+  size_t ml_bytes;  // partial max/sum  [BH][n_chunks][3][S_pad][2] f32
+  size_t total;
+};
+
+bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out);
+
+svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
+                          const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
+                          float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
+                          cudaStream_t stream);
+
+}  // namespace svg

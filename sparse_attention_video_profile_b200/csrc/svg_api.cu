@@ -1,0 +1,323 @@
+// svg_api.cu -- the C ABI declared in include/svg.h: argument checking,
+// workspace accounting and kernel dispatch.  No entry point allocates
+// memory or synchronises the stream.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "internal.h"
+
+namespace svg {
+
+static thread_local char g_last_error[512] = "";
+
+svg_status fail(svg_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+svg_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SVG_OK;
+  return fail(SVG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+namespace {
+
+// Per-device status word used when the caller passes no status_dev.
+__device__ int g_internal_status;
+
+size_t elem_size(int dtype) { return dtype == SVG_FP32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+svg_status check_shape(const svg_shape* s) {
+  if (s == nullptr) return fail(SVG_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->H < 1 || s->N < 1 || s->F < 1 || s->d < 1)
+    return fail(SVG_ERR_INVALID_ARG, "B, H, N, F, d must be >= 1 (got %d %d %d %d %d)", s->B, s->H, s->N, s->F, s->d);
+  if (static_cast<long long>(s->N) * s->F > (1LL << 30))
+    return fail(SVG_ERR_INVALID_ARG, "L = N*F = %lld is too large", static_cast<long long>(s->N) * s->F);
+  if (s->dtype != SVG_BF16 && s->dtype != SVG_FP32) return fail(SVG_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+  if (!(s->scale >= 0.f) || isinf(s->scale)) return fail(SVG_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (s->dtype == SVG_BF16 && s->d != 64 && s->d != 128)
+    return fail(SVG_ERR_UNSUPPORTED, "bf16 supports d in {64, 128}, got %d", s->d);
+  if (s->dtype == SVG_FP32 && s->d != 32 && s->d != 64 && s->d != 128)
+    return fail(SVG_ERR_UNSUPPORTED, "fp32 supports d in {32, 64, 128}, got %d", s->d);
+  return SVG_OK;
+}
+
+float eff_scale(const svg_shape* s) { return s->scale > 0.f ? s->scale : 1.0f / sqrtf(static_cast<float>(s->d)); }
+
+svg_status check_tensors(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(SVG_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    if (!aligned16(p)) return fail(SVG_ERR_INVALID_ARG, "a tensor pointer is not 16-byte aligned");
+  }
+  return SVG_OK;
+}
+
+// Clamp a band so that (g + a) * G cannot overflow: a >= ceil(L/G) already
+// keeps every pair.
+int clamp_band(int a, int G, int L) {
+  const int full = (L + G - 1) / G;
+  return a > full ? full : a;
+}
+
+svg_status status_word(int32_t* user, int** out, cudaStream_t stream) {
+  if (user != nullptr) {
+    *out = user;
+    return SVG_OK;
+  }
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_internal_status);
+  if (e != cudaSuccess) return cuda_check(e, "cudaGetSymbolAddress(status)");
+  e = cudaMemsetAsync(p, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_check(e, "cudaMemsetAsync(status)");
+  *out = static_cast<int*>(p);
+  return SVG_OK;
+}
+
+svg_status run_attention(const svg_shape* s, BandAttnArgs& a, int32_t* status_dev, cudaStream_t stream) {
+  a.B = s->B;
+  a.H = s->H;
+  a.L = s->N * s->F;
+  a.d = s->d;
+  a.dtype = s->dtype;
+  a.scale = eff_scale(s);
+  a.wait_ns = kDefaultWaitNs;
+  svg_status st = status_word(status_dev, &a.status, stream);
+  if (st != SVG_OK) return st;
+  if (s->dtype == SVG_BF16) return launch_attn_sm100(a, stream);
+  return launch_attn_simt(a, stream);
+}
+
+}  // namespace
+}  // namespace svg
+
+using namespace svg;
+
+extern "C" {
+
+int32_t svg_abi_version(void) { return SVG_ABI_VERSION; }
+
+const char* svg_status_string(int32_t st) {
+  switch (st) {
+    case SVG_OK: return "SVG_OK";
+    case SVG_ERR_INVALID_ARG: return "SVG_ERR_INVALID_ARG";
+    case SVG_ERR_UNSUPPORTED: return "SVG_ERR_UNSUPPORTED";
+    case SVG_ERR_CUDA: return "SVG_ERR_CUDA";
+    case SVG_ERR_TIMEOUT: return "SVG_ERR_TIMEOUT";
+    case SVG_ERR_WORKSPACE: return "SVG_ERR_WORKSPACE";
+    default: return "SVG_ERR_UNKNOWN";
+  }
+}
+
+const char* svg_last_error(void) { return g_last_error; }
+
+svg_status svg_attn_tile(int32_t dtype, int32_t d, int32_t* Bq, int32_t* Bk) {
+  if (Bq == nullptr || Bk == nullptr) return fail(SVG_ERR_INVALID_ARG, "NULL output");
+  if (dtype == SVG_BF16) {
+    if (d != 64 && d != 128) return fail(SVG_ERR_UNSUPPORTED, "bf16 supports d in {64, 128}");
+    *Bq = kAttnBq;
+    *Bk = kAttnBk;
+    return SVG_OK;
+  }
+  if (dtype == SVG_FP32) {  // one row at a time, 32 keys per step
+    *Bq = 1;
+    *Bk = 32;
+    return SVG_OK;
+  }
+  return fail(SVG_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+}
+
+svg_status svg_block_list(int32_t L, int32_t G, int32_t a, int32_t Bq, int32_t Bk, int32_t* kb_lo, int32_t* kb_hi,
+                          int32_t* full_lo, int32_t* full_hi) {
+  if (L < 1 || G < 1 || a < 1 || Bq < 1 || Bk < 1) return fail(SVG_ERR_INVALID_ARG, "L, G, a, Bq, Bk must be >= 1");
+  if (!kb_lo || !kb_hi || !full_lo || !full_hi) return fail(SVG_ERR_INVALID_ARG, "NULL output array");
+  const int nq = (L + Bq - 1) / Bq;
+  const long long aa = clamp_band(a, G, L);
+  for (int qb = 0; qb < nq; ++qb) {
+    const long long q0 = static_cast<long long>(qb) * Bq;
+    const long long q1 = q0 + Bq < L ? q0 + Bq : L;
+    const long long g_lo = q0 / G, g_hi = (q1 - 1) / G;
+    // keys any row of the tile keeps: union of the rows' bands
+    long long lo = (g_lo - aa + 1) * G;
+    if (lo < 0) lo = 0;
+    long long hi = (g_hi + aa) * G;
+    if (hi > L) hi = L;
+    kb_lo[qb] = static_cast<int32_t>(lo / Bk);
+    kb_hi[qb] = static_cast<int32_t>((hi + Bk - 1) / Bk);
+    // keys every row keeps: intersection of the rows' bands
+    long long flo = (g_hi - aa + 1) * G;
+    if (flo < 0) flo = 0;
+    long long fhi = (g_lo + aa) * G;
+    if (fhi > L) fhi = L;
+    long long f0 = (flo + Bk - 1) / Bk;  // first tile starting at or after flo
+    long long f1;                         // one past the last tile ending at or before fhi
+    if (fhi >= L) f1 = (L + Bk - 1) / Bk;  // the ragged last tile ends at L
+    else f1 = fhi / Bk;
+    if (f1 < f0) f1 = f0;
+    full_lo[qb] = static_cast<int32_t>(f0);
+    full_hi[qb] = static_cast<int32_t>(f1);
+  }
+  return SVG_OK;
+}
+
+size_t svg_profile_workspace_size(const svg_shape* shape, int32_t S) {
+  if (check_shape(shape) != SVG_OK) return 0;
+  ProfileLayout lay;
+  if (!profile_layout(shape->B, shape->H, shape->N * shape->F, shape->d, shape->dtype, S, &lay)) return 0;
+  return lay.total;
+}
+
+svg_status svg_profile_heads(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
+                             int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v})) != SVG_OK) return st;
+  if (!rows || !mse || !label || !workspace) return fail(SVG_ERR_INVALID_ARG, "NULL rows/mse/label/workspace");
+  if (a1 < 1 || a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a1 and a2 must be >= 1");
+  const int L = shape->N * shape->F;
+  if (S < 1 || S > 128 || S > L) return fail(SVG_ERR_INVALID_ARG, "S must be in [1, min(128, L)], got %d", S);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  ProfileLayout lay;
+  profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay);
+  if (workspace_bytes < lay.total)
+    return fail(SVG_ERR_WORKSPACE, "profile workspace %zu bytes < %zu required", workspace_bytes, lay.total);
+  return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, eff_scale(shape), q, k, v,
+                        clamp_band(a1, 1, shape->N), clamp_band(a2, 1, shape->F), rows, S, mse, label, workspace, lay,
+                        static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_permute(const svg_shape* shape, const void* x, void* xp, const int8_t* label, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({x, xp})) != SVG_OK) return st;
+  if (x == xp) return fail(SVG_ERR_INVALID_ARG, "permute cannot run in place");
+  const void* src[1] = {x};
+  void* dst[1] = {xp};
+  return launch_permute(1, src, dst, shape->B * shape->H, shape->N, shape->F,
+                        static_cast<int>(shape->d * elem_size(shape->dtype)), label, true,
+                        static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_permute_qkv(const svg_shape* shape, const void* q, const void* k, const void* v, void* qp, void* kp,
+                           void* vp, const int8_t* label, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v, qp, kp, vp})) != SVG_OK) return st;
+  if (q == qp || k == kp || v == vp) return fail(SVG_ERR_INVALID_ARG, "permute cannot run in place");
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qp, kp, vp};
+  return launch_permute(3, src, dst, shape->B * shape->H, shape->N, shape->F,
+                        static_cast<int>(shape->d * elem_size(shape->dtype)), label, true,
+                        static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_unpermute(const svg_shape* shape, const void* xp, void* x, const int8_t* label, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({xp, x})) != SVG_OK) return st;
+  if (x == xp) return fail(SVG_ERR_INVALID_ARG, "unpermute cannot run in place");
+  const void* src[1] = {xp};
+  void* dst[1] = {x};
+  return launch_permute(1, src, dst, shape->B * shape->H, shape->N, shape->F,
+                        static_cast<int>(shape->d * elem_size(shape->dtype)), label, false,
+                        static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_block_sparse_attn(const svg_shape* shape, const void* q, const void* k, const void* v, const void* qp,
+                                 const void* kp, const void* vp, void* o, void* op, const int8_t* label, int32_t a1,
+                                 int32_t a2, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v, o, qp, kp, vp, op})) != SVG_OK) return st;
+  if (label == nullptr) return fail(SVG_ERR_INVALID_ARG, "label is NULL");
+  if (a1 < 1 || a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a1 and a2 must be >= 1");
+  const int L = shape->N * shape->F;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.qp = qp;
+  a.kp = kp;
+  a.vp = vp;
+  a.op = op;
+  a.label = label;
+  a.G0 = shape->F;
+  a.a0 = clamp_band(a1, shape->F, L);
+  a.G1 = shape->N;
+  a.a1 = clamp_band(a2, shape->N, L);
+  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_banded_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o, int32_t G,
+                           int32_t a_band, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (G < 1 || a_band < 1) return fail(SVG_ERR_INVALID_ARG, "G and a must be >= 1");
+  const int L = shape->N * shape->F;
+  if (G > L) G = L;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.label = nullptr;
+  a.G0 = G;
+  a.a0 = clamp_band(a_band, G, L);
+  a.G1 = a.G0;
+  a.a1 = a.a0;
+  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_dense_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                          int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  return svg_banded_attn(shape, q, k, v, o, shape->N * shape->F, 1, status_dev, stream);
+}
+
+size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t S) {
+  if (check_shape(shape) != SVG_OK) return 0;
+  const size_t prof = svg_profile_workspace_size(shape, S);
+  if (prof == 0) return 0;
+  const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
+  const size_t t_al = (t + 255) / 256 * 256;
+  return 4 * t_al + prof;
+}
+
+svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o, int32_t a1,
+                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
+                              size_t workspace_bytes, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (!workspace) return fail(SVG_ERR_INVALID_ARG, "workspace is NULL");
+  const size_t need = svg_sparse_3d_attn_workspace_size(shape, S);
+  if (need == 0) return fail(SVG_ERR_INVALID_ARG, "S must be in [1, 128]");
+  if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
+  const size_t t_al = (t + 255) / 256 * 256;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void *qp = w, *kp = w + t_al, *vp = w + 2 * t_al, *op = w + 3 * t_al;
+  void* prof_ws = w + 4 * t_al;
+  const size_t prof_bytes = workspace_bytes - 4 * t_al;
+  if ((st = svg_profile_heads(shape, q, k, v, a1, a2, rows, S, mse, label, prof_ws, prof_bytes, stream)) != SVG_OK)
+    return st;
+  if ((st = svg_permute_qkv(shape, q, k, v, qp, kp, vp, label, stream)) != SVG_OK) return st;
+  if ((st = svg_block_sparse_attn(shape, q, k, v, qp, kp, vp, o, op, label, a1, a2, status_dev, stream)) != SVG_OK)
+    return st;
+  return svg_unpermute(shape, op, o, label, stream);
+}
+
+}  // extern "C"

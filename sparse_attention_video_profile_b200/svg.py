@@ -1,0 +1,282 @@
+"""ctypes binding of libsvg.so, the CUDA library behind include/svg.h.
+
+Argument marshalling only: every step of the computation runs in the
+library's kernels.  PyTorch supplies device memory (outputs and workspaces
+are allocated with torch when the caller does not pass them) and the current
+CUDA stream.  Importing this module raises ImportError if libsvg.so has not
+been built -- there is no fallback path.
+
+Function names match the C entry points.  Tensors are contiguous
+[B, H, L, d] CUDA tensors (bf16 or fp32) with L = N * F in frame-major order
+(token (i, j) at row i*F + j); labels are int8 [B, H] with 0 = spatial and
+1 = temporal.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsvg.so")
+
+SVG_OK = 0
+SVG_BF16 = 0
+SVG_FP32 = 1
+SPATIAL = 0
+TEMPORAL = 1
+SVG_DEV_TIMEOUT = 0x1
+
+# Every symbol include/svg.h declares.
+EXPORTED = (
+    "svg_abi_version", "svg_status_string", "svg_last_error", "svg_attn_tile", "svg_block_list",
+    "svg_profile_workspace_size", "svg_profile_heads", "svg_permute", "svg_permute_qkv", "svg_unpermute",
+    "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
+    "svg_sparse_3d_attn",
+)
+
+
+class SvgError(RuntimeError):
+    """A libsvg entry point returned a non-OK status."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class svg_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_Z = ctypes.c_size_t
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m sparse_attention_video_profile_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "svg_abi_version": (_I, []),
+        "svg_status_string": (ctypes.c_char_p, [_I]),
+        "svg_last_error": (ctypes.c_char_p, []),
+        "svg_attn_tile": (_I, [_I, _I, _P, _P]),
+        "svg_block_list": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P]),
+        "svg_profile_workspace_size": (_Z, [_P, _I]),
+        "svg_profile_heads": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
+        "svg_permute": (_I, [_P, _P, _P, _P, _P]),
+        "svg_permute_qkv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "svg_unpermute": (_I, [_P, _P, _P, _P, _P]),
+        "svg_block_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
+        "svg_banded_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _P]),
+        "svg_dense_attn": (_I, [_P, _P, _P, _P, _P, _P, _P]),
+        "svg_sparse_3d_attn_workspace_size": (_Z, [_P, _I]),
+        "svg_sparse_3d_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P, _P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != SVG_OK:
+        name = lib.svg_status_string(status).decode()
+        msg = lib.svg_last_error().decode()
+        raise SvgError(status, f"{name}: {msg}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SVG_BF16
+    if t.dtype == torch.float32:
+        return SVG_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def make_shape(x: torch.Tensor, N: int, F: int, scale: float = 0.0) -> svg_shape:
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, L, d] tensor")
+    B, H, L, d = x.shape
+    if L != N * F:
+        raise ValueError(f"L = {L} but N*F = {N * F}")
+    return svg_shape(B, H, N, F, d, _dtype_code(x), float(scale))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _same(ref: torch.Tensor, *ts: torch.Tensor):
+    for t in ts:
+        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("q, k, v (and outputs) must share shape, dtype and device")
+
+
+# ------------------------------------------------------------------ host-only
+
+def svg_abi_version() -> int:
+    return int(lib.svg_abi_version())
+
+
+def svg_attn_tile(dtype: int, d: int):
+    bq, bk = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.svg_attn_tile(dtype, d, ctypes.byref(bq), ctypes.byref(bk)))
+    return bq.value, bk.value
+
+
+def svg_block_list(L: int, G: int, a: int, Bq: int, Bk: int):
+    """(kb_lo, kb_hi, full_lo, full_hi) int32 numpy arrays, one entry per query tile."""
+    nq = -(-L // Bq)
+    arrs = [np.zeros(nq, dtype=np.int32) for _ in range(4)]
+    _check(lib.svg_block_list(L, G, a, Bq, Bk, *(a_.ctypes.data_as(ctypes.c_void_p) for a_ in arrs)))
+    return tuple(arrs)
+
+
+def svg_profile_workspace_size(shape: svg_shape, S: int) -> int:
+    return int(lib.svg_profile_workspace_size(ctypes.byref(shape), S))
+
+
+def svg_sparse_3d_attn_workspace_size(shape: svg_shape, S: int) -> int:
+    return int(lib.svg_sparse_3d_attn_workspace_size(ctypes.byref(shape), S))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ device calls
+
+def svg_profile_heads(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, mse=None, label=None,
+                      workspace=None, scale: float = 0.0, stream=None):
+    """Online profiling.  Returns (mse [B,H,2] f32, label [B,H] int8) on q's device."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if rows.dtype != torch.int32 or rows.device != q.device:
+        raise ValueError("rows must be an int32 tensor on q's device")
+    S = rows.numel()
+    if mse is None:
+        mse = torch.empty(shape.B, shape.H, 2, dtype=torch.float32, device=q.device)
+    if label is None:
+        label = torch.empty(shape.B, shape.H, dtype=torch.int8, device=q.device)
+    need = svg_profile_workspace_size(shape, S)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check(lib.svg_profile_heads(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), a1, a2, _ptr(rows), S, _ptr(mse),
+                                 _ptr(label), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return mse, label
+
+
+def svg_permute(x, N: int, F: int, label=None, *, out=None, stream=None):
+    shape = make_shape(x, N, F)
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib.svg_permute(ctypes.byref(shape), _ptr(x), _ptr(out), _ptr(label), _stream(stream)))
+    return out
+
+
+def svg_permute_qkv(q, k, v, N: int, F: int, label=None, *, out: Optional[Sequence] = None, stream=None):
+    _same(q, k, v)
+    shape = make_shape(q, N, F)
+    qp, kp, vp = out if out is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    _check(lib.svg_permute_qkv(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp),
+                               _ptr(label), _stream(stream)))
+    return qp, kp, vp
+
+
+def svg_unpermute(xp, N: int, F: int, label=None, *, out=None, stream=None):
+    shape = make_shape(xp, N, F)
+    if out is None:
+        out = torch.empty_like(xp)
+    _check(lib.svg_unpermute(ctypes.byref(shape), _ptr(xp), _ptr(out), _ptr(label), _stream(stream)))
+    return out
+
+
+def svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N: int, F: int, a1: int, a2: int, *, o=None, op=None,
+                          status=None, scale: float = 0.0, stream=None):
+    """Returns (o, op): spatial heads' output in o, temporal heads' in op."""
+    _same(q, k, v, qp, kp, vp)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if op is None:
+        op = torch.empty_like(q)
+    _check(lib.svg_block_sparse_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp),
+                                     _ptr(o), _ptr(op), _ptr(label), a1, a2, _ptr(status), _stream(stream)))
+    return o, op
+
+
+def svg_banded_attn(q, k, v, N: int, F: int, G: int, a: int, *, o=None, status=None, scale: float = 0.0,
+                    stream=None):
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib.svg_banded_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), G, a, _ptr(status),
+                               _stream(stream)))
+    return o
+
+
+def svg_dense_attn(q, k, v, N: int, F: int, *, o=None, status=None, scale: float = 0.0, stream=None):
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib.svg_dense_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(status),
+                              _stream(stream)))
+    return o
+
+
+def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, o=None, mse=None,
+                       label=None, workspace=None, status=None, scale: float = 0.0, stream=None):
+    """One whole sparse 3D-attention call.  Returns (o, mse, label)."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    S = rows.numel()
+    if o is None:
+        o = torch.empty_like(q)
+    if mse is None:
+        mse = torch.empty(shape.B, shape.H, 2, dtype=torch.float32, device=q.device)
+    if label is None:
+        label = torch.empty(shape.B, shape.H, dtype=torch.int8, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(svg_sparse_3d_attn_workspace_size(shape, S), q.device)
+    _check(lib.svg_sparse_3d_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), a1, a2, _ptr(rows), S,
+                                  _ptr(mse), _ptr(label), _ptr(workspace), workspace.numel(), _ptr(status),
+                                  _stream(stream)))
+    return o, mse, label
+
+
+class SparseAttention3D:
+    """A reusable sparse 3D-attention call for one video shape: keeps its
+    workspace between calls (profile -> permute -> attention -> unpermute)."""
+
+    def __init__(self, N: int, F: int, a1: int, a2: int, scale: float = 0.0):
+        self.N, self.F, self.a1, self.a2, self.scale = N, F, a1, a2, scale
+        self._ws = None
+
+    def __call__(self, q, k, v, rows, *, o=None, mse=None, label=None, status=None, stream=None):
+        shape = make_shape(q, self.N, self.F, self.scale)
+        need = svg_sparse_3d_attn_workspace_size(shape, rows.numel())
+        if self._ws is None or self._ws.numel() < need or self._ws.device != q.device:
+            self._ws = alloc_workspace(need, q.device)
+        return svg_sparse_3d_attn(q, k, v, self.N, self.F, self.a1, self.a2, rows, o=o, mse=mse, label=label,
+                                  workspace=self._ws, status=status, scale=self.scale, stream=stream)

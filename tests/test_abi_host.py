@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+* libsvg.so loads and exports every function include/svg.h declares;
+* svg_block_list (the block schedule the attention kernel walks) equals the
+  oracle's brute-force tile classification of the explicit mask, bit for bit;
+* argument validation rejects bad calls before anything is enqueued.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from sparse_attention_video_profile_b200 import svg
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "svg.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:SVG_API\s+)?(?:const\s+)?\w+\**\s+\**(svg_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert len(names) >= 15
+    assert sorted(svg.EXPORTED) == names
+    for n in names:
+        assert hasattr(svg.lib, n), n
+
+
+def test_version_and_status_strings():
+    assert svg.svg_abi_version() == 1
+    assert svg.lib.svg_status_string(0) == b"SVG_OK"
+    assert svg.lib.svg_status_string(5) == b"SVG_ERR_WORKSPACE"
+    assert svg.lib.svg_status_string(99) == b"SVG_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("L,G,a", [(256, 64, 1), (2048, 256, 2), (2048, 8, 16), (700, 33, 3), (517, 50, 2),
+                                   (300, 7, 100), (129, 129, 1), (1000, 1000, 1), (4000, 13, 40)])
+@pytest.mark.parametrize("tile", [(128, 128), (64, 128), (128, 64), (256, 128)])
+def test_block_list_matches_bruteforce(L, G, a, tile):
+    Bq, Bk = tile
+    kb_lo, kb_hi, f_lo, f_hi = svg.svg_block_list(L, G, a, Bq, Bk)
+    active, full = oracle.block_list(oracle.banded_mask(L, G, a), Bq, Bk)
+    for qb in range(active.shape[0]):
+        got_a = np.zeros(active.shape[1], bool)
+        got_a[kb_lo[qb]:kb_hi[qb]] = True
+        got_f = np.zeros(full.shape[1], bool)
+        got_f[f_lo[qb]:f_hi[qb]] = True
+        np.testing.assert_array_equal(got_a, active[qb])
+        np.testing.assert_array_equal(got_f, full[qb])
+
+
+def test_block_list_kernel_tile_on_video_shapes():
+    """At the attention kernel's own tile size, for the spatial band and the
+    token-major temporal band of the two video-model shapes."""
+    Bq, Bk = svg.svg_attn_tile(svg.SVG_BF16, 128)
+    assert (Bq, Bk) == (128, 128)
+    for (N, F, a1, a2) in ((13, 1350, 3, 181), (33, 3600, 3, 281)):
+        L = N * F
+        for (G, a) in ((F, a1), (N, a2)):
+            kb_lo, kb_hi, f_lo, f_hi = svg.svg_block_list(L, G, a, Bq, Bk)
+            # brute force on a sample of query tiles (rows of the explicit mask)
+            for qb in np.linspace(0, len(kb_lo) - 1, 9).astype(int):
+                rows = np.arange(qb * Bq, min(L, (qb + 1) * Bq))
+                m = oracle.banded_mask(L, G, a, rows)
+                nk = -(-L // Bk)
+                act = np.array([m[:, kb * Bk:(kb + 1) * Bk].any() for kb in range(nk)])
+                ful = np.array([m[:, kb * Bk:(kb + 1) * Bk].all() for kb in range(nk)])
+                assert set(np.nonzero(act)[0]) == set(range(kb_lo[qb], kb_hi[qb]))
+                assert set(np.nonzero(ful)[0]) == set(range(f_lo[qb], f_hi[qb]))
+
+
+def _shape(B=1, H=2, N=4, F=64, d=64, dtype=svg.SVG_BF16):
+    return svg.svg_shape(B, H, N, F, d, dtype, 0.0)
+
+
+def test_validation_rejects_bad_arguments():
+    s = _shape(d=96)
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    st = svg.lib.svg_permute(ctypes.byref(s), p, ctypes.c_void_p(2 << 20), None, None)
+    assert st == 2  # SVG_ERR_UNSUPPORTED (bf16 d = 96)
+    assert b"d in {64, 128}" in svg.lib.svg_last_error()
+    s = _shape()
+    assert svg.lib.svg_permute(ctypes.byref(s), None, p, None, None) == 1
+    assert svg.lib.svg_permute(ctypes.byref(s), ctypes.c_void_p((1 << 20) + 8), p, None, None) == 1  # misaligned
+    assert svg.lib.svg_permute(ctypes.byref(s), p, p, None, None) == 1  # in place
+    bad = _shape(N=0)
+    assert svg.lib.svg_dense_attn(ctypes.byref(bad), p, p, p, p, None, None) == 1
+    assert svg.lib.svg_block_sparse_attn(ctypes.byref(s), p, p, p, p, p, p, p, p, None, 1, 1, None, None) == 1
+    assert svg.lib.svg_block_sparse_attn(ctypes.byref(s), p, p, p, p, p, p, p, p, p, 0, 1, None, None) == 1
+    assert svg.lib.svg_banded_attn(ctypes.byref(s), p, p, p, p, 0, 1, None, None) == 1
+    ws = ctypes.c_void_p(1 << 24)
+    assert svg.lib.svg_profile_heads(ctypes.byref(s), p, p, p, 1, 1, p, 0, p, p, ws, 1 << 30, None) == 1  # S = 0
+    assert svg.lib.svg_profile_heads(ctypes.byref(s), p, p, p, 1, 1, p, 129, p, p, ws, 1 << 30, None) == 1
+    assert svg.lib.svg_profile_heads(ctypes.byref(s), p, p, p, 1, 1, p, 32, p, p, ws, 16, None) == 5  # workspace
+    assert svg.lib.svg_block_list(0, 1, 1, 1, 1, p, p, p, p) == 1
+
+
+def test_workspace_sizes():
+    s = _shape(B=1, H=24, N=33, F=3600, d=128)
+    prof = svg.svg_profile_workspace_size(s, 128)
+    assert prof > 0 and prof % 256 == 0
+    t = 24 * 33 * 3600 * 128 * 2
+    assert svg.svg_sparse_3d_attn_workspace_size(s, 128) == 4 * t + prof
+    assert svg.svg_profile_workspace_size(s, 0) == 0
+    assert svg.svg_profile_workspace_size(s, 129) == 0
+    f = _shape(dtype=svg.SVG_FP32, d=32)
+    assert svg.svg_profile_workspace_size(f, 32) > 0

@@ -1,0 +1,309 @@
+"""GPU parity: every CUDA entry point against the fp64 oracle.
+
+Tolerances (outputs compared element by element with the oracle run on the
+very same, already-rounded inputs):
+  bf16 inputs, fp32 accumulation, bf16 output: max-abs 2e-2 and relative L2
+      1e-2.
+  fp32 inputs and outputs (CUDA-core fp32 arithmetic): max-abs 1e-4 and
+      relative L2 1e-5.  fp32 accumulation over at most a few thousand
+      terms of magnitude <= 1 stays well inside these.
+Data movement (permute / unpermute) and labels are bit-exact.  Labels are
+compared on heads whose oracle MSE gap exceeds 1e-3 relative.  Profiling MSEs
+are compared as root-mean-square distances: by the triangle inequality
+|sqrt(mse_gpu) - sqrt(mse_oracle)| is at most the RMS error of the two
+outputs it compares, which the attention tolerance bounds by about 1e-2 for
+bf16 (1e-5 for fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_video_profile_b200 import svg, synth
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+TOL = {torch.bfloat16: (2e-2, 1e-2), torch.float32: (1e-4, 1e-5)}
+RMS_TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-5}
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def assert_close(got, ref, dtype, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    max_abs = float(np.max(np.abs(got - ref)))
+    rel_l2 = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    ta, tr = TOL[dtype]
+    assert max_abs <= ta and rel_l2 <= tr, f"{what}: max_abs {max_abs:.3e} rel_l2 {rel_l2:.3e}"
+
+
+def rand_qkv(B, H, L, d, dtype, seed, scale=1.0):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return tuple((torch.randn(B, H, L, d, generator=g, device=DEV) * scale).to(dtype) for _ in range(3))
+
+
+def sync_ok(status=None):
+    torch.cuda.synchronize()
+    if status is not None:
+        assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+
+# ---------------------------------------------------------------- permute
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 64), (torch.bfloat16, 128), (torch.float32, 32)])
+@pytest.mark.parametrize("N,F", [(5, 37), (13, 1350), (1, 9), (7, 1)])
+def test_permute_unpermute_bit_exact(dtype, d, N, F):
+    B, H = 2, 3
+    L = N * F
+    x, _, _ = rand_qkv(B, H, L, d, dtype, 1)
+    label = torch.tensor([[1, 0, 1], [0, 1, 1]], dtype=torch.int8, device=DEV)
+    sentinel = torch.full_like(x, 7.0)
+    xp = svg.svg_permute(x, N, F, label, out=sentinel.clone())
+    back = svg.svg_unpermute(xp, N, F, label, out=sentinel.clone())
+    torch.cuda.synchronize()
+    xn, xpn, bn = f64(x), f64(xp), f64(back)
+    ref = oracle.permute(xn, N, F)
+    for b in range(B):
+        for h in range(H):
+            if label[b, h] == 1:
+                np.testing.assert_array_equal(xpn[b, h], ref[b, h])
+                np.testing.assert_array_equal(bn[b, h], xn[b, h])
+            else:  # untouched
+                assert np.all(xpn[b, h] == 7.0) and np.all(bn[b, h] == 7.0)
+    # label = NULL: every head; the three-tensor launch gives the same bytes
+    allp = svg.svg_permute(x, N, F, None)
+    qp, kp, vp = svg.svg_permute_qkv(x, x, x, N, F, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(f64(allp), ref)
+    for t in (qp, kp, vp):
+        assert torch.equal(t, allp)
+
+
+# ---------------------------------------------------------------- attention kernel
+
+BAND_CASES = [  # (N, F, G, a)
+    (3, 100, 100, 1),   # spatial-like, ragged L = 300 (one full + one partial CTA)
+    (3, 100, 3, 5),     # temporal-like small groups
+    (4, 64, 64, 1),     # the tiny shape
+    (8, 256, 256, 2),   # the small shape, several key tiles
+    (8, 256, 8, 16),
+    (5, 61, 1, 1),      # diagonal only
+    (5, 61, 7, 4),
+    (2, 40, 80, 1),     # L = 80 < one tile
+    (6, 300, 6, 1000),  # band wider than the sequence -> dense
+]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("case", BAND_CASES, ids=lambda c: "N{}F{}G{}a{}".format(*c))
+def test_banded_attention_bf16(d, case):
+    N, F, G, a = case
+    L = N * F
+    q, k, v = rand_qkv(1, 2, L, d, torch.bfloat16, 2)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_banded_attn(q, k, v, N, F, G, a, status=status)
+    sync_ok(status)
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    mask = oracle.banded_mask(L, min(G, L), a)
+    for h in range(2):
+        ref = oracle.attention(qn[0, h], kn[0, h], vn[0, h], mask)
+        assert_close(f64(o)[0, h], ref, torch.bfloat16, f"head {h}")
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("case", BAND_CASES[:6], ids=lambda c: "N{}F{}G{}a{}".format(*c))
+def test_banded_attention_fp32(d, case):
+    N, F, G, a = case
+    L = N * F
+    q, k, v = rand_qkv(1, 2, L, d, torch.float32, 3)
+    o = svg.svg_banded_attn(q, k, v, N, F, G, a)
+    sync_ok()
+    mask = oracle.banded_mask(L, min(G, L), a)
+    for h in range(2):
+        ref = oracle.attention(f64(q)[0, h], f64(k)[0, h], f64(v)[0, h], mask)
+        assert_close(f64(o)[0, h], ref, torch.float32, f"head {h}")
+
+
+def test_diagonal_band_copies_values_exactly():
+    """G = 1, a = 1 keeps only the self pair: softmax weight exactly 1, so the
+    output is V itself, bit for bit."""
+    q, k, v = rand_qkv(2, 3, 777, 128, torch.bfloat16, 4)
+    o = svg.svg_banded_attn(q, k, v, 7, 111, 1, 1)
+    sync_ok()
+    assert torch.equal(o, v)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 64), (torch.bfloat16, 128), (torch.float32, 64)])
+def test_dense_attention(dtype, d):
+    N, F = 4, 77
+    q, k, v = rand_qkv(1, 2, N * F, d, dtype, 5)
+    o = svg.svg_dense_attn(q, k, v, N, F)
+    sync_ok()
+    ref = oracle.dense_attention(f64(q), f64(k), f64(v))
+    assert_close(f64(o), ref, dtype, "dense")
+
+
+def test_large_logits_stay_finite():
+    """Scores spanning hundreds of units exercise the lazy-rescale path."""
+    q, k, v = rand_qkv(1, 2, 1024, 64, torch.bfloat16, 6, scale=4.0)
+    o = svg.svg_banded_attn(q, k, v, 4, 256, 256, 2)
+    sync_ok()
+    mask = oracle.banded_mask(1024, 256, 2)
+    for h in range(2):
+        ref = oracle.attention(f64(q)[0, h], f64(k)[0, h], f64(v)[0, h], mask)
+        assert_close(f64(o)[0, h], ref, torch.bfloat16, f"head {h}")
+
+
+# ---------------------------------------------------------------- labelled heads
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_attn_with_labels(d):
+    N, F, a1, a2 = 6, 90, 2, 7
+    L = N * F
+    q, k, v = rand_qkv(2, 2, L, d, torch.bfloat16, 7)
+    label = torch.tensor([[0, 1], [1, 0]], dtype=torch.int8, device=DEV)
+    qp, kp, vp = svg.svg_permute_qkv(q, k, v, N, F, label)
+    o, op = svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, a1, a2)
+    out = svg.svg_unpermute(op, N, F, label, out=o)
+    sync_ok()
+    ref = oracle.sparse_attention(f64(q), f64(k), f64(v), label.cpu().numpy(), N, F, a1, a2)
+    assert_close(f64(out), ref, torch.bfloat16, "block-sparse")
+
+
+# ---------------------------------------------------------------- profiling
+
+def check_profile(mse, label, ref_mse, ref_label, dtype):
+    mse = mse.cpu().numpy().astype(np.float64)
+    label = label.cpu().numpy()
+    gap = np.abs(ref_mse[..., 0] - ref_mse[..., 1]) / np.maximum(ref_mse.max(-1), 1e-300)
+    decided = gap > 1e-3
+    np.testing.assert_array_equal(label[decided], ref_label[decided])
+    assert np.all(np.isin(label, [0, 1]))
+    dist = np.abs(np.sqrt(mse) - np.sqrt(ref_mse))
+    assert dist.max() <= RMS_TOL[dtype], f"rms distance {dist.max():.3e}"
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_profile_synthetic(name):
+    wl = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(wl, seed=0, device=DEV)
+    rows_np = synth.sample_rows(wl.L, wl.S, 0)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    mse, label = svg.svg_profile_heads(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows)
+    sync_ok()
+    ref_mse, ref_label = oracle.profile_heads(f64(q), f64(k), f64(v), wl.N, wl.F, wl.a1, wl.a2, rows_np)
+    check_profile(mse, label, ref_mse, ref_label, q.dtype)
+    np.testing.assert_array_equal(label.cpu().numpy(), synth.head_kinds(wl, 0))
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 64), (torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("S", [1, 17, 64, 128])
+def test_profile_random(dtype, d, S):
+    N, F, a1, a2 = 5, 133, 2, 11
+    L = N * F
+    q, k, v = rand_qkv(1, 3, L, d, dtype, 8 + S)
+    rows_np = np.sort(np.random.default_rng(S).choice(L, S, replace=False)).astype(np.int32)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    mse, label = svg.svg_profile_heads(q, k, v, N, F, a1, a2, rows)
+    sync_ok()
+    ref_mse, ref_label = oracle.profile_heads(f64(q), f64(k), f64(v), N, F, a1, a2, rows_np)
+    check_profile(mse, label, ref_mse, ref_label, dtype)
+
+
+def test_profile_special_cases_and_determinism():
+    N, F = 4, 200
+    q, k, v = rand_qkv(1, 2, N * F, 64, torch.bfloat16, 9)
+    rows = torch.tensor([0, 5, 199, 200, 401, 799], dtype=torch.int32, device=DEV)
+    mse, label = svg.svg_profile_heads(q, k, v, N, F, N, 3, rows)  # spatial band = all keys
+    sync_ok()
+    assert torch.all(mse[..., 0] == 0) and torch.all(mse[..., 1] > 0) and torch.all(label == 0)
+    mse, label = svg.svg_profile_heads(q, k, v, N, F, 1, F, rows)  # temporal band = all keys
+    sync_ok()
+    assert torch.all(mse[..., 1] == 0) and torch.all(mse[..., 0] > 0) and torch.all(label == 1)
+    a = svg.svg_profile_heads(q, k, v, N, F, 2, 5, rows)[0].clone()
+    b = svg.svg_profile_heads(q, k, v, N, F, 2, 5, rows)[0].clone()
+    sync_ok()
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- whole call
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_sparse_3d_attn_end_to_end(name):
+    wl = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(wl, seed=1, device=DEV)
+    rows_np = synth.sample_rows(wl.L, wl.S, 1)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, mse, label = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, status=status)
+    sync_ok(status)
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    ref_mse, ref_label = oracle.profile_heads(qn, kn, vn, wl.N, wl.F, wl.a1, wl.a2, rows_np)
+    check_profile(mse, label, ref_mse, ref_label, q.dtype)
+    ref = oracle.sparse_attention(qn, kn, vn, label.cpu().numpy(), wl.N, wl.F, wl.a1, wl.a2)
+    assert_close(f64(o), ref, q.dtype, name)
+
+
+def test_full_bands_equal_dense():
+    wl = synth.WORKLOADS["small"]
+    q, k, v = synth.make_qkv(wl, seed=2, device=DEV)
+    rows = torch.from_numpy(synth.sample_rows(wl.L, wl.S, 2)).to(DEV)
+    dense = svg.svg_dense_attn(q, k, v, wl.N, wl.F)
+    ref = oracle.dense_attention(f64(q), f64(k), f64(v))
+    for a1, a2 in ((wl.N, wl.a2), (wl.a1, wl.F), (wl.N, wl.F)):
+        o, _, label = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, a1, a2, rows)
+        sync_ok()
+        assert_close(f64(o), ref, q.dtype, f"a1={a1} a2={a2}")
+        full = (label.cpu().numpy() == 0) if a1 == wl.N else (label.cpu().numpy() == 1)
+        if a1 == wl.N and a2 == wl.F:
+            full[:] = True
+        # heads whose band covers every key run the same tiles as dense: same bits
+        dn, on = dense.cpu(), o.cpu()
+        for b, h in zip(*np.nonzero(full)):
+            if (label[b, h] == 0 and a1 == wl.N):
+                assert torch.equal(on[b, h], dn[b, h])
+    assert_close(f64(dense), ref, q.dtype, "dense")
+
+
+# ---------------------------------------------------------------- video-model shapes
+
+def sampled_rows(wl, n_extra=40, seed=0):
+    """Rows at frame, tile and sequence boundaries plus random ones."""
+    L, F, N = wl.L, wl.F, wl.N
+    rows = {0, 1, L - 1, L - 2, F - 1, F, 127, 128, 255, 256, (L // 256) * 256, (L // 256) * 256 - 1}
+    rows |= {i * F + j for i in (0, N // 2, N - 1) for j in (0, F - 1)}
+    rows |= set(np.random.default_rng(seed).choice(L, n_extra, replace=False).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < L))
+
+
+@pytest.mark.parametrize("name", ["cogvideox", "hunyuan"])
+def test_video_shape_sampled(name):
+    wl = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(wl, seed=0, device=DEV)
+    rows_np = synth.sample_rows(wl.L, wl.S, 0)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, mse, label = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, status=status)
+    sync_ok(status)
+    label_np = label.cpu().numpy()
+    mse_np = mse.cpu().numpy()
+    check_rows = sampled_rows(wl)
+    heads = range(wl.H) if name == "cogvideox" else range(0, wl.H, 3)
+    for h in range(wl.H):
+        qn, kn, vn = (f64(t[:, h:h + 1]) for t in (q, k, v))
+        ref_mse, ref_label = oracle.profile_heads(qn, kn, vn, wl.N, wl.F, wl.a1, wl.a2, rows_np)
+        check_profile(torch.from_numpy(mse_np[:, h:h + 1]), torch.from_numpy(label_np[:, h:h + 1]),
+                      ref_mse, ref_label, q.dtype)
+        if h in heads:
+            ref = oracle.sparse_attention(qn, kn, vn, label_np[:, h:h + 1], wl.N, wl.F, wl.a1, wl.a2,
+                                          rows=check_rows)
+            got = f64(o[:, h:h + 1, torch.from_numpy(check_rows).to(DEV)])
+            assert_close(got, ref, q.dtype, f"{name} head {h}")
+    assert set(np.unique(label_np)) <= {0, 1}

@@ -1,0 +1,424 @@
+"""Benchmark: one sparse 3D-attention call per step on the HunyuanVideo-shaped
+workload (B=1, H=24, N=33 latent frames x F=3600 tokens, L=118800, d=128,
+bf16, a1=3 / a2=281 for ~15% mask density, S=128 sampled profiling rows).
+
+A step is the whole hot path through the C ABI: online profiling ->
+token-major permutation of temporal heads -> block-sparse attention ->
+inverse permutation.  Inputs are synthetic (seeded generator with the
+workload's shape and head structure) and resident in HBM; they are larger
+than L2 (3 x 730 MB), so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  value = ms per call for the whole job
+(max-over-ranks step time divided by the calls all ranks made; each rank runs
+its own independent call, so scaling is weak).  N > 1 runs under torchrun.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_video_profile_b200 import metrics, synth  # noqa: E402
+
+METRIC = "ms per sparse 3D-attention call; effective TFLOPS vs bf16 peak; speedup vs dense"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus):
+    if n_gpus <= 1 and "WORLD_SIZE" not in os.environ:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's SM clock and throttle reasons while
+    the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            ident = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "200"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"], "samples": 0}
+        # median over the samples taken under load (the top half of clocks
+        # excludes idle gaps at the edges of the window)
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+
+def head_f64(wl, q, k, v, h=0):
+    """fp64 host copies of one head's q, k, v ([1, 1, L, d]) for the oracle."""
+    return tuple(t[:, h:h + 1].to("cpu", torch.float64).numpy() for t in (q, k, v))
+
+
+def oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=16, n_attn_rows=16, seed=0):
+    """Times the fp64 oracle, as it stands, on a bounded sample of one call
+    and scales the time linearly to the whole call: profiling of
+    n_prof_rows sampled rows of one head (the call profiles S rows of every
+    head) and masked attention of n_attn_rows query rows of one head (the
+    call computes all L rows of every head).
+    Returns (ms_per_call_estimate, description, seconds_spent)."""
+    import oracle  # test infrastructure: only this baseline leg runs it
+    rng = np.random.default_rng(seed)
+    qn, kn, vn = qkv64
+    prof_rows = np.sort(rng.choice(rows_np, n_prof_rows, replace=False))
+    t0 = time.perf_counter()
+    oracle.profile_heads(qn, kn, vn, wl.N, wl.F, wl.a1, wl.a2, prof_rows)
+    t_prof = time.perf_counter() - t0
+    sample = np.sort(rng.choice(wl.L, n_attn_rows, replace=False))
+    t0 = time.perf_counter()
+    oracle.sparse_attention(qn, kn, vn, labels[:, :1], wl.N, wl.F, wl.a1, wl.a2, rows=sample)
+    t_attn = time.perf_counter() - t0
+    heads = wl.B * wl.H
+    per_call_s = t_prof * (wl.S / n_prof_rows) * heads + t_attn * (wl.L / n_attn_rows) * heads
+    desc = (f"fp64 oracle: profiling of {n_prof_rows} of the {wl.S} sampled rows and masked attention of "
+            f"{n_attn_rows} of the {wl.L} query rows, both on 1 of the {heads} heads, scaled linearly to the call")
+    return per_call_s * 1e3, desc, t_prof + t_attn
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args, wl, rank, world):
+    """The oracle on the host cores, on a bounded sample of the workload per
+    step (rank 0 only)."""
+    if rank != 0:
+        return
+    q, k, v = synth.make_qkv(wl, seed=0, device="cpu")
+    rows_np = synth.sample_rows(wl.L, wl.S, 0)
+    labels = synth.head_kinds(wl, 0)
+    qkv64 = head_f64(wl, q, k, v)
+    del q, k, v
+    for w in range(args.warmup):
+        oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=4, n_attn_rows=4, seed=1000 + w)
+    ests, secs = [], 0.0
+    desc = ""
+    for s in range(args.steps):
+        ms, desc, sec = oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=32, n_attn_rows=64, seed=s)
+        ests.append(ms)
+        secs += sec
+    value = float(np.mean(ests))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "ms/call", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, world),
+        "cpu_baseline": {"value": value, "unit": "ms/call", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": desc + " (per step)"},
+        "e2e": {"value": value, "unit": "ms/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl, world):
+    return {"workload": f"HunyuanVideo-shaped {wl.name}: B={wl.B} H={wl.H} N={wl.N} F={wl.F} L={wl.L} d={wl.d}",
+            "B": wl.B, "H": wl.H, "N": wl.N, "F": wl.F, "L": wl.L, "d": wl.d, "a1": wl.a1, "a2": wl.a2, "S": wl.S,
+            "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (Q,K,V 3 x 730 MB); no flush"}
+
+
+def run_ours(args, wl, rank, world, local):
+    from sparse_attention_video_profile_b200 import svg
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    q, k, v = synth.make_qkv(wl, seed=rank, device=dev)
+    rows_np = synth.sample_rows(wl.L, wl.S, rank)
+    rows = torch.from_numpy(rows_np).to(dev)
+    N, F = wl.N, wl.F
+    o = torch.empty_like(q)
+    qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
+    mse = torch.empty(wl.B, wl.H, 2, dtype=torch.float32, device=dev)
+    label = torch.empty(wl.B, wl.H, dtype=torch.int8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    shape = svg.make_shape(q, N, F)
+    prof_ws = svg.alloc_workspace(svg.svg_profile_workspace_size(shape, wl.S), dev)
+
+    names = ("profile", "permute", "attn", "unpermute")
+
+    def new_events():
+        return {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
+
+    def step(e=None):
+        if e:
+            e["profile"][0].record(stream)
+        svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws)
+        if e:
+            e["profile"][1].record(stream)
+            e["permute"][0].record(stream)
+        svg.svg_permute_qkv(q, k, v, N, F, label, out=(qp, kp, vp))
+        if e:
+            e["permute"][1].record(stream)
+            e["attn"][0].record(stream)
+        svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status)
+        if e:
+            e["attn"][1].record(stream)
+            e["unpermute"][0].record(stream)
+        svg.svg_unpermute(op, N, F, label, out=o)
+        if e:
+            e["unpermute"][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    labels_np = label.cpu().numpy()
+    n_temporal = int(labels_np.sum())
+    pairs = metrics.effective_pairs(N, F, wl.a1, wl.a2, labels_np)
+    flops = metrics.attention_flops(pairs, wl.d)
+
+    step_events = [new_events() for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for e in step_events:
+            step(e)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    acc = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in step_events) for n in names}
+    step_ms_local = t_start.elapsed_time(t_end) / args.steps
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status word {int(status.item())} after the timed region")
+    step_ms = max_over_ranks(step_ms_local, world)
+    kern_ms = {n: acc[n] / args.steps for n in acc}
+    value = step_ms / world  # ms per call, whole job (world calls per step)
+
+    # dense reference on the same inputs (speedup vs dense), outside the timed region
+    dense_ms = None
+    if not args.no_dense:
+        od = torch.empty_like(q)
+        svg.svg_dense_attn(q, k, v, N, F, o=od)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 2
+        a.record(stream)
+        for _ in range(reps):
+            svg.svg_dense_attn(q, k, v, N, F, o=od)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = a.elapsed_time(b) / reps
+        del od
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        mseh = torch.empty(mse.shape, dtype=mse.dtype, pin_memory=True)
+        labh = torch.empty(label.shape, dtype=label.dtype, pin_memory=True)
+        rowsh = torch.from_numpy(rows_np).pin_memory()
+        call = svg.SparseAttention3D(N, F, wl.a1, wl.a2)
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        rowsd = torch.empty_like(rows)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            rowsd.copy_(rowsh, non_blocking=True)
+            od_, msed, labd = call(qd, kd, vd, rowsd, o=o, mse=mse, label=label)
+            oh.copy_(od_, non_blocking=True)
+            mseh.copy_(msed, non_blocking=True)
+            labh.copy_(labd, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world) / world
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, rowsh))
+        d2h = sum(t.numel() * t.element_size() for t in (oh, mseh, labh))
+        e2e = {"value": e2e_ms, "unit": "ms/call", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del qh, kh, vh, oh, qd, kd, vd
+
+    peaks, peak_kind = load_peaks()
+    attn_tflops = flops / (kern_ms["attn"] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    perm_bytes = 2 * 3 * n_temporal * wl.B * wl.L * wl.d * 2
+    unperm_bytes = 2 * n_temporal * wl.B * wl.L * wl.d * 2
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qkv64 = head_f64(wl, q, k, v)
+        ms, desc, _ = oracle_sample(wl, qkv64, rows_np, labels_np, n_prof_rows=wl.S, n_attn_rows=1024)
+        cpu = {"value": ms, "unit": "ms/call", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "ms/call", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl, world),
+        "effective_tflops": attn_tflops, "effective_tflops_call": flops / (step_ms * 1e-3) / 1e12,
+        "frac_bf16_peak": attn_tflops / peak,
+        "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
+        "dense_ms": dense_ms,
+        "kernel_ms": kern_ms,
+        "permute_gbs": perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal else None,
+        "unpermute_gbs": unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal else None,
+        "temporal_heads": n_temporal,
+        "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "traffic": args.traffic,
+                     "algorithmic_work": f"{flops:.4e} flops/launch = 4*d*unmasked pairs"},
+        "hbm_peak_gbs": hbm,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": 5 * args.steps,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="hunyuan")
+    ap.add_argument("--density", type=float, default=None, help="HunyuanVideo sweep density (0.05..0.5)")
+    ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per attention launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[args.workload]
+    if args.density is not None:
+        a1, a2 = synth.HUNYUAN_SWEEP[args.density]
+        wl = wl.with_bands(a1, a2)
+    if args.heads is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, H=args.heads, name=f"{wl.name}-{args.heads}heads")
+    if args.impl == "reference":
+        # the oracle runs on host cores; no process group is needed: rank 0
+        # works, the other ranks exit at once
+        run_reference(args, wl, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("no CUDA device: the benchmark measures the CUDA path only")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, wl, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -292,9 +292,12 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       for (int c = 0; c < 64; ++c) {
         const float p0 = ex2_approx(fmaf(s[2 * c], sl2, nb));
         const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, nb));
-        ls0 += p0;
-        ls1 += p1;
-        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+        const uint32_t pp = pack_bf16x2(p0, p1);
+        // The row sum uses the same bf16-rounded weights the P V product
+        // sees, so each output row is an exact convex combination of V rows.
+        ls0 += bf16lo_f32(pp);
+        ls1 += bf16hi_f32(pp);
+        pk[c >> 5][c & 31] = pp;
       }
       l += ls0 + ls1;
       __syncwarp();

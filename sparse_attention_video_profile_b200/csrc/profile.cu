@@ -238,25 +238,25 @@ __global__ void __launch_bounds__(128) profile_mma_kernel(const ProfParams p) {
         const float m_new = fmaxf(m_old, mx);
         const float alpha = (m_new == m_old) ? 1.f : ex2_approx((m_old - m_new) * sl2);
         const float nb = (m_new == -INFINITY) ? 0.f : -m_new * sl2;
-        float ps = 0.f;
         float pv[16];
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          pv[cc] = ex2_approx(fmaf(sv[cc], sl2, nb));  // -inf -> 0
-          ps += pv[cc];
-        }
-        l[vv][h] = l[vv][h] * alpha + ps;
+        for (int cc = 0; cc < 16; ++cc) pv[cc] = ex2_approx(fmaf(sv[cc], sl2, nb));  // -inf -> 0
         m[vv][h] = m_new;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
           o[vv][nt][2 * h] *= alpha;
           o[vv][nt][2 * h + 1] *= alpha;
         }
+        float ps = 0.f;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           pf[ks][h] = pack_bf16x2(pv[4 * ks + 0], pv[4 * ks + 1]);      // keys 16ks + 2tq (+1)
           pf[ks][2 + h] = pack_bf16x2(pv[4 * ks + 2], pv[4 * ks + 3]);  // keys 16ks + 8 + 2tq (+1)
+          // sum the bf16-rounded weights the P V product uses
+          ps += bf16lo_f32(pf[ks][h]) + bf16hi_f32(pf[ks][h]) + bf16lo_f32(pf[ks][2 + h]) +
+                bf16hi_f32(pf[ks][2 + h]);
         }
+        l[vv][h] = l[vv][h] * alpha + ps;
       }
       // O_v += P_v V over this warp's 64 output columns
 #pragma unroll

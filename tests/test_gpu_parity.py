@@ -151,8 +151,10 @@ def test_dense_attention(dtype, d):
 
 
 def test_large_logits_stay_finite():
-    """Scores spanning hundreds of units exercise the lazy-rescale path."""
-    q, k, v = rand_qkv(1, 2, 1024, 64, torch.bfloat16, 6, scale=4.0)
+    """Scores spanning hundreds of units exercise the lazy-rescale path (Q and
+    K scaled up; V keeps unit scale so the bf16 output grid stays fine)."""
+    q, k, _ = rand_qkv(1, 2, 1024, 64, torch.bfloat16, 6, scale=4.0)
+    _, _, v = rand_qkv(1, 2, 1024, 64, torch.bfloat16, 6)
     o = svg.svg_banded_attn(q, k, v, 4, 256, 256, 2)
     sync_ok()
     mask = oracle.banded_mask(1024, 256, 2)

@@ -32,6 +32,19 @@ sys.path.insert(0, ROOT)
 from sparse_attention_video_profile_b200 import metrics, synth  # noqa: E402
 
 METRIC = "ms per sparse 3D-attention call; effective TFLOPS vs bf16 peak; speedup vs dense"
+
+# DRAM bytes (read + write) per full-size launch of the attention kernel, from
+# an ncu capture (profiles/attn_sm100_hunyuan.md), keyed by the sha256 prefix
+# of the kernel sources it was taken on.  Any other source revision reports
+# traffic as null until it is captured again.
+NCU_TRAFFIC = {("0fc4f35ca5f50d0f", "87c6d3d476966093"): 2.809e9}
+
+
+def attn_source_key():
+    import hashlib
+    csrc = os.path.join(ROOT, "sparse_attention_video_profile_b200", "csrc")
+    return tuple(hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()[:16]
+                 for f in ("attn_sm100.cu", "sm100.cuh"))
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -367,7 +380,8 @@ def run_ours(args, wl, rank, world, local):
         "temporal_heads": n_temporal,
         "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "traffic": args.traffic,
+                     "traffic": args.traffic if args.traffic is not None else (
+                         NCU_TRAFFIC.get(attn_source_key()) if wl.name == "hunyuan" else None),
                      "algorithmic_work": f"{flops:.4e} flops/launch = 4*d*unmasked pairs"},
         "hbm_peak_gbs": hbm,
         "clocks": clocks.summary(),

@@ -159,6 +159,39 @@ SVG_API svg_status svg_profile_heads(const svg_shape* shape, const void* q, cons
                              int8_t* label, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * svg_profile_heads_noalloc -- svg_profile_heads for callers that cannot
+ * allocate device memory.  The pages describe nothing like it; it exists for
+ * integration only.
+ *
+ * Who needs it: code that is handed only its input and output tensors and
+ * has no allocator of its own (a plugin inside a host framework that owns
+ * all device memory), and loops that must never call cudaMalloc, because
+ * that call can synchronise the whole device at an unpredictable moment.
+ * Instead of a caller workspace, this variant uses a fixed scratch array of
+ * SVG_PROFILE_NOALLOC_SCRATCH_BYTES that lives in the library's device image.
+ * Every GPU on which the library is used holds that array until the process
+ * exits.  It computes the same quantities as svg_profile_heads.  When the
+ * default key split would not fit the array, it splits the keys into fewer
+ * chunks, so results can differ from svg_profile_heads in the last bits.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (which also loads the library's kernels on that device) and remembers it.
+ * Make that first call before any stream capture on that device.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents.  Nothing in it needs to start at zero, because each call
+ * writes every byte it later reads.  Calls whose kernels overlap on the GPU,
+ * for example on two streams, race on the array: serialise them.
+ * Limits: shapes whose partial results cannot fit the array even with one
+ * key chunk (bf16), or at all (fp32, which always uses one chunk), return
+ * SVG_ERR_WORKSPACE before anything is enqueued.  The call allocates and
+ * frees nothing.  Arguments are otherwise as for svg_profile_heads.
+ */
+#define SVG_PROFILE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, const void* q, const void* k,
+                                             const void* v, int32_t a1, int32_t a2, const int32_t* rows,
+                                             int32_t S, float* mse, int8_t* label, void* stream);
+
+/*
  * svg_permute -- the layout transformation ("Sparse VideoGen ...", Abstract;
  * SVG2 explainer 2.A) of one tensor: for every head with label[b,h] ==
  * SVG_TEMPORAL, xp[b,h, j*N+i, :] = x[b,h, i*F+j, :].  Rows of spatial heads

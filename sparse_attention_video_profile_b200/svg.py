@@ -34,7 +34,7 @@ EXPORTED = (
     "svg_abi_version", "svg_status_string", "svg_last_error", "svg_attn_tile", "svg_block_list",
     "svg_profile_workspace_size", "svg_profile_heads", "svg_permute", "svg_permute_qkv", "svg_unpermute",
     "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
-    "svg_sparse_3d_attn",
+    "svg_sparse_3d_attn", "svg_profile_heads_noalloc",
 )
 
 
@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "svg_dense_attn": (_I, [_P, _P, _P, _P, _P, _P, _P]),
         "svg_sparse_3d_attn_workspace_size": (_Z, [_P, _I]),
         "svg_sparse_3d_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P, _P]),
+        "svg_profile_heads_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -182,6 +183,25 @@ def svg_profile_heads(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Ten
         workspace = alloc_workspace(need, q.device)
     _check(lib.svg_profile_heads(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), a1, a2, _ptr(rows), S, _ptr(mse),
                                  _ptr(label), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return mse, label
+
+
+def svg_profile_heads_noalloc(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, mse=None,
+                              label=None, scale: float = 0.0, stream=None):
+    """Online profiling without a workspace, for callers that cannot allocate
+    device memory.  The library's fixed scratch array stands in for the
+    workspace (see include/svg.h).  mse and label should be passed in by
+    such callers; they are allocated here only for convenience."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if rows.dtype != torch.int32 or rows.device != q.device:
+        raise ValueError("rows must be an int32 tensor on q's device")
+    if mse is None:
+        mse = torch.empty(shape.B, shape.H, 2, dtype=torch.float32, device=q.device)
+    if label is None:
+        label = torch.empty(shape.B, shape.H, dtype=torch.int8, device=q.device)
+    _check(lib.svg_profile_heads_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), a1, a2, _ptr(rows),
+                                         rows.numel(), _ptr(mse), _ptr(label), _stream(stream)))
     return mse, label
 
 

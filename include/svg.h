@@ -83,6 +83,7 @@ typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
 
 /* Bits of the device status word. */
 #define SVG_DEV_TIMEOUT 0x1u  /* a pipeline wait exceeded its bound; outputs invalid */
+#define SVG_DEV_RANGE 0x2u    /* profiling: in-band weights underflowed (see svg_profile_heads) */
 
 typedef struct svg_shape {
   int32_t B, H, N, F, d;
@@ -143,6 +144,12 @@ SVG_API size_t svg_profile_workspace_size(const svg_shape* shape, int32_t S);
  *   mse[b,h,1] = mean over S*d of (O_t - O_dense)^2,
  *   label[b,h] = SVG_TEMPORAL if mse[b,h,1] < mse[b,h,0] else SVG_SPATIAL.
  * The reduction order is fixed, so repeated calls give identical bits.
+ * The three softmaxes of a row share one reference (the row's running max
+ * over all keys), so every key needs one exponential.  If a row's in-band
+ * logits all lie more than about 126 / (scale * log2(e)) below its largest
+ * logit (about 990 raw units for d = 128), their weights underflow.  That
+ * case, like a device-side wait that ran out, is reported rather than
+ * returned: every label is set to -1 and every MSE to NaN.
  *
  * q, k, v   device, [B,H,L,d] frame-major, dtype of shape.
  * rows      device, int32 [S], each in [0, L) (duplicates allowed), shared by

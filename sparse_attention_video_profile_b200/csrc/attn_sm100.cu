@@ -14,7 +14,8 @@
 // in memory -- and masks elementwise only in tiles a row's band does not
 // fully cover.
 //
-// One CTA = 256 query rows = two 128-row Q tiles sharing every K/V tile:
+// One CTA = 256 query rows = two 128-row Q tiles sharing every K/V tile, 12
+// warps (warps 10-11 only hold their share of the register split):
 //   warp 8      TMA producer: Q tiles once, then K_k / V_k into a ring of
 //               128-key slots (128-byte swizzle, OOB rows zero-filled);
 //   warp 9      one thread issues tcgen05.mma: S_i = Q_i K^T into TMEM, and
@@ -26,7 +27,8 @@
 //               only when the max grew by more than 2^8 (lazy rescaling).
 // The MMA order S_0, S_1, then per key tile {P_0 V, S_0 <- next}, {P_1 V,
 // S_1 <- next} lets the tensor core work on one Q tile while the other's
-// softmax runs.
+// softmax runs.  (Two issuing threads, one per tile, measured slower: the
+// finely interleaved MMAs of two accumulators ran below this order's rate.)
 // TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D,256+2D).
 #include <cuda_bf16.h>
 
@@ -34,6 +36,9 @@
 #include "sm100.cuh"
 
 namespace svg {
+
+svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D);
+
 namespace {
 
 struct AttnParams {
@@ -57,15 +62,27 @@ struct Cfg {
   static constexpr int HALVES = D / 64;   // 128-byte swizzle rows hold 64 bf16
   static constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = BK * D * 2;
-  static constexpr int NS = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int NS = (D == 128) ? 5 : 8;  // K/V ring slots (fills shared memory)
   static constexpr int SMEM_Q = 2 * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_Q + NS * TILE_BYTES;
   static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;  // barriers + alignment slack
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;     // 3 warpgroups: softmax 0, softmax 1, producer/MMA
+  // Register split (setmaxnreg): launched at 168 per thread, the producer/MMA
+  // warpgroup gives back down to 88 and the two softmax warpgroups grow to
+  // 208.  384 * 168 = 256 * 208 + 128 * 88 = 64512, the block's launch total.
+  static constexpr int REGS_SOFTMAX = 208;
+  static constexpr int REGS_CONTROL = 88;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t col_s(int i) { return 128u * i; }
   static constexpr uint32_t col_o(int i) { return 256u + D * i; }
 };
+
+// Pairs (of 8) per softmax row chunk whose exponentials use the FMA-pipe
+// polynomial instead of the MUFU ex2 unit.
+#ifndef SVG_EXP_POLY_PAIRS
+#define SVG_EXP_POLY_PAIRS 2
+#endif
+constexpr int kExpPoly = SVG_EXP_POLY_PAIRS;
 
 __device__ __forceinline__ void record_timeout(const AttnParams& p, volatile int* abort_flag) {
   *abort_flag = 1;
@@ -79,7 +96,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(384, 1) attn_sm100_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -136,9 +153,14 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   const int nk = (hi_cta + C::BK - 1) / C::BK - kt0;
   const bool run = (*abort_flag == 0);
 
-  if (run && warp == 8) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0) {
+  // Every warp takes part in the register split before anything else, so the
+  // increase can always be satisfied; each role's code sits inside the branch
+  // that set its register budget.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CONTROL));
+    if (run && warp == 8 && lane == 0) {
+      // ------------------------------------------------ TMA producer
+      {
       const CUtensorMap* tq = lab ? &p.tm_qp : &p.tm_q;
       const CUtensorMap* tk = lab ? &p.tm_kp : &p.tm_k;
       const CUtensorMap* tv = lab ? &p.tm_vp : &p.tm_v;
@@ -166,30 +188,32 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, row, bh);
       }
     }
-  } else if (run && warp == 9) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (run && warp == 9 && lane == 0) {
+      // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_u32(sQ);
       const uint32_t ring_base = smem_u32(sRing);
+      // Descriptors are built once; offsets go into the start-address field
+      // (address >> 4 in the low bits; every operand lies below 256 KB).
+      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(ring_base, 16, 1024);
+      const uint64_t dv = smem_desc_sw128(ring_base, C::HALF_BYTES, 1024);
       auto issue_qk = [&](int i, int slot) {
-        const uint32_t a0 = q_base + i * C::TILE_BYTES;
-        const uint32_t b0 = ring_base + slot * C::TILE_BYTES;
+        const uint64_t a = dq + static_cast<uint64_t>((i * C::TILE_BYTES) >> 4);
+        const uint64_t b = dk + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::HALF_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + C::col_s(i), smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024),
-                  idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
+          umma_ss(tmem + C::col_s(i), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bar_s[i]);
       };
       auto issue_pv = [&](int i, int slot, bool acc) {
-        const uint32_t b0 = ring_base + slot * C::TILE_BYTES;
+        const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
-                  smem_desc_sw128(b0 + kk * 16 * 128, C::HALF_BYTES, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8, b + static_cast<uint64_t>((kk * 16 * 128) >> 4),
+                  idesc_pv, (acc || kk > 0) ? 1u : 0u);
         umma_commit(&bar_o[i]);
       };
       bool ok = mbar_wait(bar_q, 0, p.wait_ns) && mbar_wait(&bar_full[0], 0, p.wait_ns);
@@ -209,6 +233,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           if (!ok) break;
           tc_fence_after();
           issue_pv(i, slotV, k > 0);
+          // V_k is free once both tiles' P V products have read it.
+          if (i == 1) umma_commit(&bar_empty[slotV]);
           if (has_next) {
             if (i == 0) {
               ok = mbar_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
@@ -219,12 +245,13 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           }
         }
         if (!ok) break;
-        umma_commit(&bar_empty[slotV]);
         if (has_next) umma_commit(&bar_empty[slotK]);
       }
       if (!ok) record_timeout(p, abort_flag);
     }
-  } else if (run && warp < 8) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+    if (run) {
     // ------------------------------------------------ softmax / epilogue
     const int i = warp >> 2;
     const int quad = warp & 3;
@@ -268,15 +295,15 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           if (y < lo_r || y >= hi_r) s[c] = -INFINITY;
         }
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
+      for (int c = 8; c < 128; c += 8) {
+        mx0 = fmax3f(mx0, s[c], s[c + 1]);
+        mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
+        mx2 = fmax3f(mx2, s[c + 4], s[c + 5]);
+        mx3 = fmax3f(mx3, s[c + 6], s[c + 7]);
       }
-      const float m_new = fmaxf(fmaxf(m_used, fmaxf(mx0, mx1)), fmaxf(mx2, mx3));
+      const float m_new = fmax3f(m_used, fmax3f(mx0, mx1, mx2), mx3);
       float alpha = 1.f;
       bool resc = false;
       if (m_new > m_used + p.lazy_th) {  // false while both are -inf
@@ -286,20 +313,28 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       }
       l *= alpha;
       const float nb = (m_used == -INFINITY) ? 0.f : -m_used * sl2;
+      const float2 sl2x2 = make_float2(sl2, sl2), nb2 = make_float2(nb, nb);
       uint32_t pk[2][32];
-      float ls0 = 0.f, ls1 = 0.f;
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, nb));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, nb));
-        const uint32_t pp = pack_bf16x2(p0, p1);
+        const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
+        float2 pr;
+        if ((c & 7) < kExpPoly) {  // a fixed share of the pairs on the FMA pipe
+          pr = exp2_poly2(x);
+        } else {
+          pr.x = ex2_approx(x.x);
+          pr.y = ex2_approx(x.y);
+        }
+        const uint32_t pp = pack_bf16x2(pr.x, pr.y);
         // The row sum uses the same bf16-rounded weights the P V product
         // sees, so each output row is an exact convex combination of V rows.
-        ls0 += bf16lo_f32(pp);
-        ls1 += bf16hi_f32(pp);
+        const float2 pw = make_float2(bf16lo_f32(pp), bf16hi_f32(pp));
+        if (c & 1) acc1 = __fadd2_rn(acc1, pw);
+        else acc0 = __fadd2_rn(acc0, pw);
         pk[c >> 5][c & 31] = pp;
       }
-      l += ls0 + ls1;
+      l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
       __syncwarp();
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
@@ -349,6 +384,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     } else {
       record_timeout(p, abort_flag);
     }
+    }
   }
 
   tc_fence_before();
@@ -362,37 +398,6 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
 
 // ---------------------------------------------------------------- host side
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// [BH, L, D] bf16, box = 64 elements x 128 rows x 1 head, 128-byte swizzle.
-svg_status make_map(CUtensorMap* map, const void* base, int BH, int L, int D) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (enc == nullptr) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-  return SVG_OK;
-}
-
 template <int D>
 svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   using C = Cfg<D>;
@@ -400,13 +405,13 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   memset(&p, 0, sizeof(p));
   const int BH = a.B * a.H;
   svg_status st;
-  if ((st = make_map(&p.tm_q, a.q, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_map(&p.tm_k, a.k, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_map(&p.tm_v, a.v, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_q, a.q, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_k, a.k, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_v, a.v, BH, a.L, D)) != SVG_OK) return st;
   const bool perm = a.label != nullptr;
-  if ((st = make_map(&p.tm_qp, perm ? a.qp : a.q, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_map(&p.tm_kp, perm ? a.kp : a.k, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_map(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_qp, perm ? a.qp : a.q, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_kp, perm ? a.kp : a.k, BH, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.op = static_cast<__nv_bfloat16*>(perm ? a.op : a.o);
   p.label = a.label;
@@ -435,6 +440,37 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [BH, L, D] bf16, box = 64 elements x 128 rows x 1 head, 128-byte swizzle.
+svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SVG_OK;
+}
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream) {
   switch (a.d) {

@@ -58,16 +58,27 @@ struct ProfileLayout {
   int S_pad;      // sampled rows rounded up to the row-block of the kernel
   int n_chunks;   // key chunks per head
   int chunk;      // keys per chunk (multiple of 64)
-  size_t o_bytes;   // partial outputs  [BH][n_chunks][3][S_pad][d] f32
-  size_t ml_bytes;  // partial max/sum  [BH][n_chunks][3][S_pad][2] f32
+  size_t o_bytes;     // partial outputs  [BH][n_chunks][3][S_pad][d] f32
+  size_t ml_bytes;    // partial max/sum  [BH][n_chunks][3][S_pad][2] f32
+  size_t part_bytes;  // per-row squared-difference sums [BH][S_pad][2] f64
   size_t total;
 };
 
-bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out);
+// Workspace layout of the profiling kernels.  max_chunks > 0 caps the number
+// of key chunks (fewer chunks need less workspace); fp32 always uses one.
+bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks = 0);
 
 svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
                           const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
                           float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
                           cudaStream_t stream);
+
+// bf16 stage 1 of profiling on the tensor cores (profile_sm100.cu).
+svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const void* q, const void* k,
+                                const void* v, int a1, int a2, const int32_t* rows, int S, float* ws_o,
+                                float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream);
+
+// A zeroed per-device status word for kernels whose entry point takes none.
+svg_status internal_status_word(int** out, cudaStream_t stream);
 
 }  // namespace svg

@@ -8,16 +8,15 @@
 // (O_t) -- and the head is labelled by the lower of
 //   mse_s = mean (O_s - O_d)^2,  mse_t = mean (O_t - O_d)^2.
 //
-// Stage 1 (profile_mma_kernel, bf16): the key axis is split into chunks so
-// that B*H*chunks*row-blocks CTAs cover the GPU; each CTA streams its chunk
-// of K and V once through shared memory (cp.async double buffer, XOR
-// swizzle) and keeps, per sampled row, three online-softmax states (max,
-// sum, unnormalised output) updated from one shared Q K^T tile.  The
-// products use mma.sync m16n8k16 bf16 -> fp32.  Partial (max, sum, output)
-// triples go to the workspace.
-// Stage 2 (profile_combine_kernel): per head, merges the chunk partials in a
-// fixed order, forms O_d, O_s, O_t, and reduces the squared differences in
-// fp64 with a fixed tree -- so repeated calls return identical bits.
+// Stage 1, bf16 (profile_sm100.cu): the key axis is split into chunks, one
+// CTA per (chunk, head) holds all sampled rows as one 128-row tile, computes
+// S = Q K^T on the tensor cores and keeps the three online-softmax states,
+// with P V products into three TMEM accumulators.  Partial (max, sum,
+// unnormalised output) triples go to the workspace.
+// Stage 2 (profile_combine_rows_kernel, one block per sampled row and head;
+// profile_finalize_kernel, one block per head): merges the chunk partials in
+// a fixed order, forms O_d, O_s, O_t, and reduces the squared differences in
+// fp64 with fixed trees -- so repeated calls return identical bits.
 // fp32 inputs use profile_simt_kernel (one warp per row, all keys) for stage
 // 1 and the same stage 2.
 #include <cuda_bf16.h>
@@ -28,7 +27,7 @@
 namespace svg {
 namespace {
 
-constexpr int kKT = 64;  // keys per tile in stage 1
+constexpr int kKT = 128;  // keys per tile of the bf16 stage 1
 
 struct ProfParams {
   const void* q;
@@ -41,260 +40,6 @@ struct ProfParams {
   int a1, a2;
   float sl2;
 };
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Byte offset of 16-byte chunk c of row `row` in a [rows][D] bf16 tile whose
-// chunks are XOR-swizzled by the row's low three bits (conflict-free
-// ldmatrix on both the row and the transposed access).
-template <int D>
-__device__ __forceinline__ uint32_t swz(int row, int c) {
-  return static_cast<uint32_t>(row * D * 2 + ((c ^ (row & 7)) << 4));
-}
-
-template <int D>
-struct ProfCfg {
-  static constexpr int DS = D / 64;      // warps sharing a row block, one per 64 output columns
-  static constexpr int RG = 4 / DS;      // 16-row blocks per CTA
-  static constexpr int ROWS = 16 * RG;   // sampled rows per CTA
-  static constexpr int TILE = kKT * D * 2;
-  static constexpr int SMEM = ROWS * D * 2 + 4 * TILE + 4 * kKT * 4;
-};
-
-template <int D>
-__global__ void __launch_bounds__(128) profile_mma_kernel(const ProfParams p) {
-  using C = ProfCfg<D>;
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::ROWS * D * 2;  // [2][TILE]
-  uint8_t* sV = sK + 2 * C::TILE;        // [2][TILE]
-  int* sIY = reinterpret_cast<int*>(sV + 2 * C::TILE);  // [2][kKT]
-  int* sJY = sIY + 2 * kKT;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rg = warp / C::DS, ds = warp % C::DS;
-  const int row_base = blockIdx.x * C::ROWS;  // first sampled-row index of this CTA
-  const int chunk = blockIdx.y;
-  const int bh = blockIdx.z;
-  const size_t hoff = static_cast<size_t>(bh) * p.L * D;
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q) + hoff;
-  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(p.k) + hoff;
-  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(p.v) + hoff;
-  const int y_begin = chunk * p.chunk;
-  const int y_end = min(p.L, y_begin + p.chunk);
-  const int ntiles = (y_end - y_begin + kKT - 1) / kKT;
-
-  // gather the CTA's sampled query rows (padding rows repeat the last row)
-  for (int e = tid; e < C::ROWS * CPR; e += 128) {
-    const int r = e / CPR, c = e % CPR;
-    const int s = min(row_base + r, p.S - 1);
-    const int x = min(max(p.rows[s], 0), p.L - 1);
-    cp_async16(smem_u32(sQ) + swz<D>(r, c), q + static_cast<size_t>(x) * D + c * 8, true);
-  }
-  auto load_tile = [&](int t, int stage) {
-    const int y0 = y_begin + t * kKT;
-    const uint32_t kb = smem_u32(sK + stage * C::TILE), vb = smem_u32(sV + stage * C::TILE);
-    for (int e = tid; e < kKT * CPR; e += 128) {
-      const int r = e / CPR, c = e % CPR;
-      const int y = y0 + r;
-      const bool ok = y < p.L;
-      const size_t off = static_cast<size_t>(ok ? y : 0) * D + c * 8;
-      cp_async16(kb + swz<D>(r, c), k + off, ok);
-      cp_async16(vb + swz<D>(r, c), v + off, ok);
-    }
-    if (tid < kKT) {
-      const int y = y0 + tid;
-      sIY[stage * kKT + tid] = y / p.F;
-      sJY[stage * kKT + tid] = y % p.F;
-    }
-  };
-  load_tile(0, 0);
-  cp_async_commit();
-
-  // the two rows this thread owns in the mma fragments
-  const int g = lane >> 2, tq = lane & 3;
-  int ir[2], jr[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int s = min(row_base + rg * 16 + g + 8 * h, p.S - 1);
-    const int x = min(max(p.rows[s], 0), p.L - 1);
-    ir[h] = x / p.F;
-    jr[h] = x % p.F;
-  }
-
-  float m[3][2], l[3][2], o[3][8][4];
-#pragma unroll
-  for (int vv = 0; vv < 3; ++vv)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      m[vv][h] = -INFINITY;
-      l[vv][h] = 0.f;
-    }
-#pragma unroll
-  for (int vv = 0; vv < 3; ++vv)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[vv][nt][e] = 0.f;
-
-  uint32_t qf[D / 16][4];
-  const float sl2 = p.sl2;
-
-  for (int t = 0; t < ntiles; ++t) {
-    const int stage = t & 1;
-    if (t + 1 < ntiles) {
-      load_tile(t + 1, stage ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (t == 0) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        ldsm_x4(qf[kk], smem_u32(sQ) + swz<D>(rg * 16 + (lane & 15), kk * 2 + (lane >> 4)));
-    }
-    const uint32_t kb = smem_u32(sK + stage * C::TILE), vb = smem_u32(sV + stage * C::TILE);
-    // S = Q K^T for this warp's 16 rows x 64 keys
-    float sacc[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t b[4];
-        ldsm_x4(b, kb + swz<D>(np * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)));
-        mma_bf16(sacc[2 * np], qf[kk], b[0], b[1]);
-        mma_bf16(sacc[2 * np + 1], qf[kk], b[2], b[3]);
-      }
-    }
-    // frame / position of this thread's 16 key columns
-    const int y0 = y_begin + t * kKT;
-    int iy[16], jy[16];
-    bool in_chunk[16];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int c = nt * 8 + tq * 2 + e;
-        iy[nt * 2 + e] = sIY[stage * kKT + c];
-        jy[nt * 2 + e] = sJY[stage * kKT + c];
-        in_chunk[nt * 2 + e] = (y0 + c) < y_end;
-      }
-#pragma unroll
-    for (int vv = 0; vv < 3; ++vv) {
-      uint32_t pf[4][4];  // P as A fragments, 4 k-steps of 16 keys
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float sv[16];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int cc = nt * 2 + e;
-            bool ok = in_chunk[cc];
-            if (vv == 1) ok = ok && (abs(ir[h] - iy[cc]) < p.a1);
-            if (vv == 2) ok = ok && (abs(jr[h] - jy[cc]) < p.a2);
-            sv[cc] = ok ? sacc[nt][2 * h + e] : -INFINITY;
-            mx = fmaxf(mx, sv[cc]);
-          }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_old = m[vv][h];
-        const float m_new = fmaxf(m_old, mx);
-        const float alpha = (m_new == m_old) ? 1.f : ex2_approx((m_old - m_new) * sl2);
-        const float nb = (m_new == -INFINITY) ? 0.f : -m_new * sl2;
-        float pv[16];
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) pv[cc] = ex2_approx(fmaf(sv[cc], sl2, nb));  // -inf -> 0
-        m[vv][h] = m_new;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          o[vv][nt][2 * h] *= alpha;
-          o[vv][nt][2 * h + 1] *= alpha;
-        }
-        float ps = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          pf[ks][h] = pack_bf16x2(pv[4 * ks + 0], pv[4 * ks + 1]);      // keys 16ks + 2tq (+1)
-          pf[ks][2 + h] = pack_bf16x2(pv[4 * ks + 2], pv[4 * ks + 3]);  // keys 16ks + 8 + 2tq (+1)
-          // sum the bf16-rounded weights the P V product uses
-          ps += bf16lo_f32(pf[ks][h]) + bf16hi_f32(pf[ks][h]) + bf16lo_f32(pf[ks][2 + h]) +
-                bf16hi_f32(pf[ks][2 + h]);
-        }
-        l[vv][h] = l[vv][h] * alpha + ps;
-      }
-      // O_v += P_v V over this warp's 64 output columns
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t b[4];
-          ldsm_x4_t(b, vb + swz<D>(ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), ds * 8 + np * 2 + (lane >> 4)));
-          mma_bf16(o[vv][2 * np], pf[ks], b[0], b[1]);
-          mma_bf16(o[vv][2 * np + 1], pf[ks], b[2], b[3]);
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  // write partials
-#pragma unroll
-  for (int vv = 0; vv < 3; ++vv) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float ls = l[vv][h];
-      ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-      ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-      const int s = row_base + rg * 16 + g + 8 * h;
-      const size_t base = ((static_cast<size_t>(bh) * p.nch + chunk) * 3 + vv) * p.S_pad + s;
-      float* orow = p.ws_o + base * D + ds * 64;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-        *reinterpret_cast<float2*>(orow + nt * 8 + tq * 2) = make_float2(o[vv][nt][2 * h], o[vv][nt][2 * h + 1]);
-      if (tq == 0 && ds == 0) {
-        const float mm = m[vv][h];
-        p.ws_ml[base * 2 + 0] = (mm == -INFINITY) ? -INFINITY : mm * sl2;
-        p.ws_ml[base * 2 + 1] = ls;
-      }
-    }
-  }
-}
 
 // fp32 stage 1: one warp per (head, sampled row), all keys, chunk count 1.
 template <int D>
@@ -382,18 +127,19 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
   }
 }
 
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 128;
 
-// Stage 2: merge chunk partials, form O_d / O_s / O_t, reduce the MSEs.
+// Stage 2a: one block per (sampled row, head).  Merges the chunk partials of
+// the three outputs of that row (thread c owns column c) and reduces the
+// row's squared differences (O_s - O_d)^2 and (O_t - O_d)^2 over d in a fixed
+// order, in fp64.
 __global__ void __launch_bounds__(kCombineThreads)
-    profile_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int S, int S_pad, int D,
-                           int nch, float* __restrict__ mse, int8_t* __restrict__ label) {
-  __shared__ double red[2][kCombineThreads];
-  const int bh = blockIdx.x;
-  double acc_s = 0.0, acc_t = 0.0;
-  const int total = S * D;
-  for (int e = threadIdx.x; e < total; e += kCombineThreads) {
-    const int s = e / D, c = e % D;
+    profile_combine_rows_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int S_pad, int D,
+                                int nch, double* __restrict__ part) {
+  __shared__ double red[2][kCombineThreads / 32];
+  const int s = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  double dsq = 0.0, dtq = 0.0;
+  if (c < D) {
     float ov[3];
 #pragma unroll
     for (int vv = 0; vv < 3; ++vv) {
@@ -417,11 +163,45 @@ __global__ void __launch_bounds__(kCombineThreads)
     }
     const double dsp = static_cast<double>(ov[1]) - ov[0];
     const double dtp = static_cast<double>(ov[2]) - ov[0];
-    acc_s += dsp * dsp;
-    acc_t += dtp * dtp;
+    dsq = dsp * dsp;
+    dtq = dtp * dtp;
   }
-  red[0][threadIdx.x] = acc_s;
-  red[1][threadIdx.x] = acc_t;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    dsq += __shfl_xor_sync(0xffffffffu, dsq, off);
+    dtq += __shfl_xor_sync(0xffffffffu, dtq, off);
+  }
+  if ((c & 31) == 0) {
+    red[0][c >> 5] = dsq;
+    red[1][c >> 5] = dtq;
+  }
+  __syncthreads();
+  if (c == 0) {
+    double a = 0.0, b = 0.0;
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) {
+      a += red[0][w];
+      b += red[1][w];
+    }
+    part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 0] = a;
+    part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 1] = b;
+  }
+}
+
+// Stage 2b: per head, sums the S rows' partial sums in a fixed order and
+// writes the two MSEs and the label.
+__global__ void __launch_bounds__(kCombineThreads)
+    profile_finalize_kernel(const double* __restrict__ part, int S, int S_pad, int D, float* __restrict__ mse,
+                            int8_t* __restrict__ label, const int* __restrict__ status) {
+  __shared__ double red[2][kCombineThreads];
+  const int bh = blockIdx.x;
+  double a = 0.0, b = 0.0;
+  for (int s = threadIdx.x; s < S; s += kCombineThreads) {
+    a += part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 0];
+    b += part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 1];
+  }
+  red[0][threadIdx.x] = a;
+  red[1][threadIdx.x] = b;
   __syncthreads();
   for (int w = kCombineThreads / 2; w > 0; w >>= 1) {
     if (threadIdx.x < w) {
@@ -431,22 +211,13 @@ __global__ void __launch_bounds__(kCombineThreads)
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    const double n = static_cast<double>(total);
+    const double n = static_cast<double>(S) * D;
     const float ms = static_cast<float>(red[0][0] / n), mt = static_cast<float>(red[1][0] / n);
-    mse[bh * 2 + 0] = ms;
-    mse[bh * 2 + 1] = mt;
-    label[bh] = (mt < ms) ? SVG_TEMPORAL : SVG_SPATIAL;
+    const bool failed = status != nullptr && (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE));
+    mse[bh * 2 + 0] = failed ? __int_as_float(0x7fc00000) : ms;
+    mse[bh * 2 + 1] = failed ? __int_as_float(0x7fc00000) : mt;
+    label[bh] = failed ? static_cast<int8_t>(-1) : ((mt < ms) ? SVG_TEMPORAL : SVG_SPATIAL);
   }
-}
-
-template <int D>
-svg_status launch_stage1_bf16(const ProfParams& p, cudaStream_t stream) {
-  using C = ProfCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(profile_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(profile smem)");
-  dim3 grid(p.S_pad / C::ROWS, p.nch, p.BH);
-  profile_mma_kernel<D><<<grid, 128, C::SMEM, stream>>>(p);
-  return cuda_check(cudaGetLastError(), "profile launch");
 }
 
 template <int D>
@@ -456,15 +227,12 @@ svg_status launch_stage1_f32(const ProfParams& p, cudaStream_t stream) {
   return cuda_check(cudaGetLastError(), "fp32 profile launch");
 }
 
-int row_block(int d, int dtype) {
-  if (dtype == SVG_FP32) return 4;
-  return d == 128 ? ProfCfg<128>::ROWS : ProfCfg<64>::ROWS;
-}
+int row_block(int /*d*/, int dtype) { return dtype == SVG_FP32 ? 4 : 128; }
 
 }  // namespace
 
-bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out) {
-  if (B < 1 || H < 1 || L < 1 || S < 1 || S > 128) return false;
+bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks) {
+  if (B < 1 || H < 1 || L < 1 || S < 1 || S > 128 || max_chunks < 0) return false;
   const int rb = row_block(d, dtype);
   ProfileLayout lay{};
   lay.S_pad = (S + rb - 1) / rb * rb;
@@ -472,13 +240,22 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
     lay.n_chunks = 1;
     lay.chunk = L;
   } else {
-    // Aim for about four CTAs per SM over all heads and row blocks, with at
-    // least four key tiles per chunk.
-    const long long ctas_per_chunk = static_cast<long long>(B) * H * (lay.S_pad / rb);
-    long long nch = (148LL * 4 + ctas_per_chunk - 1) / ctas_per_chunk;
-    const long long max_nch = (L + 4 * kKT - 1) / (4 * kKT);
-    if (nch > max_nch) nch = max_nch;
-    if (nch < 1) nch = 1;
+    // One CTA per (chunk, head), one CTA per SM.  Pick the chunk count that
+    // minimises waves x (key tiles per chunk + a fixed per-CTA cost of about
+    // two tiles for setup, Q gather and the partials' store).
+    const long long heads = static_cast<long long>(B) * H;
+    const long long tiles = (L + kKT - 1) / kKT;
+    long long limit = tiles;
+    if (max_chunks > 0 && limit > max_chunks) limit = max_chunks;
+    long long nch = 1, best = -1;
+    for (long long c = 1; c <= limit && c <= 4096; ++c) {
+      const long long waves = (heads * c + 147) / 148;
+      const long long cost = waves * ((tiles + c - 1) / c + 2);
+      if (best < 0 || cost < best) {
+        best = cost;
+        nch = c;
+      }
+    }
     long long chunk = (L + nch - 1) / nch;
     chunk = (chunk + kKT - 1) / kKT * kKT;
     lay.chunk = static_cast<int>(chunk);
@@ -487,7 +264,8 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
   const size_t rows_total = static_cast<size_t>(B) * H * lay.n_chunks * 3 * lay.S_pad;
   lay.o_bytes = (rows_total * d * sizeof(float) + 255) / 256 * 256;
   lay.ml_bytes = (rows_total * 2 * sizeof(float) + 255) / 256 * 256;
-  lay.total = lay.o_bytes + lay.ml_bytes;
+  lay.part_bytes = (static_cast<size_t>(B) * H * lay.S_pad * 2 * sizeof(double) + 255) / 256 * 256;
+  lay.total = lay.o_bytes + lay.ml_bytes + lay.part_bytes;
   *out = lay;
   return true;
 }
@@ -515,11 +293,12 @@ svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float sc
   p.a2 = a2;
   p.sl2 = scale * 1.4426950408889634f;
   if (p.BH > 65535) return fail(SVG_ERR_UNSUPPORTED, "B*H = %d exceeds the grid limit", p.BH);
-  svg_status st;
+  int* status = nullptr;
+  svg_status st = internal_status_word(&status, stream);
+  if (st != SVG_OK) return st;
   if (dtype == SVG_BF16) {
-    if (d == 64) st = launch_stage1_bf16<64>(p, stream);
-    else if (d == 128) st = launch_stage1_bf16<128>(p, stream);
-    else return fail(SVG_ERR_UNSUPPORTED, "bf16 profiling supports d in {64, 128}, got %d", d);
+    st = launch_profile_sm100(p.BH, N, F, d, scale, q, k, v, a1, a2, rows, S, p.ws_o, p.ws_ml, lay.n_chunks,
+                              lay.chunk, status, stream);
   } else {
     if (d == 32) st = launch_stage1_f32<32>(p, stream);
     else if (d == 64) st = launch_stage1_f32<64>(p, stream);
@@ -527,9 +306,13 @@ svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float sc
     else return fail(SVG_ERR_UNSUPPORTED, "fp32 profiling supports d in {32, 64, 128}, got %d", d);
   }
   if (st != SVG_OK) return st;
-  profile_combine_kernel<<<p.BH, kCombineThreads, 0, stream>>>(p.ws_o, p.ws_ml, S, lay.S_pad, d, lay.n_chunks,
-                                                                mse, label);
-  return cuda_check(cudaGetLastError(), "profile combine launch");
+  double* part = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
+  profile_combine_rows_kernel<<<dim3(S, p.BH), kCombineThreads, 0, stream>>>(p.ws_o, p.ws_ml, lay.S_pad, d,
+                                                                              lay.n_chunks, part);
+  st = cuda_check(cudaGetLastError(), "profile combine launch");
+  if (st != SVG_OK) return st;
+  profile_finalize_kernel<<<p.BH, kCombineThreads, 0, stream>>>(part, S, lay.S_pad, d, mse, label, status);
+  return cuda_check(cudaGetLastError(), "profile finalize launch");
 }
 
 }  // namespace svg

@@ -76,22 +76,16 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
   constexpr size_t kMax = SVG_PROFILE_NOALLOC_SCRATCH_BYTES;
   if (lay.total > kMax) {
     // Fewer, longer key chunks need less scratch (bf16 path; fp32 uses one chunk).
-    const size_t rows_per_chunk = static_cast<size_t>(shape->B) * shape->H * 3 * lay.S_pad;
-    const size_t per_chunk = rows_per_chunk * (static_cast<size_t>(shape->d) + 2) * sizeof(float);
-    const long long fit = static_cast<long long>((kMax - 512) / per_chunk);
-    if (shape->dtype != SVG_BF16 || fit < 1)
+    ProfileLayout one;
+    profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &one, 1);
+    const size_t per_chunk = one.o_bytes + one.ml_bytes;  // bytes that scale with the chunk count
+    const long long fit = static_cast<long long>((kMax - one.part_bytes - 512) / per_chunk);
+    if (shape->dtype != SVG_BF16 || one.total > kMax || fit < 1)
       return fail(SVG_ERR_WORKSPACE,
                   "profiling this shape needs at least %zu bytes of scratch, more than the %zu-byte static "
                   "array of svg_profile_heads_noalloc; use svg_profile_heads with a workspace",
-                  shape->dtype != SVG_BF16 ? lay.total : per_chunk + 512, kMax);
-    long long chunk = (L + fit - 1) / fit;
-    chunk = (chunk + 63) / 64 * 64;
-    lay.chunk = static_cast<int>(chunk);
-    lay.n_chunks = static_cast<int>((L + chunk - 1) / chunk);
-    const size_t rows_total = rows_per_chunk * lay.n_chunks;
-    lay.o_bytes = (rows_total * shape->d * sizeof(float) + 255) / 256 * 256;
-    lay.ml_bytes = (rows_total * 2 * sizeof(float) + 255) / 256 * 256;
-    lay.total = lay.o_bytes + lay.ml_bytes;
+                  shape->dtype != SVG_BF16 ? lay.total : one.total, kMax);
+    profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay, static_cast<int>(fit));
     if (lay.total > kMax) return fail(SVG_ERR_WORKSPACE, "scratch layout does not fit the static array");
   }
   void* scratch = nullptr;

@@ -1,0 +1,465 @@
+// profile_sm100.cu -- stage 1 of online profiling on B200 tensor cores
+// ("Sparse Video-Gen", Weakness 1 answer on online profiling: every step and
+// layer, right before 3D attention; "Sparse VideoGen ...", Abstract: heads
+// are classified spatial or temporal online).
+//
+// For the S sampled query rows of one head (padded to one 128-row tile) and
+// one chunk of keys, computes three online-softmax attention states at once:
+// unmasked (d), spatial |i_x - i_y| < a1 (s) and temporal |j_x - j_y| < a2
+// (t).  Per 128-key tile:
+//   S = Q K^T                       one tcgen05.mma group into TMEM
+//   P_d, P_s (bf16) written over S  -> O_d += P_d V, O_s += P_s V
+//   P_t written over P_d once P_d V has read it -> O_t += P_t V
+// The three variants share one softmax reference, the running max over all
+// kept keys, so each key needs one exponential: P_s and P_t are P_d
+// restricted to the spatial and temporal masks (the normalisation of each
+// variant divides the reference out again).
+// The three P V products read P straight from TMEM (A-from-TMEM form).  The
+// partial (max, sum, unnormalised output) triples of every row and variant
+// go to the workspace; the combine kernels merge the chunks.
+// TMEM: S [0,128), O_d [128,128+D), O_s [128+D,128+2D), O_t [128+2D,128+3D).
+//
+// Warps 0-3: one thread per sampled row (Q gather, masks, three softmaxes,
+// epilogue).  Warp 4: TMA producer of K and V.  Warp 5: MMA issuer.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace svg {
+
+struct ProfSm100Params {
+  CUtensorMap tm_k, tm_v;  // frame-major [BH, L, D] bf16
+  const __nv_bfloat16* q;
+  const int32_t* rows;
+  float* ws_o;   // [BH][nch][3][128][D]
+  float* ws_ml;  // [BH][nch][3][128][2]  (max in log2 units, sum)
+  int BH, L, N, F, S, nch, chunk;
+  int a1, a2;
+  float sl2;
+  float lazy_th;
+  int* status;
+  uint64_t wait_ns;
+};
+
+namespace {
+
+template <int D>
+struct PCfg {
+  static constexpr int HALVES = D / 64;
+  static constexpr int HALF_BYTES = 128 * 128;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NS = (D == 128) ? 5 : 8;
+  static constexpr int SMEM_BAR = TILE_BYTES + NS * TILE_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t COL_S = 0;
+  static constexpr uint32_t col_o(int v) { return 128u + D * v; }
+};
+
+__device__ __forceinline__ bool warp_wait_p(uint64_t* bar, uint32_t parity, uint64_t limit) {
+  const bool ok = mbar_wait(bar, parity, limit);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bit c of a 128-bit mask (four 32-bit words), c a compile-time constant.
+__device__ __forceinline__ bool bit128(const uint32_t (&m)[4], int c) { return (m[c >> 5] >> (c & 31)) & 1u; }
+
+// Sets bits [lo, hi) of a 128-bit mask (0 <= lo, hi <= 128).
+__device__ __forceinline__ void set_range128(uint32_t (&m)[4], int lo, int hi) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 32);
+    if (a < b) {
+      const uint32_t hi_bits = (b >= 32) ? 0xFFFFFFFFu : ((1u << b) - 1u);
+      m[w] |= hi_bits & ~((1u << a) - 1u);
+    }
+  }
+}
+
+// Packs P = e for the keys whose mask bit is set (0 elsewhere) as bf16 pairs
+// and returns the sum of the rounded weights.
+__device__ __forceinline__ float pack_masked(const float (&e)[128], const uint32_t (&m)[4], uint32_t (&pk)[64]) {
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const float p0 = bit128(m, 2 * c) ? e[2 * c] : 0.f;
+    const float p1 = bit128(m, 2 * c + 1) ? e[2 * c + 1] : 0.f;
+    const uint32_t pp = pack_bf16x2(p0, p1);
+    const float2 pw = make_float2(bf16lo_f32(pp), bf16hi_f32(pp));
+    if (c & 1) a1 = __fadd2_rn(a1, pw);
+    else a0 = __fadd2_rn(a0, pw);
+    pk[c] = pp;
+  }
+  return (a0.x + a1.x) + (a0.y + a1.y);
+}
+
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t ov[32];
+    tmem_ld32(t_o + c * 32, ov);
+    tmem_wait_ld();
+    reg_fence32(ov);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+    tmem_st32(t_o + c * 32, ov);
+  }
+}
+
+__device__ __forceinline__ void st_p64(uint32_t taddr, const uint32_t (&pk)[64]) {
+  uint32_t a[32], b[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    a[e] = pk[e];
+    b[e] = pk[32 + e];
+  }
+  tmem_st32(taddr, a);
+  tmem_st32(taddr + 32, b);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_constant__ ProfSm100Params p) {
+  using C = PCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sRing = smem + C::TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
+  uint64_t* bar_q = bars;                       // 128 arrivals: Q gathered
+  uint64_t* bar_full = bars + 1;                // [NS]
+  uint64_t* bar_empty = bars + 1 + C::NS;       // [NS]
+  uint64_t* bar_s = bars + 1 + 2 * C::NS;       // S ready
+  uint64_t* bar_p01 = bar_s + 1;                // 128 arrivals: P_d, P_s written
+  uint64_t* bar_o01 = bar_s + 2;                // P_d V, P_s V done
+  uint64_t* bar_pt = bar_s + 3;                 // 128 arrivals: P_t written
+  uint64_t* bar_ot = bar_s + 4;                 // P_t V done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int y_begin = chunk * p.chunk;
+  const int y_end = min(p.L, y_begin + p.chunk);
+  const int kt0 = y_begin / 128;
+  const int nk = (y_end - y_begin + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = (*reinterpret_cast<volatile int*>(p.status) & SVG_DEV_TIMEOUT) ? 1 : 0;
+    mbar_init(bar_q, 128);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_p01, 128);
+    mbar_init(bar_o01, 1);
+    mbar_init(bar_pt, 128);
+    mbar_init(bar_ot, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool run = (*abort_flag == 0);
+
+  if (run && warp == 4 && lane == 0) {
+    // ------------------------------------------------ TMA producer (K, V)
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    for (int n = 0; n < 2 * nk; ++n) {
+      const int slot = n % C::NS;
+      if (!mbar_wait(&bar_empty[slot], ((n / C::NS) & 1) ^ 1, p.wait_ns)) {
+        *abort_flag = 1;
+        atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
+        break;
+      }
+      const CUtensorMap* tm = (n & 1) ? &p.tm_v : &p.tm_k;
+      mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
+#pragma unroll
+      for (int h = 0; h < C::HALVES; ++h)
+        tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64,
+                    (kt0 + (n >> 1)) * 128, bh);
+    }
+  } else if (run && warp == 5 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t ring_base = smem_u32(sRing);
+    const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dk = smem_desc_sw128(ring_base, 16, 1024);
+    const uint64_t dv = smem_desc_sw128(ring_base, C::HALF_BYTES, 1024);
+    auto pv = [&](int v, uint32_t pcol, int slot, bool acc) {
+      const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        umma_ts(tmem + C::col_o(v), tmem + pcol + kk * 8, b + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                (acc || kk > 0) ? 1u : 0u);
+    };
+    bool ok = mbar_wait(bar_q, 0, p.wait_ns);
+    for (int k = 0; ok && k < nk; ++k) {
+      const int nK = 2 * k, nV = 2 * k + 1;
+      const int slotK = nK % C::NS, slotV = nV % C::NS;
+      ok = mbar_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const uint64_t b = dk + static_cast<uint64_t>((slotK * C::TILE_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
+          umma_ss(tmem + C::COL_S, dq + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      }
+      umma_commit(bar_s);
+      umma_commit(&bar_empty[slotK]);
+      ok = mbar_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns) && mbar_wait(bar_p01, k & 1, p.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+      pv(0, C::COL_S, slotV, k > 0);       // O_d += P_d V
+      pv(1, C::COL_S + 64, slotV, k > 0);  // O_s += P_s V
+      umma_commit(bar_o01);
+      ok = mbar_wait(bar_pt, k & 1, p.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+      pv(2, C::COL_S, slotV, k > 0);  // O_t += P_t V
+      umma_commit(bar_ot);
+      umma_commit(&bar_empty[slotV]);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
+    }
+  } else if (run && warp < 4) {
+    // ------------------------------------------------ rows: gather, softmax, epilogue
+    const int r = threadIdx.x;  // row of the tile = sampled-row index (padded)
+    const int x = min(max(p.rows[min(r, p.S - 1)], 0), p.L - 1);
+    {
+      // gather Q row x into the 128-byte-swizzled K-major tile layout
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.L + x) * D);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 val = __ldg(src + c);
+        const int h = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(sQ + h * C::HALF_BYTES + r * 128 + ((cc ^ (r & 7)) << 4)) = val;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar_q);
+    }
+    const int ir = x / p.F, jr = x - (x / p.F) * p.F;
+    const int lo_s = max(0, (ir - p.a1 + 1) * p.F);
+    const int hi_s = min(p.L, (ir + p.a1) * p.F);
+    const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + C::COL_S;
+    const float sl2 = p.sl2;
+    // One softmax reference (the running max over all kept keys) serves the
+    // three variants: P_s and P_t are P_d restricted to their masks.
+    float m_ref = -INFINITY, l_d = 0.f, l_s = 0.f, l_t = 0.f;
+    int inband_s = 0, inband_t = 0;
+    bool ok = true;
+    for (int k = 0; k < nk; ++k) {
+      if (!warp_wait_p(bar_s, k & 1, p.wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(sr[c][e]);
+
+      const int kbase = (kt0 + k) * 128;
+      const int nvalid = min(128, y_end - kbase);  // keys of this chunk in the tile
+      // Key masks of the tile: dense (chunk end), spatial (one key interval
+      // of frames), temporal (|j - j_r| < a2 within each frame segment).
+      uint32_t md[4] = {0u, 0u, 0u, 0u}, ms[4] = {0u, 0u, 0u, 0u}, mt[4] = {0u, 0u, 0u, 0u};
+      set_range128(md, 0, nvalid);
+      set_range128(ms, max(lo_s - kbase, 0), min(hi_s - kbase, nvalid));
+      {
+        int c = 0;
+        int j0 = kbase % p.F;
+        while (c < nvalid) {  // one frame segment per pass: keys c .. c + (F - j0) - 1
+          const int seg_end = min(nvalid, c + (p.F - j0));
+          const int lo = max(c, c + (jr - p.a2 + 1 - j0));
+          const int hi = min(seg_end, c + (jr + p.a2 - j0));
+          if (lo < hi) set_range128(mt, lo, hi);
+          c = seg_end;
+          j0 = 0;
+        }
+      }
+      // one max over the kept keys; every variant uses it as its reference
+      if (nvalid < 128) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (!bit128(md, c)) s[c] = -INFINITY;
+      }
+      float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]), m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
+#pragma unroll
+      for (int c = 8; c < 128; c += 8) {
+        m0 = fmax3f(m0, s[c], s[c + 1]);
+        m1 = fmax3f(m1, s[c + 2], s[c + 3]);
+        m2 = fmax3f(m2, s[c + 4], s[c + 5]);
+        m3 = fmax3f(m3, s[c + 6], s[c + 7]);
+      }
+      const float m_new = fmax3f(m_ref, fmax3f(m0, m1, m2), m3);
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_new > m_ref + p.lazy_th) {
+        alpha = ex2_approx((m_ref - m_new) * sl2);
+        m_ref = m_new;
+        resc = true;
+      }
+      const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref * sl2;
+      {
+        const float2 sl2x2 = make_float2(sl2, sl2), nb2 = make_float2(nb, nb);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
+          s[2 * c] = ex2_approx(x.x);  // s now holds the weights e
+          s[2 * c + 1] = ex2_approx(x.y);
+        }
+      }
+      inband_s += __popc(ms[0]) + __popc(ms[1]) + __popc(ms[2]) + __popc(ms[3]);
+      inband_t += __popc(mt[0]) + __popc(mt[1]) + __popc(mt[2]) + __popc(mt[3]);
+      uint32_t pk[64];
+      l_d = l_d * alpha + pack_masked(s, md, pk);
+      __syncwarp();
+      st_p64(tS, pk);
+      l_s = l_s * alpha + pack_masked(s, ms, pk);
+      __syncwarp();
+      st_p64(tS + 64, pk);
+      const bool any_resc = k > 0 && __any_sync(0xffffffffu, resc);
+      if (any_resc) {
+        if (!warp_wait_p(bar_o01, (k - 1) & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        rescale_o<D>(tmem + lane_bits + C::col_o(0), alpha);
+        rescale_o<D>(tmem + lane_bits + C::col_o(1), alpha);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p01);
+      l_t = l_t * alpha + pack_masked(s, mt, pk);
+      // P_t goes over P_d once P_d V has read it
+      if (!warp_wait_p(bar_o01, k & 1, p.wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      st_p64(tS, pk);
+      if (any_resc) {
+        if (!warp_wait_p(bar_ot, (k - 1) & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        rescale_o<D>(tmem + lane_bits + C::col_o(2), alpha);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_pt);
+    }
+    // Kept keys whose weights all underflowed relative to the shared reference
+    // (in-band logits more than ~126 / (scale log2 e) below the row max):
+    // report it rather than return a wrong label.
+    if ((inband_s > 0 && !(l_s > 0.f)) || (inband_t > 0 && !(l_t > 0.f))) atomicOr(p.status, SVG_DEV_RANGE);
+    if (ok && warp_wait_p(bar_ot, (nk - 1) & 1, p.wait_ns)) {
+      tc_fence_after();
+#pragma unroll
+      for (int v = 0; v < 3; ++v) {
+        const size_t base = ((static_cast<size_t>(bh) * p.nch + chunk) * 3 + v) * 128 + r;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + base * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          __syncwarp();
+          tmem_ld32(tmem + lane_bits + C::col_o(v) + c * 32, ov);
+          tmem_wait_ld();
+          reg_fence32(ov);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                         __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+        }
+        const float lv = (v == 0) ? l_d : (v == 1 ? l_s : l_t);
+        const int nin = (v == 0) ? 1 : (v == 1 ? inband_s : inband_t);
+        // max in log2 units; a variant with no kept key in this chunk has none
+        p.ws_ml[base * 2 + 0] = (m_ref == -INFINITY || nin == 0) ? -INFINITY : m_ref * sl2;
+        p.ws_ml[base * 2 + 1] = lv;
+      }
+    } else {
+      *abort_flag = 1;
+      atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// [BH, L, D] bf16 tensor map with 64 x 128 x 1 boxes (defined in attn_sm100.cu).
+svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D);
+
+template <int D>
+svg_status launch_profile_sm100_d(ProfSm100Params& p, const void* k, const void* v, cudaStream_t stream) {
+  using C = PCfg<D>;
+  svg_status st;
+  if ((st = make_tile_map_bf16(&p.tm_k, k, p.BH, p.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_v, v, p.BH, p.L, D)) != SVG_OK) return st;
+  cudaError_t e = cudaFuncSetAttribute(profile_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(profile smem)");
+  profile_sm100_kernel<D><<<dim3(p.nch, p.BH), C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cuda_check(cudaGetLastError(), "profile launch");
+}
+
+svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const void* q, const void* k,
+                                const void* v, int a1, int a2, const int32_t* rows, int S, float* ws_o,
+                                float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream) {
+  ProfSm100Params p;
+  memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.rows = rows;
+  p.ws_o = ws_o;
+  p.ws_ml = ws_ml;
+  p.BH = BH;
+  p.L = N * F;
+  p.N = N;
+  p.F = F;
+  p.S = S;
+  p.nch = nch;
+  p.chunk = chunk;
+  p.a1 = a1;
+  p.a2 = a2;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.lazy_th = 8.0f / p.sl2;
+  p.status = status;
+  p.wait_ns = kDefaultWaitNs;
+  if (d == 64) return launch_profile_sm100_d<64>(p, k, v, stream);
+  if (d == 128) return launch_profile_sm100_d<128>(p, k, v, stream);
+  return fail(SVG_ERR_UNSUPPORTED, "bf16 profiling supports d in {64, 128}, got %d", d);
+}
+
+}  // namespace svg

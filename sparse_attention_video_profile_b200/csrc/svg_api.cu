@@ -25,10 +25,10 @@ svg_status cuda_check(cudaError_t e, const char* what) {
   return fail(SVG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-namespace {
-
 // Per-device status word used when the caller passes no status_dev.
 __device__ int g_internal_status;
+
+namespace {
 
 size_t elem_size(int dtype) { return dtype == SVG_FP32 ? 4 : 2; }
 
@@ -71,6 +71,12 @@ svg_status status_word(int32_t* user, int** out, cudaStream_t stream) {
     *out = user;
     return SVG_OK;
   }
+  return internal_status_word(out, stream);
+}
+
+}  // namespace
+
+svg_status internal_status_word(int** out, cudaStream_t stream) {
   void* p = nullptr;
   cudaError_t e = cudaGetSymbolAddress(&p, g_internal_status);
   if (e != cudaSuccess) return cuda_check(e, "cudaGetSymbolAddress(status)");
@@ -79,6 +85,8 @@ svg_status status_word(int32_t* user, int** out, cudaStream_t stream) {
   *out = static_cast<int*>(p);
   return SVG_OK;
 }
+
+namespace {
 
 svg_status run_attention(const svg_shape* s, BandAttnArgs& a, int32_t* status_dev, cudaStream_t stream) {
   a.B = s->B;

@@ -225,10 +225,11 @@ def run_reference(args, wl, rank, world):
 
 
 def config_dict(wl, world):
-    return {"workload": f"HunyuanVideo-shaped {wl.name}: B={wl.B} H={wl.H} N={wl.N} F={wl.F} L={wl.L} d={wl.d}",
+    shape_name = "mixed sparse-pattern" if wl.name.startswith("mixed") else "HunyuanVideo-shaped"
+    return {"workload": f"{shape_name} {wl.name}: B={wl.B} H={wl.H} N={wl.N} F={wl.F} L={wl.L} d={wl.d}",
             "B": wl.B, "H": wl.H, "N": wl.N, "F": wl.F, "L": wl.L, "d": wl.d, "a1": wl.a1, "a2": wl.a2, "S": wl.S,
             "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": "inputs larger than L2 (Q,K,V 3 x 730 MB); no flush"}
+            "l2": f"inputs larger than L2 (Q,K,V 3 x {wl.B * wl.H * wl.L * wl.d * 2 / 1e6:.0f} MB); no flush"}
 
 
 def run_ours(args, wl, rank, world, local):
@@ -248,12 +249,35 @@ def run_ours(args, wl, rank, world, local):
     shape = svg.make_shape(q, N, F)
     prof_ws = svg.alloc_workspace(svg.svg_profile_workspace_size(shape, wl.S), dev)
 
-    names = ("profile", "permute", "attn", "unpermute")
+    mixed = wl.name.startswith("mixed")
+    if mixed:
+        prm = synth.MIXED_PARAMS
+        modes_np = synth.head_modes(wl.B, wl.H, rank)
+        mode = torch.from_numpy(modes_np).to(dev)
+    names = ("permute", "attn", "unpermute") if mixed else ("profile", "permute", "attn", "unpermute")
 
     def new_events():
         return {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
 
+    def step_mixed(e=None):
+        if e:
+            e["permute"][0].record(stream)
+        svg.svg_permute_qkv(q, k, v, N, F, md_label, out=(qp, kp, vp))
+        if e:
+            e["permute"][1].record(stream)
+            e["attn"][0].record(stream)
+        svg.svg_mixed_attn(q, k, v, qp, kp, vp, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
+                           op=op, status=status)
+        if e:
+            e["attn"][1].record(stream)
+            e["unpermute"][0].record(stream)
+        svg.svg_unpermute(op, N, F, md_label, out=o)
+        if e:
+            e["unpermute"][1].record(stream)
+
     def step(e=None):
+        if mixed:
+            return step_mixed(e)
         if e:
             e["profile"][0].record(stream)
         svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws)
@@ -272,12 +296,19 @@ def run_ours(args, wl, rank, world, local):
         if e:
             e["unpermute"][1].record(stream)
 
+    if mixed:
+        # heads that run on token-major copies (label 1 for the permute calls)
+        md_label = torch.from_numpy((modes_np == 3).astype(np.int8)).to(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    labels_np = label.cpu().numpy()
+    if mixed:
+        labels_np = (modes_np == 3).astype(np.int8)
+        pairs = metrics.mixed_pairs(N, F, modes_np, prm["window"], prm["md_half"], prm["stripe"])
+    else:
+        labels_np = label.cpu().numpy()
+        pairs = metrics.effective_pairs(N, F, wl.a1, wl.a2, labels_np)
     n_temporal = int(labels_np.sum())
-    pairs = metrics.effective_pairs(N, F, wl.a1, wl.a2, labels_np)
     flops = metrics.attention_flops(pairs, wl.d)
 
     step_events = [new_events() for _ in range(args.steps)]
@@ -317,7 +348,7 @@ def run_ours(args, wl, rank, world, local):
 
     # end to end through the public call with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not mixed:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
         mseh = torch.empty(mse.shape, dtype=mse.dtype, pin_memory=True)
@@ -361,7 +392,7 @@ def run_ours(args, wl, rank, world, local):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not mixed:
         qkv64 = head_f64(wl, q, k, v)
         ms, desc, _ = oracle_sample(wl, qkv64, rows_np, labels_np, n_prof_rows=wl.S, n_attn_rows=1024)
         cpu = {"value": ms, "unit": "ms/call", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
@@ -386,7 +417,7 @@ def run_ours(args, wl, rank, world, local):
         "hbm_peak_gbs": hbm,
         "clocks": clocks.summary(),
         "e2e": e2e,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": (3 if mixed else 5) * args.steps,
         "cpu_baseline": cpu,
     }
     if rank == 0:

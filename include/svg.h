@@ -281,6 +281,69 @@ SVG_API svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, con
                               float* mse, int8_t* label, void* workspace, size_t workspace_bytes,
                               int32_t* status_dev, void* stream);
 
+/*
+ * Mixed sparse patterns ("Sparse-vDiT" review, pith.science, "What carries
+ * the argument": every head takes one of five modes -- full attention, skip,
+ * diagonal, multi-diagonal, vertical stripe -- and heads that share a mode
+ * are fused into one operation; the multi-diagonal pattern is handled by a
+ * token rearrangement that turns it into a diagonal one).  Per-head modes,
+ * as int8 values in a device array [B, H]:
+ *   SVG_MODE_FULL       every key
+ *   SVG_MODE_SKIP       no key: the head's output is zero
+ *   SVG_MODE_DIAGONAL   |x - y| <= window (a band of width 2*window + 1)
+ *   SVG_MODE_MULTIDIAG  |j_x - j_y| <= md_half: the same in-frame position
+ *                       (+-md_half) in every frame, i.e. diagonals of stride F;
+ *                       run on token-major copies, where it is block-banded
+ *                       with G = N and a = md_half + 1
+ *   SVG_MODE_STRIPE     y < stripe (the first `stripe` keys)
+ */
+#define SVG_MODE_FULL 0
+#define SVG_MODE_SKIP 1
+#define SVG_MODE_DIAGONAL 2
+#define SVG_MODE_MULTIDIAG 3
+#define SVG_MODE_STRIPE 4
+
+/*
+ * svg_mixed_attn -- attention of every head under its own mode, all heads in
+ * one launch (bf16 only).  Multi-diagonal heads read qp,kp,vp (token-major)
+ * and write op; every other head reads q,k,v and writes o (skipped heads
+ * write zeros to o).  window, md_half >= 0; stripe >= 1.  Other arguments as
+ * for svg_block_sparse_attn.
+ */
+SVG_API svg_status svg_mixed_attn(const svg_shape* shape, const void* q, const void* k, const void* v,
+                                  const void* qp, const void* kp, const void* vp, void* o, void* op,
+                                  const int8_t* mode, int32_t window, int32_t md_half, int32_t stripe,
+                                  int32_t* status_dev, void* stream);
+
+/* svg_mixed_3d_attn_workspace_size -- workspace of svg_mixed_3d_attn (bytes; 0 on bad arguments). */
+SVG_API size_t svg_mixed_3d_attn_workspace_size(const svg_shape* shape);
+
+/*
+ * svg_mixed_3d_attn -- one mixed-pattern attention call: permute the
+ * multi-diagonal heads' q, k, v to token-major order, run svg_mixed_attn,
+ * and permute their output back into o (frame-major [B,H,L,d]).
+ */
+SVG_API svg_status svg_mixed_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                     const int8_t* mode, int32_t window, int32_t md_half, int32_t stripe,
+                                     void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                     void* stream);
+
+/*
+ * svg_selftest_wait_bound -- failure-detection self-test (test hook).
+ *
+ * Runs the bf16 attention kernel (one band covering all keys) with its
+ * producer's loads withheld, so nothing ever arrives on the barriers its
+ * consumers wait for.  Every wait must give up after wait_ns.  The kernel
+ * then sets SVG_DEV_TIMEOUT in *status_dev, frees its tensor memory and
+ * exits; CTAs that start later see the bit and skip their work.  The CUDA
+ * context stays usable.  o is left unspecified.  The call itself returns
+ * SVG_OK once the launch is enqueued.
+ * wait_ns in [1e6, 1e10]; status_dev is required and must be zero on entry.
+ */
+SVG_API svg_status svg_selftest_wait_bound(const svg_shape* shape, const void* q, const void* k,
+                                           const void* v, void* o, uint64_t wait_ns,
+                                           int32_t* status_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

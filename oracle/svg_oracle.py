@@ -22,6 +22,11 @@ Sources (cited by page title and section):
   [SVG2]   SVG2 explainer (gist.science), section 2.A "Semantic-Aware
            Permutation" (a token permutation applied before attention and
            undone after it leaves the result mathematically unchanged).
+  [SvDiT]  "Sparse-vDiT" review (pith.science), "What carries the argument"
+           and "The reading": per-head modes {full, skip, diagonal,
+           multi-diagonal, vertical stripe}; skipped heads have their output
+           zeroed; the multi-diagonal pattern is turned into a diagonal one by
+           a token rearrangement.
 
 Readings taken where the pages are silent or garbled:
   * Temporal mask: the (i, j) form |j1 - j2| < a2 is authoritative.  The
@@ -37,6 +42,10 @@ Readings taken where the pages are silent or garbled:
     -1 / +1.
   * Layout transformation: token (i, j) moves from frame-major position
     x = i*F + j to token-major position x' = j*N + i.
+  * Mixed modes (widths from the workload definition): diagonal of width 2W
+    keeps |x1 - x2| <= W; multi-diagonal of stride F and width 2h keeps
+    |j1 - j2| <= h (the (i, j) form, as for the temporal mask); vertical
+    stripe keeps the first P keys; skip gives a zero output.
 """
 from __future__ import annotations
 
@@ -282,3 +291,59 @@ def block_list(mask: np.ndarray, Bq: int, Bk: int):
             active[qb, kb] = bool(t.any())
             full[qb, kb] = bool(t.all())
     return active, full
+
+
+# --------------------------------------------------------------------------
+# mixed sparse patterns  [SvDiT]
+# --------------------------------------------------------------------------
+
+MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
+
+
+def window_mask(L: int, W: int, rows=None) -> np.ndarray:
+    """Diagonal band: keep (x, y) iff |x - y| <= W."""
+    x = np.arange(L)
+    xq = x if rows is None else x[np.asarray(rows)]
+    return np.abs(xq[:, None] - x[None, :]) <= W
+
+
+def prefix_mask(L: int, P: int, rows=None) -> np.ndarray:
+    """Vertical stripe: keep (x, y) iff y < P."""
+    R = L if rows is None else len(rows)
+    return np.broadcast_to(np.arange(L)[None, :] < P, (R, L)).copy()
+
+
+def mode_mask(mode: int, N: int, F: int, window: int, md_half: int, stripe: int, rows=None):
+    """The mask of one mixed-pattern head in the original layout (None for skip)."""
+    L = N * F
+    R = L if rows is None else len(rows)
+    if mode == MODE_FULL:
+        return np.ones((R, L), dtype=bool)
+    if mode == MODE_DIAGONAL:
+        return window_mask(L, window, rows)
+    if mode == MODE_MULTIDIAG:
+        return temporal_mask(N, F, md_half + 1, rows)  # |j1 - j2| <= md_half
+    if mode == MODE_STRIPE:
+        return prefix_mask(L, stripe, rows)
+    if mode == MODE_SKIP:
+        return None
+    raise ValueError(mode)
+
+
+def mixed_attention(q, k, v, modes, N: int, F: int, window: int, md_half: int, stripe: int, scale=None,
+                    rows=None) -> np.ndarray:
+    """Each head under its mode; skipped heads give zeros.  [B, H, R, d]."""
+    q = np.asarray(q)
+    B, H, L, d = q.shape
+    all_rows = np.arange(L) if rows is None else np.asarray(rows)
+    out = np.zeros((B, H, all_rows.size, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            m = int(np.asarray(modes)[b, h])
+            if m == MODE_SKIP:
+                continue
+            out[b, h] = attention_rows(
+                np.asarray(q[b, h], np.float64), np.asarray(k[b, h], np.float64),
+                np.asarray(v[b, h], np.float64), all_rows,
+                lambda rr, m=m: mode_mask(m, N, F, window, md_half, stripe, rr), scale)
+    return out

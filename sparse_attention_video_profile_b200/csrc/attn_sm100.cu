@@ -46,13 +46,16 @@ struct AttnParams {
   CUtensorMap tm_qp, tm_kp, tm_vp;  // token-major [BH, L, D] bf16
   __nv_bfloat16* o;
   __nv_bfloat16* op;
-  const int8_t* label;
+  const int8_t* label;  // spatial (0) / temporal (1) per head, or nullptr
+  const int8_t* modes;  // mixed-pattern mode per head (SVG_MODE_*), or nullptr
   int BH, L, n_ctiles;
   int G0, a0, G1, a1;
+  int win, md_a, stripe, N;  // mixed modes: window half-width, multi-diagonal band, stripe length
   float sl2;      // scale * log2(e)
   float lazy_th;  // rescale threshold in raw score units (8 / sl2)
   int* status;
   uint64_t wait_ns;
+  int withhold_loads;  // self-test only: the producer issues nothing
 };
 
 template <int D>
@@ -87,6 +90,49 @@ constexpr int kExpPoly = SVG_EXP_POLY_PAIRS;
 __device__ __forceinline__ void record_timeout(const AttnParams& p, volatile int* abort_flag) {
   *abort_flag = 1;
   atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
+}
+
+// The keys one head keeps for query row x form one interval [lo, hi):
+//   GROUP  (G, a): |floor(x/G) - floor(y/G)| < a  -> [(g-a+1)G, (g+a)G), g = floor(x/G)
+//   WINDOW (W):    |x - y| <= W                     -> [x-W, x+W+1)
+//   PREFIX (P):    y < P                            -> [0, P)
+//   SKIP:          no key (the output row is zero)
+// each clipped to [0, L).  lo and hi never decrease as x grows, so a tile of
+// rows [x0, x1] needs keys [lo(x0), hi(x1)).
+enum BandKind { kGroup = 0, kWindow = 1, kPrefix = 2, kSkip = 3 };
+struct HeadBand {
+  int kind, G, a, perm;  // perm: the head runs on the token-major copies
+};
+
+__device__ __forceinline__ void row_interval(const HeadBand& b, int x, int L, int& lo, int& hi) {
+  if (b.kind == kGroup) {
+    const long long g = x / b.G;
+    lo = static_cast<int>(max(0LL, (g - b.a + 1) * b.G));
+    hi = static_cast<int>(min(static_cast<long long>(L), (g + b.a) * b.G));
+  } else if (b.kind == kWindow) {
+    lo = max(0, x - b.G);
+    hi = min(L, x + b.G + 1);
+  } else if (b.kind == kPrefix) {
+    lo = 0;
+    hi = min(L, b.G);
+  } else {
+    lo = 0;
+    hi = 0;
+  }
+}
+
+__device__ __forceinline__ HeadBand head_band(const AttnParams& p, int bh) {
+  if (p.modes != nullptr) {
+    switch (p.modes[bh]) {
+      case SVG_MODE_FULL: return HeadBand{kGroup, p.L, 1, 0};
+      case SVG_MODE_DIAGONAL: return HeadBand{kWindow, p.win, 0, 0};
+      case SVG_MODE_MULTIDIAG: return HeadBand{kGroup, p.N, p.md_a, 1};
+      case SVG_MODE_STRIPE: return HeadBand{kPrefix, p.stripe, 0, 0};
+      default: return HeadBand{kSkip, 1, 0, 0};
+    }
+  }
+  const int lab = p.label ? static_cast<int>(p.label[bh]) : 0;
+  return lab ? HeadBand{kGroup, p.G1, p.a1, 1} : HeadBand{kGroup, p.G0, p.a0, 0};
 }
 
 // Warp-uniform bounded wait.
@@ -140,17 +186,16 @@ __global__ void __launch_bounds__(384, 1) attn_sm100_kernel(const __grid_constan
   // ---- work item: (head, 256-row query slab)
   const int ct = blockIdx.x % p.n_ctiles;
   const int bh = blockIdx.x / p.n_ctiles;
-  const int lab = p.label ? static_cast<int>(p.label[bh]) : 0;
-  const int G = lab ? p.G1 : p.G0;
-  const int a = lab ? p.a1 : p.a0;
+  const HeadBand band = head_band(p, bh);
+  const int lab = band.perm;
   const int L = p.L;
   const int q0 = ct * 256;
   const int q_last = min(q0 + 255, L - 1);
-  const long long g_first = q0 / G, g_last = q_last / G;
-  const int lo_cta = static_cast<int>(max(0LL, (g_first - a + 1) * G));
-  const int hi_cta = static_cast<int>(min(static_cast<long long>(L), (g_last + a) * G));
+  int lo_cta, hi_cta, lo_unused, hi_unused;
+  row_interval(band, q0, L, lo_cta, hi_unused);
+  row_interval(band, q_last, L, lo_unused, hi_cta);
   const int kt0 = lo_cta / C::BK;
-  const int nk = (hi_cta + C::BK - 1) / C::BK - kt0;
+  const int nk = (hi_cta > lo_cta) ? (hi_cta + C::BK - 1) / C::BK - kt0 : 0;  // 0: skipped head
   const bool run = (*abort_flag == 0);
 
   // Every warp takes part in the register split before anything else, so the
@@ -158,7 +203,7 @@ __global__ void __launch_bounds__(384, 1) attn_sm100_kernel(const __grid_constan
   // that set its register budget.
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CONTROL));
-    if (run && warp == 8 && lane == 0) {
+    if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads) {
       // ------------------------------------------------ TMA producer
       {
       const CUtensorMap* tq = lab ? &p.tm_qp : &p.tm_q;
@@ -188,7 +233,7 @@ __global__ void __launch_bounds__(384, 1) attn_sm100_kernel(const __grid_constan
           tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, row, bh);
       }
     }
-    } else if (run && warp == 9 && lane == 0) {
+    } else if (run && nk > 0 && warp == 9 && lane == 0) {
       // ------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
@@ -258,11 +303,7 @@ __global__ void __launch_bounds__(384, 1) attn_sm100_kernel(const __grid_constan
     const int r = q0 + i * C::BQ + quad * 32 + lane;  // query row in the head's layout
     const bool row_ok = r < L;
     int lo_r = 0, hi_r = 0;
-    if (row_ok) {
-      const long long g = r / G;
-      lo_r = static_cast<int>(max(0LL, (g - a + 1) * G));
-      hi_r = static_cast<int>(min(static_cast<long long>(L), (g + a) * G));
-    }
+    if (row_ok) row_interval(band, r, L, lo_r, hi_r);
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::col_s(i);
     const uint32_t tO = tmem + lane_bits + C::col_o(i);
@@ -360,7 +401,14 @@ __global__ void __launch_bounds__(384, 1) attn_sm100_kernel(const __grid_constan
       tc_fence_before();
       mbar_arrive(&bar_p[i]);
     }
-    if (ok && warp_wait(&bar_o[i], (nk - 1) & 1, p.wait_ns)) {
+    if (nk == 0) {
+      // skipped head: its output rows are zero
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * L + r) * D);
+#pragma unroll
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else if (ok && warp_wait(&bar_o[i], (nk - 1) & 1, p.wait_ns)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* out = (lab ? p.op : p.o) + (static_cast<size_t>(bh) * L + (row_ok ? r : 0)) * D;
@@ -408,13 +456,18 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   if ((st = make_tile_map_bf16(&p.tm_q, a.q, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_k, a.k, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_v, a.v, BH, a.L, D)) != SVG_OK) return st;
-  const bool perm = a.label != nullptr;
+  const bool perm = a.label != nullptr || a.modes != nullptr;
   if ((st = make_tile_map_bf16(&p.tm_qp, perm ? a.qp : a.q, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_kp, perm ? a.kp : a.k, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.op = static_cast<__nv_bfloat16*>(perm ? a.op : a.o);
   p.label = a.label;
+  p.modes = a.modes;
+  p.win = a.win;
+  p.md_a = a.md_a;
+  p.stripe = a.stripe;
+  p.N = a.N;
   p.BH = BH;
   p.L = a.L;
   p.n_ctiles = (a.L + 255) / 256;
@@ -426,6 +479,7 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   p.lazy_th = 8.0f / p.sl2;
   p.status = a.status;
   p.wait_ns = a.wait_ns;
+  p.withhold_loads = a.withhold_loads;
   const long long grid = static_cast<long long>(BH) * p.n_ctiles;
   if (grid > 0x7fffffffLL) return fail(SVG_ERR_UNSUPPORTED, "grid too large");
   static bool attr_set = false;

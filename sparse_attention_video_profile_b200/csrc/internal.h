@@ -24,8 +24,10 @@ svg_status cuda_check(cudaError_t e, const char* what);
 // Moves rows between frame-major (x = i*F + j) and token-major (x' = j*N + i)
 // order for up to three tensors.  to_token_major: src frame-major -> dst
 // token-major; otherwise the inverse.  label == nullptr: every head.
+// Only heads whose label equals `sel` move (SVG_TEMPORAL unless given).
 svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F,
-                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream);
+                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream,
+                          int sel = SVG_TEMPORAL);
 
 // ------------------------------------------------------------- attention
 
@@ -42,8 +44,11 @@ struct BandAttnArgs {
   const int8_t* label;  // nullptr -> every head uses band 0 on (q, k, v, o)
   int G0, a0;           // band of label-0 heads
   int G1, a1;           // band of label-1 heads
+  const int8_t* modes;  // mixed-pattern modes (overrides label), or nullptr
+  int win, md_a, stripe, N;
   int* status;          // device status word (never null here)
   uint64_t wait_ns;
+  int withhold_loads;   // self-test of the bounded waits (tcgen05 kernel only)
 };
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);

@@ -20,6 +20,7 @@ struct PermuteParams {
   const uint4* src[3];
   uint4* dst[3];
   const int8_t* label;
+  int sel;                    // heads whose label equals sel move
   long long chunks_per_head;  // L * row_chunks
   int row_chunks;             // 16-byte chunks per row
   int BH, N, F;
@@ -32,7 +33,7 @@ constexpr int kPermUnroll = 4;
 __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const __grid_constant__ PermuteParams p) {
   const int t = blockIdx.y / p.BH;       // tensor
   const int bh = blockIdx.y - t * p.BH;  // head
-  if (p.label != nullptr && p.label[bh] != SVG_TEMPORAL) return;
+  if (p.label != nullptr && p.label[bh] != p.sel) return;
   const long long head_off = static_cast<long long>(bh) * p.chunks_per_head;
   const uint4* __restrict__ src = p.src[t] + head_off;
   uint4* __restrict__ dst = p.dst[t] + head_off;
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const __grid
 }  // namespace
 
 svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F,
-                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream) {
+                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream, int sel) {
   if (row_bytes % 16 != 0) return fail(SVG_ERR_UNSUPPORTED, "row of %d bytes is not a multiple of 16", row_bytes);
   PermuteParams p{};
   for (int t = 0; t < ntensors; ++t) {
@@ -77,6 +78,7 @@ svg_status launch_permute(int ntensors, const void* const* src, void* const* dst
     p.dst[t] = static_cast<uint4*>(dst[t]);
   }
   p.label = label;
+  p.sel = sel;
   p.row_chunks = row_bytes / 16;
   p.chunks_per_head = static_cast<long long>(N) * F * p.row_chunks;
   p.BH = BH;

@@ -50,11 +50,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with the given parity has completed, for at most
 // `limit_ns` nanoseconds of wall time.  Returns false if the bound ran out;
 // the caller then records the failure and leaves its pipeline loop.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
+  if (mbar_test_wait(addr, parity)) return true;  // already complete: no suspend
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {

@@ -88,14 +88,15 @@ svg_status internal_status_word(int** out, cudaStream_t stream) {
 
 namespace {
 
-svg_status run_attention(const svg_shape* s, BandAttnArgs& a, int32_t* status_dev, cudaStream_t stream) {
+svg_status run_attention(const svg_shape* s, BandAttnArgs& a, int32_t* status_dev, cudaStream_t stream,
+                         uint64_t wait_ns = kDefaultWaitNs) {
   a.B = s->B;
   a.H = s->H;
   a.L = s->N * s->F;
   a.d = s->d;
   a.dtype = s->dtype;
   a.scale = eff_scale(s);
-  a.wait_ns = kDefaultWaitNs;
+  a.wait_ns = wait_ns;
   svg_status st = status_word(status_dev, &a.status, stream);
   if (st != SVG_OK) return st;
   if (s->dtype == SVG_BF16) return launch_attn_sm100(a, stream);
@@ -326,6 +327,96 @@ svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void*
   if ((st = svg_block_sparse_attn(shape, q, k, v, qp, kp, vp, o, op, label, a1, a2, status_dev, stream)) != SVG_OK)
     return st;
   return svg_unpermute(shape, op, o, label, stream);
+}
+
+svg_status svg_mixed_attn(const svg_shape* shape, const void* q, const void* k, const void* v, const void* qp,
+                          const void* kp, const void* vp, void* o, void* op, const int8_t* mode, int32_t window,
+                          int32_t md_half, int32_t stripe, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "mixed-pattern attention runs in bf16 only");
+  if ((st = check_tensors({q, k, v, o, qp, kp, vp, op})) != SVG_OK) return st;
+  if (mode == nullptr) return fail(SVG_ERR_INVALID_ARG, "mode is NULL");
+  if (window < 0 || md_half < 0 || stripe < 1) return fail(SVG_ERR_INVALID_ARG, "window, md_half >= 0 and stripe >= 1");
+  const int L = shape->N * shape->F;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.qp = qp;
+  a.kp = kp;
+  a.vp = vp;
+  a.op = op;
+  a.modes = mode;
+  a.G0 = L;
+  a.a0 = 1;
+  a.G1 = L;
+  a.a1 = 1;
+  a.win = window < L ? window : L;
+  a.N = shape->N;
+  a.md_a = clamp_band(md_half + 1, shape->N, L);
+  a.stripe = stripe < L ? stripe : L;
+  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+size_t svg_mixed_3d_attn_workspace_size(const svg_shape* shape) {
+  if (check_shape(shape) != SVG_OK) return 0;
+  const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
+  return 4 * ((t + 255) / 256 * 256);
+}
+
+svg_status svg_mixed_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                             const int8_t* mode, int32_t window, int32_t md_half, int32_t stripe, void* workspace,
+                             size_t workspace_bytes, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (!workspace || !mode) return fail(SVG_ERR_INVALID_ARG, "workspace or mode is NULL");
+  const size_t need = svg_mixed_3d_attn_workspace_size(shape);
+  if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t t_al = need / 4;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void *qp = w, *kp = w + t_al, *vp = w + 2 * t_al, *op = w + 3 * t_al;
+  const int BH = shape->B * shape->H;
+  const int rb = static_cast<int>(shape->d * elem_size(shape->dtype));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* src3[3] = {q, k, v};
+  void* dst3[3] = {qp, kp, vp};
+  if ((st = launch_permute(3, src3, dst3, BH, shape->N, shape->F, rb, mode, true, s, SVG_MODE_MULTIDIAG)) != SVG_OK)
+    return st;
+  if ((st = svg_mixed_attn(shape, q, k, v, qp, kp, vp, o, op, mode, window, md_half, stripe, status_dev, stream)) !=
+      SVG_OK)
+    return st;
+  const void* src1[1] = {op};
+  void* dst1[1] = {o};
+  return launch_permute(1, src1, dst1, BH, shape->N, shape->F, rb, mode, false, s, SVG_MODE_MULTIDIAG);
+}
+
+svg_status svg_selftest_wait_bound(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                   uint64_t wait_ns, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "the self-test runs the bf16 tensor-core kernel");
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (status_dev == nullptr) return fail(SVG_ERR_INVALID_ARG, "status_dev is required");
+  if (wait_ns < 1000000ull || wait_ns > 10000000000ull)
+    return fail(SVG_ERR_INVALID_ARG, "wait_ns must be in [1 ms, 10 s]");
+  const int L = shape->N * shape->F;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.label = nullptr;
+  a.G0 = L;
+  a.a0 = 1;
+  a.G1 = L;
+  a.a1 = 1;
+  a.withhold_loads = 1;
+  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream), wait_ns);
 }
 
 }  // extern "C"

@@ -44,3 +44,18 @@ def effective_pairs(N: int, F: int, a1: int, a2: int, labels) -> int:
 
 def attention_flops(pairs: int, d: int) -> float:
     return 4.0 * d * float(pairs)
+
+
+def window_pairs(L: int, W: int) -> int:
+    """Pairs |x - y| <= W on 0..L-1: L*(2W+1) - W*(W+1) for W < L."""
+    W = min(W, L - 1)
+    return L * (2 * W + 1) - W * (W + 1)
+
+
+def mixed_pairs(N: int, F: int, modes, window: int, md_half: int, stripe: int) -> int:
+    """Unmasked pairs summed over heads of the mixed-pattern call (modes 0 full,
+    1 skip, 2 diagonal, 3 multi-diagonal, 4 vertical stripe)."""
+    L = N * F
+    per = {0: L * L, 1: 0, 2: window_pairs(L, window), 3: temporal_pairs(N, F, md_half + 1),
+           4: L * min(stripe, L)}
+    return int(sum(per[int(m)] for m in np.asarray(modes).reshape(-1)))

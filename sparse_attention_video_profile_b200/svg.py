@@ -34,8 +34,11 @@ EXPORTED = (
     "svg_abi_version", "svg_status_string", "svg_last_error", "svg_attn_tile", "svg_block_list",
     "svg_profile_workspace_size", "svg_profile_heads", "svg_permute", "svg_permute_qkv", "svg_unpermute",
     "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
-    "svg_sparse_3d_attn", "svg_profile_heads_noalloc",
+    "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
+    "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn",
 )
+
+MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
 
 
 class SvgError(RuntimeError):
@@ -77,6 +80,10 @@ def _load() -> ctypes.CDLL:
         "svg_sparse_3d_attn_workspace_size": (_Z, [_P, _I]),
         "svg_sparse_3d_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P, _P]),
         "svg_profile_heads_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P]),
+        "svg_selftest_wait_bound": (_I, [_P, _P, _P, _P, _P, ctypes.c_uint64, _P, _P]),
+        "svg_mixed_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+        "svg_mixed_3d_attn_workspace_size": (_Z, [_P]),
+        "svg_mixed_3d_attn": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _Z, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -283,6 +290,48 @@ def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Te
                                   _ptr(mse), _ptr(label), _ptr(workspace), workspace.numel(), _ptr(status),
                                   _stream(stream)))
     return o, mse, label
+
+
+def svg_mixed_attn(q, k, v, qp, kp, vp, mode, N: int, F: int, window: int, md_half: int, stripe: int, *,
+                   o=None, op=None, status=None, scale: float = 0.0, stream=None):
+    """Every head under its own mode (SVG_MODE_*), one launch.  Returns (o, op)."""
+    _same(q, k, v, qp, kp, vp)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if op is None:
+        op = torch.empty_like(q)
+    _check(lib.svg_mixed_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp),
+                              _ptr(o), _ptr(op), _ptr(mode), window, md_half, stripe, _ptr(status),
+                              _stream(stream)))
+    return o, op
+
+
+def svg_mixed_3d_attn(q, k, v, mode, N: int, F: int, window: int, md_half: int, stripe: int, *, o=None,
+                      workspace=None, status=None, scale: float = 0.0, stream=None):
+    """One mixed-pattern call (permutation of multi-diagonal heads included)."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(int(lib.svg_mixed_3d_attn_workspace_size(ctypes.byref(shape))), q.device)
+    _check(lib.svg_mixed_3d_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(mode), window,
+                                 md_half, stripe, _ptr(workspace), workspace.numel(), _ptr(status),
+                                 _stream(stream)))
+    return o
+
+
+def svg_selftest_wait_bound(q, k, v, N: int, F: int, status, *, wait_ns: int = 50_000_000, o=None,
+                            stream=None):
+    """Failure-detection self-test: the attention kernel with its loads
+    withheld must time out, set SVG_DEV_TIMEOUT in `status` and exit."""
+    shape = make_shape(q, N, F)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib.svg_selftest_wait_bound(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), int(wait_ns),
+                                       _ptr(status), _stream(stream)))
+    return o
 
 
 class SparseAttention3D:

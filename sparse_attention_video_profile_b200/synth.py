@@ -72,6 +72,16 @@ WORKLOADS = {
                         S=128, kinds="coin", weight=("uniform", 1.0, 4.0)),
 }
 
+# Mixed sparse-pattern workload (per-head modes instead of spatial/temporal
+# labels): diagonal band of width 2F, multi-diagonal of stride F and width 64
+# (half-width 32), vertical stripe over the first 512 keys.
+WORKLOADS["mixed"] = Workload("mixed", B=1, H=24, N=21, F=1560, d=128, dtype="bf16", a1=3, a2=33, S=128,
+                              kinds="coin", weight=("uniform", 1.0, 4.0))
+MIXED_PARAMS = {"window": 1560, "md_half": 32, "stripe": 512}
+# Mode shares for heads after the first five (which take modes 0..4 in order
+# so every mode is present): full, skip, diagonal, multi-diagonal, stripe.
+MIXED_MODE_P = (0.10, 0.05, 0.35, 0.30, 0.20)
+
 # HunyuanVideo-shaped density sweep: target density -> (a1, a2).
 HUNYUAN_SWEEP = {0.05: (1, 92), 0.10: (2, 185), 0.15: (3, 281), 0.20: (4, 381),
                  0.30: (6, 589), 0.40: (8, 812), 0.50: (10, 1055)}
@@ -101,6 +111,16 @@ def head_weights(wl: Workload, seed: int) -> np.ndarray:
     else:
         w = rng.uniform(wl.weight[1], wl.weight[2], n)
     return w.reshape(wl.B, wl.H)
+
+
+def head_modes(B: int, H: int, seed: int) -> np.ndarray:
+    """Mixed-pattern mode of every head, [B, H] int8 (0 full, 1 skip,
+    2 diagonal, 3 multi-diagonal, 4 vertical stripe)."""
+    rng = np.random.default_rng(seed + 15485863)
+    n = B * H
+    modes = rng.choice(5, size=n, p=MIXED_MODE_P)
+    modes[:min(5, n)] = np.arange(min(5, n))
+    return modes.reshape(B, H).astype(np.int8)
 
 
 def torch_dtype(wl: Workload) -> torch.dtype:

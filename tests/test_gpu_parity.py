@@ -309,3 +309,56 @@ def test_video_shape_sampled(name):
             got = f64(o[:, h:h + 1, torch.from_numpy(check_rows).to(DEV)])
             assert_close(got, ref, q.dtype, f"{name} head {h}")
     assert set(np.unique(label_np)) <= {0, 1}
+
+
+# ---------------------------------------------------------------- failure detection
+
+def test_bounded_waits_report_timeout_and_context_stays_usable():
+    """The attention kernel with its loads withheld: every wait gives up after
+    50 ms, the status word reports the timeout, and the next call is normal."""
+    q, k, v = rand_qkv(1, 2, 4 * 700, 128, torch.bfloat16, 21)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    svg.svg_selftest_wait_bound(q, k, v, 4, 700, status, wait_ns=50_000_000)
+    torch.cuda.synchronize()
+    assert int(status.item()) & svg.SVG_DEV_TIMEOUT
+    status.zero_()
+    o = svg.svg_dense_attn(q, k, v, 4, 700, status=status)
+    sync_ok(status)
+    ref = oracle.dense_attention(f64(q), f64(k), f64(v))
+    assert_close(f64(o), ref, torch.bfloat16, "after timeout")
+
+
+# ---------------------------------------------------------------- mixed sparse patterns
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_mixed_patterns_small(d):
+    N, F = 6, 90
+    L = N * F
+    modes_np = np.array([[0, 1, 2, 3, 4, 2, 3, 4, 0, 2]], dtype=np.int8)
+    q, k, v = rand_qkv(1, 10, L, d, torch.bfloat16, 23)
+    mode = torch.from_numpy(modes_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_mixed_3d_attn(q, k, v, mode, N, F, F, 7, 100, status=status)
+    sync_ok(status)
+    ref = oracle.mixed_attention(f64(q), f64(k), f64(v), modes_np, N, F, F, 7, 100)
+    assert_close(f64(o), ref, torch.bfloat16, "mixed")
+    assert torch.all(o[0, 1] == 0)
+
+
+def test_mixed_workload_sampled():
+    wl = synth.WORKLOADS["mixed"]
+    prm = synth.MIXED_PARAMS
+    q, k, v = synth.make_qkv(wl, seed=0, device=DEV)
+    modes_np = synth.head_modes(wl.B, wl.H, 0)
+    mode = torch.from_numpy(modes_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_mixed_3d_attn(q, k, v, mode, wl.N, wl.F, prm["window"], prm["md_half"], prm["stripe"],
+                              status=status)
+    sync_ok(status)
+    rows = sampled_rows(wl, n_extra=24)
+    idx = torch.from_numpy(rows).to(DEV)
+    for h in range(wl.H):
+        qn, kn, vn = (f64(t[:, h:h + 1]) for t in (q, k, v))
+        ref = oracle.mixed_attention(qn, kn, vn, modes_np[:, h:h + 1], wl.N, wl.F, prm["window"],
+                                     prm["md_half"], prm["stripe"], rows=rows)
+        assert_close(f64(o[:, h:h + 1, idx]), ref, q.dtype, f"mixed head {h} mode {modes_np[0, h]}")

@@ -322,3 +322,44 @@ def test_block_list_bruteforce_matches_closed_form(L, G, a, Bq, Bk):
         assert set(np.nonzero(active[qb])[0].tolist()) == act
         assert set(np.nonzero(full[qb])[0].tolist()) == ful
 
+
+
+# ------------------------------------------------------------ mixed-pattern pins
+
+@pytest.mark.parametrize("N,F,W,h,P", [(4, 7, 3, 2, 5), (3, 10, 10, 0, 1), (5, 6, 0, 5, 30)])
+def test_mixed_masks_match_definitions(N, F, W, h, P):
+    L = N * F
+    win = np.zeros((L, L), bool)
+    md = np.zeros((L, L), bool)
+    for i1, j1, i2, j2 in itertools.product(range(N), range(F), range(N), range(F)):
+        x1, x2 = i1 * F + j1, i2 * F + j2
+        win[x1, x2] = abs(x1 - x2) <= W
+        md[x1, x2] = abs(j1 - j2) <= h
+    np.testing.assert_array_equal(oracle.mode_mask(oracle.MODE_DIAGONAL, N, F, W, h, P), win)
+    np.testing.assert_array_equal(oracle.mode_mask(oracle.MODE_MULTIDIAG, N, F, W, h, P), md)
+    stripe = oracle.mode_mask(oracle.MODE_STRIPE, N, F, W, h, P)
+    assert stripe.sum() == L * min(P, L) and np.all(stripe[:, :P]) and not np.any(stripe[:, P:])
+    assert oracle.mode_mask(oracle.MODE_FULL, N, F, W, h, P).all()
+    assert oracle.mode_mask(oracle.MODE_SKIP, N, F, W, h, P) is None
+    # closed forms of the pair counts
+    assert win.sum() == L * (2 * min(W, L - 1) + 1) - min(W, L - 1) * (min(W, L - 1) + 1)
+    # multi-diagonal on token-major rows is block-banded with G = N, a = h + 1
+    inv = np.argsort(oracle.token_major_index(N, F))
+    np.testing.assert_array_equal(md[np.ix_(inv, inv)], oracle.banded_mask(L, N, h + 1))
+
+
+def test_mixed_attention_modes():
+    N, F = 4, 6
+    rng = np.random.default_rng(31)
+    q, k, v = (rng.standard_normal((1, 5, N * F, 3)) for _ in range(3))
+    modes = np.array([[0, 1, 2, 3, 4]])
+    out = oracle.mixed_attention(q, k, v, modes, N, F, 2, 1, 5)
+    np.testing.assert_allclose(out[0, 0], oracle.attention(q[0, 0], k[0, 0], v[0, 0]), rtol=1e-12, atol=1e-13)
+    assert np.all(out[0, 1] == 0)  # skipped head: zero output
+    # stripe: brute force on the first keys only
+    ref = _brute_attention(q[0, 4].tolist(), k[0, 4, :5].tolist(), v[0, 4, :5].tolist(), None, 1 / math.sqrt(3))
+    np.testing.assert_allclose(out[0, 4], ref, rtol=1e-12, atol=1e-13)
+    # multi-diagonal through the token rearrangement equals the direct mask
+    qp, kp, vp = (oracle.permute(t[0, 3], N, F) for t in (q, k, v))
+    via = oracle.unpermute(oracle.attention(qp, kp, vp, oracle.banded_mask(N * F, N, 2)), N, F)
+    np.testing.assert_allclose(out[0, 3], via, rtol=1e-12, atol=1e-13)

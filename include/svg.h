@@ -282,6 +282,35 @@ SVG_API svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, con
                               int32_t* status_dev, void* stream);
 
 /*
+ * svg_sparse_3d_attn_host_workspace_size -- device workspace of
+ * svg_sparse_3d_attn_host for a chunk of `heads_per_chunk` heads (0 on bad
+ * arguments): two slots, each with a chunk's q, k, v, o, their token-major
+ * copies and the chunk's profiling workspace.
+ */
+SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, int32_t S, int32_t heads_per_chunk);
+
+/*
+ * svg_sparse_3d_attn_host -- svg_sparse_3d_attn on HOST buffers.
+ *
+ * q_host, k_host, v_host, o_host: [B,H,L,d] in host memory, page-locked for the
+ * copies to overlap (pageable memory works, but the copies then serialise);
+ * rows_host [S], mse_host [B,H,2], label_host [B,H] in host memory.  Heads
+ * are independent, so the call is cut into chunks of heads_per_chunk heads.
+ * The host-to-device copies of one chunk, the kernels of another and the
+ * device-to-host copies of a third overlap on two internal streams plus the
+ * caller's stream.  The results are bit-identical to svg_sparse_3d_attn.
+ * The call is asynchronous: `stream` resumes after the last copy-out, so
+ * synchronise it before reading the host outputs.  Calls on one device must
+ * not run concurrently from several host threads (the internal streams and
+ * events are shared per device).
+ */
+SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q_host, const void* k_host,
+                                           const void* v_host, void* o_host, int32_t a1, int32_t a2,
+                                           const int32_t* rows_host, int32_t S, float* mse_host,
+                                           int8_t* label_host, int32_t heads_per_chunk, void* workspace,
+                                           size_t workspace_bytes, int32_t* status_dev, void* stream);
+
+/*
  * Mixed sparse patterns ("Sparse-vDiT" review, pith.science, "What carries
  * the argument": every head takes one of five modes -- full attention, skip,
  * diagonal, multi-diagonal, vertical stripe -- and heads that share a mode

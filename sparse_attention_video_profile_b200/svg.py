@@ -35,7 +35,8 @@ EXPORTED = (
     "svg_profile_workspace_size", "svg_profile_heads", "svg_permute", "svg_permute_qkv", "svg_unpermute",
     "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
     "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
-    "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn",
+    "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
+    "svg_sparse_3d_attn_host",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -84,6 +85,8 @@ def _load() -> ctypes.CDLL:
         "svg_mixed_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
         "svg_mixed_3d_attn_workspace_size": (_Z, [_P]),
         "svg_mixed_3d_attn": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _Z, _P, _P]),
+        "svg_sparse_3d_attn_host_workspace_size": (_Z, [_P, _I, _I]),
+        "svg_sparse_3d_attn_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _I, _P, _Z, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -320,6 +323,34 @@ def svg_mixed_3d_attn(q, k, v, mode, N: int, F: int, window: int, md_half: int, 
                                  md_half, stripe, _ptr(workspace), workspace.numel(), _ptr(status),
                                  _stream(stream)))
     return o
+
+
+def svg_sparse_3d_attn_host(q, k, v, N: int, F: int, a1: int, a2: int, rows, *, o=None, mse=None, label=None,
+                            heads_per_chunk: int = 4, workspace=None, status=None, scale: float = 0.0,
+                            device=None, stream=None):
+    """svg_sparse_3d_attn on host (CPU) tensors, copies overlapped with the
+    kernels.  q, k, v (and o) should be pinned.  Returns (o, mse, label) as
+    host tensors, valid after `stream` (the current stream) synchronises."""
+    for t in (q, k, v):
+        if t.device.type != "cpu":
+            raise ValueError("svg_sparse_3d_attn_host takes host tensors")
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    rows = rows.to(torch.int32).contiguous()
+    if o is None:
+        o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if mse is None:
+        mse = torch.empty(shape.B, shape.H, 2, dtype=torch.float32, pin_memory=True)
+    if label is None:
+        label = torch.empty(shape.B, shape.H, dtype=torch.int8, pin_memory=True)
+    if workspace is None:
+        need = int(lib.svg_sparse_3d_attn_host_workspace_size(ctypes.byref(shape), rows.numel(), heads_per_chunk))
+        workspace = alloc_workspace(need, dev)
+    _check(lib.svg_sparse_3d_attn_host(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), a1, a2, _ptr(rows),
+                                       rows.numel(), _ptr(mse), _ptr(label), heads_per_chunk, _ptr(workspace),
+                                       workspace.numel(), _ptr(status), _stream(stream)))
+    return o, mse, label
 
 
 def svg_selftest_wait_bound(q, k, v, N: int, F: int, status, *, wait_ns: int = 50_000_000, o=None,

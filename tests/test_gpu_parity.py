@@ -362,3 +362,21 @@ def test_mixed_workload_sampled():
         ref = oracle.mixed_attention(qn, kn, vn, modes_np[:, h:h + 1], wl.N, wl.F, prm["window"],
                                      prm["md_half"], prm["stripe"], rows=rows)
         assert_close(f64(o[:, h:h + 1, idx]), ref, q.dtype, f"mixed head {h} mode {modes_np[0, h]}")
+
+
+# ---------------------------------------------------------------- host-buffer call
+
+@pytest.mark.parametrize("hc", [1, 3, 8])
+def test_host_pipeline_bit_identical(hc):
+    wl = synth.WORKLOADS["small"]
+    q, k, v = synth.make_qkv(wl, seed=5, device=DEV)
+    rows = torch.from_numpy(synth.sample_rows(wl.L, wl.S, 5))
+    o_dev, mse_dev, lab_dev = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows.to(DEV))
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o_h, mse_h, lab_h = svg.svg_sparse_3d_attn_host(qh, kh, vh, wl.N, wl.F, wl.a1, wl.a2, rows, heads_per_chunk=hc,
+                                                    status=status)
+    sync_ok(status)
+    assert torch.equal(o_h, o_dev.cpu())
+    assert torch.equal(mse_h, mse_dev.cpu())
+    assert torch.equal(lab_h, lab_dev.cpu())

@@ -37,7 +37,7 @@ METRIC = "ms per sparse 3D-attention call; effective TFLOPS vs bf16 peak; speedu
 # an ncu capture (profiles/attn_sm100_hunyuan.md), keyed by the sha256 prefix
 # of the kernel sources it was taken on.  Any other source revision reports
 # traffic as null until it is captured again.
-NCU_TRAFFIC = {("0fc4f35ca5f50d0f", "87c6d3d476966093"): 2.809e9}
+NCU_TRAFFIC = {("dc678c73ddaa5184", "430a4a7673ed7447"): 2.8216e9}
 
 
 def attn_source_key():
@@ -79,12 +79,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (device timings are combined this way:
+    the job is as slow as its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_ms_per_call(step_ms_per_rank: float, world: int) -> float:
+    """Whole-job ms per call: every rank runs one independent call per step, so
+    the job completes `world` calls in the slowest rank's step time."""
+    return max_over_ranks(step_ms_per_rank, world) / world
 
 
 # ---------------------------------------------------------------- clocks
@@ -328,7 +337,7 @@ def run_ours(args, wl, rank, world, local):
         raise RuntimeError(f"device status word {int(status.item())} after the timed region")
     step_ms = max_over_ranks(step_ms_local, world)
     kern_ms = {n: acc[n] / args.steps for n in acc}
-    value = step_ms / world  # ms per call, whole job (world calls per step)
+    value = step_ms / world  # ms per call, whole job (world calls per step): job_ms_per_call
 
     # dense reference on the same inputs (speedup vs dense), outside the timed region
     dense_ms = None

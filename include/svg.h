@@ -358,6 +358,32 @@ SVG_API svg_status svg_mixed_3d_attn(const svg_shape* shape, const void* q, cons
                                      void* stream);
 
 /*
+ * svg_mode_search_workspace_size -- workspace of svg_mode_search (bytes; 0 on
+ * bad arguments).
+ */
+SVG_API size_t svg_mode_search_workspace_size(const svg_shape* shape, int32_t S);
+
+/*
+ * svg_mode_search -- per-head mode selection of the mixed sparse patterns
+ * ("Sparse-vDiT" review, "What carries the argument" and the referee report
+ * on Sec. 4.2, Eq. (2)).  For each head and each sparse mode i in (skip,
+ * diagonal, multi-diagonal, vertical stripe):
+ *   L_i = MSE(O_i - O_dense) + lambda * (1 - S_i),
+ * where the MSE is over the sampled rows and d (as in svg_profile_heads), O_i
+ * is the attention under mode i (zero for skip), and S_i is the share of
+ * (query, key) pairs the mode skips (1 for skip).  The head gets the mode with
+ * the smallest L_i, or SVG_MODE_FULL if every L_i exceeds epsilon.
+ * loss: device float [B,H,4] in the order skip, diagonal, multi-diagonal,
+ * stripe.  mode: device int8 [B,H] (SVG_MODE_*; -1 if a device-side wait ran
+ * out or in-band weights underflowed, with the losses set to NaN).
+ * bf16 only; other arguments as for svg_profile_heads and svg_mixed_attn.
+ */
+SVG_API svg_status svg_mode_search(const svg_shape* shape, const void* q, const void* k, const void* v,
+                                   const int32_t* rows, int32_t S, int32_t window, int32_t md_half,
+                                   int32_t stripe, float lambda, float epsilon, float* loss, int8_t* mode,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * svg_selftest_wait_bound -- failure-detection self-test (test hook).
  *
  * Runs the bf16 attention kernel (one band covering all keys) with its

@@ -347,3 +347,55 @@ def mixed_attention(q, k, v, modes, N: int, F: int, window: int, md_half: int, s
                 np.asarray(v[b, h], np.float64), all_rows,
                 lambda rr, m=m: mode_mask(m, N, F, window, md_half, stripe, rr), scale)
     return out
+
+
+# --------------------------------------------------------------------------
+# offline mode search  [SvDiT: "What carries the argument"; referee report on
+# Sec. 4.2, Eq. (2)]
+# --------------------------------------------------------------------------
+
+SEARCH_MODES = (MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE)
+
+
+def mode_sparsity(mode: int, N: int, F: int, window: int, md_half: int, stripe: int) -> float:
+    """Share of the L*L (query, key) pairs a mode does not compute, counted
+    from its mask (one row at a time)."""
+    L = N * F
+    if mode == MODE_SKIP:
+        return 1.0
+    kept = 0
+    for r0 in range(0, L, 512):
+        rows = np.arange(r0, min(L, r0 + 512))
+        kept += int(mode_mask(mode, N, F, window, md_half, stripe, rows).sum())
+    return 1.0 - kept / float(L * L)
+
+
+def mode_search(q, k, v, N: int, F: int, rows, window: int, md_half: int, stripe: int, lam: float = 0.5,
+                eps: float = 1.0, scale=None, sparsity=None):
+    """Per head and sparse mode i: L_i = MSE(O_i - O_dense) + lam * (1 - S_i)
+    over the sampled rows; the head takes the smallest L_i unless all exceed
+    eps (then full attention).  Returns loss [B, H, 4] (skip, diagonal,
+    multi-diagonal, stripe) and mode [B, H].  Readings: Eq. (2)'s
+    lam * (1 - S_i) (not the pseudocode's lam * S_i); eps compared with L_i;
+    the MSE estimated on the sampled rows."""
+    q = np.asarray(q)
+    B, H, L, d = q.shape
+    rows = np.asarray(rows)
+    if sparsity is None:
+        sparsity = [mode_sparsity(m, N, F, window, md_half, stripe) for m in SEARCH_MODES]
+    loss = np.zeros((B, H, 4))
+    mode = np.zeros((B, H), dtype=np.int8)
+    for b in range(B):
+        for h in range(H):
+            qr = np.asarray(q[b, h], np.float64)[rows]
+            kh, vh = np.asarray(k[b, h], np.float64), np.asarray(v[b, h], np.float64)
+            o_dense = attention(qr, kh, vh, None, scale)
+            for t, m in enumerate(SEARCH_MODES):
+                if m == MODE_SKIP:
+                    o_m = np.zeros_like(o_dense)
+                else:
+                    o_m = attention(qr, kh, vh, mode_mask(m, N, F, window, md_half, stripe, rows), scale)
+                loss[b, h, t] = np.mean((o_m - o_dense) ** 2) + lam * (1.0 - sparsity[t])
+            best = int(np.argmin(loss[b, h]))
+            mode[b, h] = MODE_FULL if loss[b, h, best] > eps else SEARCH_MODES[best]
+    return loss, mode

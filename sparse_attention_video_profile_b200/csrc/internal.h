@@ -65,7 +65,7 @@ struct ProfileLayout {
   int chunk;      // keys per chunk (multiple of 64)
   size_t o_bytes;     // partial outputs  [BH][n_chunks][3][S_pad][d] f32
   size_t ml_bytes;    // partial max/sum  [BH][n_chunks][3][S_pad][2] f32
-  size_t part_bytes;  // per-row squared-difference sums [BH][S_pad][2] f64
+  size_t part_bytes;  // per-row sums [BH][S_pad][3] f64: (O_1 - O_d)^2, (O_2 - O_d)^2, O_d^2
   size_t total;
 };
 
@@ -78,10 +78,32 @@ svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float sc
                           float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
                           cudaStream_t stream);
 
-// bf16 stage 1 of profiling on the tensor cores (profile_sm100.cu).
+// Masks of the two restricted variants of a profiling pass.
+constexpr int kProfFrameBand = 0;     // |i_x - i_y| < a           (spatial)
+constexpr int kProfPositionBand = 1;  // |j_x - j_y| < a           (temporal, multi-diagonal)
+constexpr int kProfWindow = 2;        // |x - y| <= a              (diagonal)
+constexpr int kProfPrefix = 3;        // y < a                     (vertical stripe)
+constexpr int kProfNone = 4;          // no key
+
+// bf16 stage 1 of profiling on the tensor cores (profile_sm100.cu): dense and
+// two restricted variants (kind[v], par[v]) of the sampled rows' attention.
 svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const void* q, const void* k,
-                                const void* v, int a1, int a2, const int32_t* rows, int S, float* ws_o,
-                                float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream);
+                                const void* v, const int (&kind)[2], const int (&par)[2], const int32_t* rows, int S,
+                                float* ws_o, float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream);
+
+// One profiling pass: stage 1 with the given variants, then the per-row sums
+// part[bh][s][3] = {sum (O_1 - O_d)^2, sum (O_2 - O_d)^2, sum O_d^2} over d.
+svg_status launch_profile_pass(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
+                               const void* k, const void* v, const int (&kind)[2], const int (&par)[2],
+                               const int32_t* rows, int S, void* ws, const ProfileLayout& lay, double* part,
+                               int* status, cudaStream_t stream);
+
+// Sparse-vDiT mode search: two passes (diagonal, multi-diagonal) and (stripe,
+// none) plus the selection kernel.  part2 holds the second pass's sums.
+svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, const void* q, const void* k,
+                              const void* v, const int32_t* rows, int S, int window, int md_half, int stripe,
+                              float lambda, float epsilon, float* loss, int8_t* mode, void* ws,
+                              const ProfileLayout& lay, double* part2, cudaStream_t stream);
 
 // A zeroed per-device status word for kernels whose entry point takes none.
 svg_status internal_status_word(int** out, cudaStream_t stream);

@@ -136,9 +136,9 @@ constexpr int kCombineThreads = 128;
 __global__ void __launch_bounds__(kCombineThreads)
     profile_combine_rows_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int S_pad, int D,
                                 int nch, double* __restrict__ part) {
-  __shared__ double red[2][kCombineThreads / 32];
+  __shared__ double red[3][kCombineThreads / 32];
   const int s = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-  double dsq = 0.0, dtq = 0.0;
+  double dsq = 0.0, dtq = 0.0, ddq = 0.0;
   if (c < D) {
     float ov[3];
 #pragma unroll
@@ -165,26 +165,31 @@ __global__ void __launch_bounds__(kCombineThreads)
     const double dtp = static_cast<double>(ov[2]) - ov[0];
     dsq = dsp * dsp;
     dtq = dtp * dtp;
+    ddq = static_cast<double>(ov[0]) * ov[0];
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     dsq += __shfl_xor_sync(0xffffffffu, dsq, off);
     dtq += __shfl_xor_sync(0xffffffffu, dtq, off);
+    ddq += __shfl_xor_sync(0xffffffffu, ddq, off);
   }
   if ((c & 31) == 0) {
     red[0][c >> 5] = dsq;
     red[1][c >> 5] = dtq;
+    red[2][c >> 5] = ddq;
   }
   __syncthreads();
   if (c == 0) {
-    double a = 0.0, b = 0.0;
+    double a = 0.0, b = 0.0, cc = 0.0;
 #pragma unroll
     for (int w = 0; w < kCombineThreads / 32; ++w) {
       a += red[0][w];
       b += red[1][w];
+      cc += red[2][w];
     }
-    part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 0] = a;
-    part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 1] = b;
+    part[(static_cast<size_t>(bh) * S_pad + s) * 3 + 0] = a;
+    part[(static_cast<size_t>(bh) * S_pad + s) * 3 + 1] = b;
+    part[(static_cast<size_t>(bh) * S_pad + s) * 3 + 2] = cc;
   }
 }
 
@@ -197,8 +202,8 @@ __global__ void __launch_bounds__(kCombineThreads)
   const int bh = blockIdx.x;
   double a = 0.0, b = 0.0;
   for (int s = threadIdx.x; s < S; s += kCombineThreads) {
-    a += part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 0];
-    b += part[(static_cast<size_t>(bh) * S_pad + s) * 2 + 1];
+    a += part[(static_cast<size_t>(bh) * S_pad + s) * 3 + 0];
+    b += part[(static_cast<size_t>(bh) * S_pad + s) * 3 + 1];
   }
   red[0][threadIdx.x] = a;
   red[1][threadIdx.x] = b;
@@ -217,6 +222,59 @@ __global__ void __launch_bounds__(kCombineThreads)
     mse[bh * 2 + 0] = failed ? __int_as_float(0x7fc00000) : ms;
     mse[bh * 2 + 1] = failed ? __int_as_float(0x7fc00000) : mt;
     label[bh] = failed ? static_cast<int8_t>(-1) : ((mt < ms) ? SVG_TEMPORAL : SVG_SPATIAL);
+  }
+}
+
+// Sparse-vDiT mode selection, one block per head ("Sparse-vDiT" review,
+// "What carries the argument" and the referee report on Sec. 4.2, Eq. (2)):
+// for each sparse mode i (skip, diagonal, multi-diagonal, stripe),
+//   L_i = MSE(O_i - O_dense) + lambda * (1 - S_i),
+// S_i the mode's sparsity (the share of (query, key) pairs it does not
+// compute; 1 for skip).  The mode with the smallest L_i wins unless every
+// L_i exceeds epsilon, in which case the head keeps full attention.  The
+// MSEs are over the sampled rows and d, like the online profiling's.
+__global__ void __launch_bounds__(kCombineThreads)
+    mode_search_kernel(const double* __restrict__ part1, const double* __restrict__ part2, int S, int S_pad, int D,
+                       float4 sparsity, float lambda, float epsilon, float* __restrict__ loss,
+                       int8_t* __restrict__ mode, const int* __restrict__ status) {
+  __shared__ double red[4][kCombineThreads];
+  const int bh = blockIdx.x;
+  double sdiag = 0.0, smd = 0.0, sskip = 0.0, sstripe = 0.0;
+  for (int s = threadIdx.x; s < S; s += kCombineThreads) {
+    const size_t r = (static_cast<size_t>(bh) * S_pad + s) * 3;
+    sdiag += part1[r + 0];
+    smd += part1[r + 1];
+    sskip += part1[r + 2];
+    sstripe += part2[r + 0];
+  }
+  red[0][threadIdx.x] = sskip;
+  red[1][threadIdx.x] = sdiag;
+  red[2][threadIdx.x] = smd;
+  red[3][threadIdx.x] = sstripe;
+  __syncthreads();
+  for (int w = kCombineThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) red[q][threadIdx.x] += red[q][threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double n = static_cast<double>(S) * D;
+    const float sp[4] = {sparsity.x, sparsity.y, sparsity.z, sparsity.w};  // skip, diagonal, multi-diag, stripe
+    const int modes[4] = {SVG_MODE_SKIP, SVG_MODE_DIAGONAL, SVG_MODE_MULTIDIAG, SVG_MODE_STRIPE};
+    const bool failed = status != nullptr && (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE));
+    int best = -1;
+    float best_l = 0.f;
+    for (int q = 0; q < 4; ++q) {
+      const float li = static_cast<float>(red[q][0] / n) + lambda * (1.f - sp[q]);
+      loss[bh * 4 + q] = failed ? __int_as_float(0x7fc00000) : li;
+      if (best < 0 || li < best_l) {
+        best = q;
+        best_l = li;
+      }
+    }
+    mode[bh] = failed ? static_cast<int8_t>(-1)
+                      : static_cast<int8_t>(best_l > epsilon ? SVG_MODE_FULL : modes[best]);
   }
 }
 
@@ -264,16 +322,16 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
   const size_t rows_total = static_cast<size_t>(B) * H * lay.n_chunks * 3 * lay.S_pad;
   lay.o_bytes = (rows_total * d * sizeof(float) + 255) / 256 * 256;
   lay.ml_bytes = (rows_total * 2 * sizeof(float) + 255) / 256 * 256;
-  lay.part_bytes = (static_cast<size_t>(B) * H * lay.S_pad * 2 * sizeof(double) + 255) / 256 * 256;
+  lay.part_bytes = (static_cast<size_t>(B) * H * lay.S_pad * 3 * sizeof(double) + 255) / 256 * 256;
   lay.total = lay.o_bytes + lay.ml_bytes + lay.part_bytes;
   *out = lay;
   return true;
 }
 
-svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
-                          const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
-                          float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
-                          cudaStream_t stream) {
+svg_status launch_profile_pass(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
+                               const void* k, const void* v, const int (&kind)[2], const int (&par)[2],
+                               const int32_t* rows, int S, void* ws, const ProfileLayout& lay, double* part,
+                               int* status, cudaStream_t stream) {
   ProfParams p{};
   p.q = q;
   p.k = k;
@@ -289,30 +347,72 @@ svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float sc
   p.S_pad = lay.S_pad;
   p.nch = lay.n_chunks;
   p.chunk = lay.chunk;
-  p.a1 = a1;
-  p.a2 = a2;
+  p.a1 = par[0];
+  p.a2 = par[1];
   p.sl2 = scale * 1.4426950408889634f;
   if (p.BH > 65535) return fail(SVG_ERR_UNSUPPORTED, "B*H = %d exceeds the grid limit", p.BH);
-  int* status = nullptr;
-  svg_status st = internal_status_word(&status, stream);
-  if (st != SVG_OK) return st;
+  svg_status st;
   if (dtype == SVG_BF16) {
-    st = launch_profile_sm100(p.BH, N, F, d, scale, q, k, v, a1, a2, rows, S, p.ws_o, p.ws_ml, lay.n_chunks,
+    st = launch_profile_sm100(p.BH, N, F, d, scale, q, k, v, kind, par, rows, S, p.ws_o, p.ws_ml, lay.n_chunks,
                               lay.chunk, status, stream);
   } else {
+    if (kind[0] != kProfFrameBand || kind[1] != kProfPositionBand)
+      return fail(SVG_ERR_UNSUPPORTED, "fp32 profiling supports the spatial / temporal pair only");
     if (d == 32) st = launch_stage1_f32<32>(p, stream);
     else if (d == 64) st = launch_stage1_f32<64>(p, stream);
     else if (d == 128) st = launch_stage1_f32<128>(p, stream);
     else return fail(SVG_ERR_UNSUPPORTED, "fp32 profiling supports d in {32, 64, 128}, got %d", d);
   }
   if (st != SVG_OK) return st;
-  double* part = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
   profile_combine_rows_kernel<<<dim3(S, p.BH), kCombineThreads, 0, stream>>>(p.ws_o, p.ws_ml, lay.S_pad, d,
                                                                               lay.n_chunks, part);
-  st = cuda_check(cudaGetLastError(), "profile combine launch");
+  return cuda_check(cudaGetLastError(), "profile combine launch");
+}
+
+svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
+                          const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
+                          float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
+                          cudaStream_t stream) {
+  int* status = nullptr;
+  svg_status st = internal_status_word(&status, stream);
   if (st != SVG_OK) return st;
-  profile_finalize_kernel<<<p.BH, kCombineThreads, 0, stream>>>(part, S, lay.S_pad, d, mse, label, status);
+  double* part = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
+  const int kind[2] = {kProfFrameBand, kProfPositionBand}, par[2] = {a1, a2};
+  if ((st = launch_profile_pass(B, H, N, F, d, dtype, scale, q, k, v, kind, par, rows, S, ws, lay, part, status,
+                                stream)) != SVG_OK)
+    return st;
+  profile_finalize_kernel<<<B * H, kCombineThreads, 0, stream>>>(part, S, lay.S_pad, d, mse, label, status);
   return cuda_check(cudaGetLastError(), "profile finalize launch");
+}
+
+svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, const void* q, const void* k,
+                              const void* v, const int32_t* rows, int S, int window, int md_half, int stripe,
+                              float lambda, float epsilon, float* loss, int8_t* mode, void* ws,
+                              const ProfileLayout& lay, double* part2, cudaStream_t stream) {
+  int* status = nullptr;
+  svg_status st = internal_status_word(&status, stream);
+  if (st != SVG_OK) return st;
+  double* part1 = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
+  const int kind1[2] = {kProfWindow, kProfPositionBand}, par1[2] = {window, md_half + 1};
+  const int kind2[2] = {kProfPrefix, kProfNone}, par2[2] = {stripe, 0};
+  if ((st = launch_profile_pass(B, H, N, F, d, SVG_BF16, scale, q, k, v, kind1, par1, rows, S, ws, lay, part1,
+                                status, stream)) != SVG_OK)
+    return st;
+  if ((st = launch_profile_pass(B, H, N, F, d, SVG_BF16, scale, q, k, v, kind2, par2, rows, S, ws, lay, part2,
+                                status, stream)) != SVG_OK)
+    return st;
+  // sparsity of each mode: 1 - kept pairs / L^2 (closed forms of the masks)
+  const double L = static_cast<double>(N) * F;
+  const double W = window < L - 1 ? window : L - 1;
+  const double a = (md_half + 1 < F) ? md_half + 1 : F;
+  const double Pn = stripe < L ? stripe : L;
+  const double diag_pairs = L * (2 * W + 1) - W * (W + 1);
+  const double md_pairs = static_cast<double>(N) * N * (F * (2 * a - 1) - a * (a - 1));
+  const float4 sparsity = make_float4(1.f, static_cast<float>(1.0 - diag_pairs / (L * L)),
+                                      static_cast<float>(1.0 - md_pairs / (L * L)), static_cast<float>(1.0 - Pn / L));
+  mode_search_kernel<<<B * H, kCombineThreads, 0, stream>>>(part1, part2, S, lay.S_pad, d, sparsity, lambda, epsilon,
+                                                            loss, mode, status);
+  return cuda_check(cudaGetLastError(), "mode search launch");
 }
 
 }  // namespace svg

@@ -35,7 +35,7 @@ struct ProfSm100Params {
   float* ws_o;   // [BH][nch][3][128][D]
   float* ws_ml;  // [BH][nch][3][128][2]  (max in log2 units, sum)
   int BH, L, N, F, S, nch, chunk;
-  int a1, a2;
+  int kind[2], par[2];  // masks of the two restricted variants (ProfMaskKind)
   float sl2;
   float lazy_th;
   int* status;
@@ -43,6 +43,9 @@ struct ProfSm100Params {
 };
 
 namespace {
+
+// Masks of the restricted variants.
+enum ProfMaskKind { kMaskFrameBand = 0, kMaskPositionBand = 1, kMaskWindow = 2, kMaskPrefix = 3, kMaskNone = 4 };
 
 template <int D>
 struct PCfg {
@@ -253,8 +256,24 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
       mbar_arrive(bar_q);
     }
     const int ir = x / p.F, jr = x - (x / p.F) * p.F;
-    const int lo_s = max(0, (ir - p.a1 + 1) * p.F);
-    const int hi_s = min(p.L, (ir + p.a1) * p.F);
+    // each restricted variant keeps one key interval of this row, except the
+    // in-frame-position band, which keeps a window in every frame
+    int lo_v[2], hi_v[2];
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int kind = p.kind[v], a = p.par[v];
+      lo_v[v] = 0;
+      hi_v[v] = 0;
+      if (kind == kMaskFrameBand) {
+        lo_v[v] = max(0, (ir - a + 1) * p.F);
+        hi_v[v] = min(p.L, (ir + a) * p.F);
+      } else if (kind == kMaskWindow) {
+        lo_v[v] = max(0, x - a);
+        hi_v[v] = min(p.L, x + a + 1);
+      } else if (kind == kMaskPrefix) {
+        hi_v[v] = min(p.L, a);
+      }
+    }
     const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::COL_S;
     const float sl2 = p.sl2;
@@ -283,21 +302,28 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
 
       const int kbase = (kt0 + k) * 128;
       const int nvalid = min(128, y_end - kbase);  // keys of this chunk in the tile
-      // Key masks of the tile: dense (chunk end), spatial (one key interval
-      // of frames), temporal (|j - j_r| < a2 within each frame segment).
+      // Key masks of the tile: dense (chunk end); each restricted variant
+      // either one key interval or, for the in-frame-position band, |j - j_r| < a
+      // within each frame segment of the tile.
       uint32_t md[4] = {0u, 0u, 0u, 0u}, ms[4] = {0u, 0u, 0u, 0u}, mt[4] = {0u, 0u, 0u, 0u};
       set_range128(md, 0, nvalid);
-      set_range128(ms, max(lo_s - kbase, 0), min(hi_s - kbase, nvalid));
-      {
-        int c = 0;
-        int j0 = kbase % p.F;
-        while (c < nvalid) {  // one frame segment per pass: keys c .. c + (F - j0) - 1
-          const int seg_end = min(nvalid, c + (p.F - j0));
-          const int lo = max(c, c + (jr - p.a2 + 1 - j0));
-          const int hi = min(seg_end, c + (jr + p.a2 - j0));
-          if (lo < hi) set_range128(mt, lo, hi);
-          c = seg_end;
-          j0 = 0;
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        uint32_t(&mv)[4] = v ? mt : ms;
+        if (p.kind[v] == kMaskPositionBand) {
+          const int a = p.par[v];
+          int c = 0;
+          int j0 = kbase % p.F;
+          while (c < nvalid) {  // one frame segment per pass: keys c .. c + (F - j0) - 1
+            const int seg_end = min(nvalid, c + (p.F - j0));
+            const int lo = max(c, c + (jr - a + 1 - j0));
+            const int hi = min(seg_end, c + (jr + a - j0));
+            if (lo < hi) set_range128(mv, lo, hi);
+            c = seg_end;
+            j0 = 0;
+          }
+        } else {
+          set_range128(mv, max(lo_v[v] - kbase, 0), min(hi_v[v] - kbase, nvalid));
         }
       }
       // one max over the kept keys; every variant uses it as its reference
@@ -436,8 +462,8 @@ svg_status launch_profile_sm100_d(ProfSm100Params& p, const void* k, const void*
 }
 
 svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const void* q, const void* k,
-                                const void* v, int a1, int a2, const int32_t* rows, int S, float* ws_o,
-                                float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream) {
+                                const void* v, const int (&kind)[2], const int (&par)[2], const int32_t* rows, int S,
+                                float* ws_o, float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream) {
   ProfSm100Params p;
   memset(&p, 0, sizeof(p));
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -451,8 +477,10 @@ svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const 
   p.S = S;
   p.nch = nch;
   p.chunk = chunk;
-  p.a1 = a1;
-  p.a2 = a2;
+  for (int i = 0; i < 2; ++i) {
+    p.kind[i] = kind[i];
+    p.par[i] = par[i];
+  }
   p.sl2 = scale * 1.4426950408889634f;
   p.lazy_th = 8.0f / p.sl2;
   p.status = status;

@@ -395,6 +395,37 @@ svg_status svg_mixed_3d_attn(const svg_shape* shape, const void* q, const void* 
   return launch_permute(1, src1, dst1, BH, shape->N, shape->F, rb, mode, false, s, SVG_MODE_MULTIDIAG);
 }
 
+size_t svg_mode_search_workspace_size(const svg_shape* shape, int32_t S) {
+  if (check_shape(shape) != SVG_OK || shape->dtype != SVG_BF16) return 0;
+  ProfileLayout lay;
+  if (!profile_layout(shape->B, shape->H, shape->N * shape->F, shape->d, shape->dtype, S, &lay)) return 0;
+  return lay.total + lay.part_bytes;
+}
+
+svg_status svg_mode_search(const svg_shape* shape, const void* q, const void* k, const void* v, const int32_t* rows,
+                           int32_t S, int32_t window, int32_t md_half, int32_t stripe, float lambda, float epsilon,
+                           float* loss, int8_t* mode, void* workspace, size_t workspace_bytes, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "the mode search runs in bf16 only");
+  if ((st = check_tensors({q, k, v})) != SVG_OK) return st;
+  if (!rows || !loss || !mode || !workspace) return fail(SVG_ERR_INVALID_ARG, "NULL rows/loss/mode/workspace");
+  if (window < 0 || md_half < 0 || stripe < 1) return fail(SVG_ERR_INVALID_ARG, "window, md_half >= 0 and stripe >= 1");
+  if (!(lambda >= 0.f) || !(epsilon >= 0.f)) return fail(SVG_ERR_INVALID_ARG, "lambda and epsilon must be >= 0");
+  const int L = shape->N * shape->F;
+  if (S < 1 || S > 128 || S > L) return fail(SVG_ERR_INVALID_ARG, "S must be in [1, min(128, L)], got %d", S);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  ProfileLayout lay;
+  profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay);
+  if (workspace_bytes < lay.total + lay.part_bytes)
+    return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, lay.total + lay.part_bytes);
+  double* part2 = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + lay.total);
+  return launch_mode_search(shape->B, shape->H, shape->N, shape->F, shape->d, eff_scale(shape), q, k, v, rows, S,
+                            window < L ? window : L, md_half < shape->F ? md_half : shape->F, stripe < L ? stripe : L,
+                            lambda, epsilon, loss, mode, workspace, lay, part2, static_cast<cudaStream_t>(stream));
+}
+
 svg_status svg_selftest_wait_bound(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
                                    uint64_t wait_ns, int32_t* status_dev, void* stream) {
   svg_status st = check_shape(shape);

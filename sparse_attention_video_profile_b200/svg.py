@@ -36,7 +36,7 @@ EXPORTED = (
     "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
     "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
     "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
-    "svg_sparse_3d_attn_host",
+    "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -87,6 +87,9 @@ def _load() -> ctypes.CDLL:
         "svg_mixed_3d_attn": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _Z, _P, _P]),
         "svg_sparse_3d_attn_host_workspace_size": (_Z, [_P, _I, _I]),
         "svg_sparse_3d_attn_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _I, _P, _Z, _P, _P]),
+        "svg_mode_search_workspace_size": (_Z, [_P, _I]),
+        "svg_mode_search": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _Z,
+                                 _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -351,6 +354,25 @@ def svg_sparse_3d_attn_host(q, k, v, N: int, F: int, a1: int, a2: int, rows, *, 
                                        rows.numel(), _ptr(mse), _ptr(label), heads_per_chunk, _ptr(workspace),
                                        workspace.numel(), _ptr(status), _stream(stream)))
     return o, mse, label
+
+
+def svg_mode_search(q, k, v, N: int, F: int, rows, window: int, md_half: int, stripe: int, *, lam: float = 0.5,
+                    epsilon: float = 1.0, loss=None, mode=None, workspace=None, scale: float = 0.0, stream=None):
+    """Sparse-vDiT mode selection per head.  Returns (loss [B,H,4]: skip,
+    diagonal, multi-diagonal, stripe; mode [B,H] int8 SVG_MODE_*)."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if loss is None:
+        loss = torch.empty(shape.B, shape.H, 4, dtype=torch.float32, device=q.device)
+    if mode is None:
+        mode = torch.empty(shape.B, shape.H, dtype=torch.int8, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(int(lib.svg_mode_search_workspace_size(ctypes.byref(shape), rows.numel())),
+                                    q.device)
+    _check(lib.svg_mode_search(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(rows), rows.numel(), window,
+                               md_half, stripe, float(lam), float(epsilon), _ptr(loss), _ptr(mode), _ptr(workspace),
+                               workspace.numel(), _stream(stream)))
+    return loss, mode
 
 
 def svg_selftest_wait_bound(q, k, v, N: int, F: int, status, *, wait_ns: int = 50_000_000, o=None,

@@ -380,3 +380,83 @@ def test_host_pipeline_bit_identical(hc):
     assert torch.equal(o_h, o_dev.cpu())
     assert torch.equal(mse_h, mse_dev.cpu())
     assert torch.equal(lab_h, lab_dev.cpu())
+
+
+# ---------------------------------------------------------------- offline mode search
+
+def check_mode_search(loss, mode, ref_loss, ref_mode, sp, lam, eps):
+    """Losses as RMS distances of their MSE parts (tolerance as for the
+    profiling MSEs); modes equal wherever the oracle's decision has a margin
+    larger than the MSE error that tolerance allows."""
+    loss = loss.cpu().numpy().astype(np.float64)
+    mode = mode.cpu().numpy()
+    assert np.all(np.isfinite(loss))
+    pen = lam * (1.0 - np.asarray(sp))
+    mse, ref_mse = np.maximum(loss - pen, 0.0), ref_loss - pen
+    dist = np.abs(np.sqrt(mse) - np.sqrt(ref_mse))
+    assert dist.max() <= RMS_TOL[torch.bfloat16], f"rms distance {dist.max():.3e}"
+    delta = RMS_TOL[torch.bfloat16]
+    err = delta * (2 * np.sqrt(ref_mse.max(-1)) + delta)  # bound on |mse_gpu - mse_ref|
+    srt = np.sort(ref_loss, -1)
+    decided = (srt[..., 1] - srt[..., 0] > 2 * err) & (np.abs(srt[..., 0] - eps) > err)
+    np.testing.assert_array_equal(mode[decided], ref_mode[decided])
+    assert np.all(np.isin(mode, [0, 1, 2, 3, 4]))
+    return decided
+
+
+def test_mode_search_structured():
+    """Attention one-hot on the key one mode keeps: that mode must win."""
+    N, F, d = 2, 32, 64
+    L = N * F
+    targets = [lambda x: x, lambda x: ((x // F + 1) % N) * F + x % F, lambda x: 0]
+    q = torch.zeros(1, 3, L, d)
+    k = torch.eye(L, d).expand(1, 3, L, d).contiguous()
+    for h, t in enumerate(targets):
+        for x in range(L):
+            q[0, h, x, t(x)] = 40.0 * 8.0  # logit 40 after the 1/sqrt(d) scale
+    v = torch.randn(1, 3, L, d, generator=torch.Generator().manual_seed(3))
+    q, k, v = (t.to(torch.bfloat16).to(DEV) for t in (q, k, v))
+    rows_np = np.arange(0, L, 3, dtype=np.int32)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    loss, mode = svg.svg_mode_search(q, k, v, N, F, rows, 0, 0, 1)
+    sync_ok()
+    ref_loss, ref_mode = oracle.mode_search(f64(q), f64(k), f64(v), N, F, rows_np, 0, 0, 1)
+    sp = [oracle.mode_sparsity(m, N, F, 0, 0, 1) for m in oracle.SEARCH_MODES]
+    check_mode_search(loss, mode, ref_loss, ref_mode, sp, 0.5, 1.0)
+    np.testing.assert_array_equal(mode.cpu().numpy()[0], [svg.MODE_DIAGONAL, svg.MODE_MULTIDIAG, svg.MODE_STRIPE])
+    _, mode = svg.svg_mode_search(q, k, v, N, F, rows, 0, 0, 1, epsilon=0.005)  # every L_i >= lam / L = 0.0078
+    sync_ok()
+    assert torch.all(mode == svg.MODE_FULL)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("S", [17, 128])
+def test_mode_search_random(d, S):
+    N, F, W, h, P = 6, 90, 90, 7, 100
+    L = N * F
+    q, k, v = rand_qkv(2, 3, L, d, torch.bfloat16, 40 + S)
+    rows_np = np.sort(np.random.default_rng(S).choice(L, S, replace=False)).astype(np.int32)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    for lam, eps in [(0.5, 1.0), (0.05, 0.3)]:
+        loss, mode = svg.svg_mode_search(q, k, v, N, F, rows, W, h, P, lam=lam, epsilon=eps)
+        sync_ok()
+        ref_loss, ref_mode = oracle.mode_search(f64(q), f64(k), f64(v), N, F, rows_np, W, h, P, lam=lam, eps=eps)
+        sp = [oracle.mode_sparsity(m, N, F, W, h, P) for m in oracle.SEARCH_MODES]
+        check_mode_search(loss, mode, ref_loss, ref_mode, sp, lam, eps)
+
+
+def test_mode_search_mixed_workload():
+    wl = synth.WORKLOADS["mixed"]
+    prm = synth.MIXED_PARAMS
+    q, k, v = synth.make_qkv(wl, seed=0, device=DEV)
+    rows_np = synth.sample_rows(wl.L, wl.S, 0)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    args = (wl.N, wl.F, prm["window"], prm["md_half"], prm["stripe"])
+    loss, mode = svg.svg_mode_search(q, k, v, wl.N, wl.F, rows, *args[2:])
+    loss2, mode2 = svg.svg_mode_search(q, k, v, wl.N, wl.F, rows, *args[2:])
+    sync_ok()
+    assert torch.equal(loss, loss2) and torch.equal(mode, mode2)  # deterministic
+    sp = [oracle.mode_sparsity(m, *args) for m in oracle.SEARCH_MODES]
+    ref_loss, ref_mode = oracle.mode_search(f64(q), f64(k), f64(v), wl.N, wl.F, rows_np, *args[2:], sparsity=sp)
+    decided = check_mode_search(loss, mode, ref_loss, ref_mode, sp, 0.5, 1.0)
+    assert decided.mean() > 0.5

@@ -363,3 +363,82 @@ def test_mixed_attention_modes():
     qp, kp, vp = (oracle.permute(t[0, 3], N, F) for t in (q, k, v))
     via = oracle.unpermute(oracle.attention(qp, kp, vp, oracle.banded_mask(N * F, N, 2)), N, F)
     np.testing.assert_allclose(out[0, 3], via, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------ offline mode search pins
+
+@pytest.mark.parametrize("N,F,W,h,P", [(3, 5, 2, 1, 4), (2, 7, 20, 6, 100), (4, 4, 0, 0, 1)])
+def test_mode_sparsity_counts(N, F, W, h, P):
+    """Sparsity S_i = share of skipped pairs, against closed forms of the three
+    masks (window band, |j1 - j2| <= h over all frame pairs, first P keys)."""
+    L = N * F
+    Wc, a, Pc = min(W, L - 1), min(h + 1, F), min(P, L)
+    closed = {
+        oracle.MODE_SKIP: 1.0,
+        oracle.MODE_DIAGONAL: 1 - (L * (2 * Wc + 1) - Wc * (Wc + 1)) / L**2,
+        oracle.MODE_MULTIDIAG: 1 - N * N * (F * (2 * a - 1) - a * (a - 1)) / L**2,
+        oracle.MODE_STRIPE: 1 - Pc / L,
+    }
+    for m, s in closed.items():
+        assert oracle.mode_sparsity(m, N, F, W, h, P) == pytest.approx(s, abs=1e-15)
+
+
+def _one_hot_qkv(N, F, d, target, logit=40.0, seed=0):
+    """Keys are unit vectors e_y, query x points at key target(x) with the
+    given logit: attention is one-hot on target(x) up to exp(-logit)."""
+    L = N * F
+    k = np.eye(L, d)[None, None]
+    q = np.zeros((1, 1, L, d))
+    for x in range(L):
+        q[0, 0, x, target(x)] = logit * math.sqrt(d)
+    v = np.random.default_rng(seed).standard_normal((1, 1, L, d))
+    return q, k, v
+
+
+@pytest.mark.parametrize("which", ["diagonal", "multidiag", "stripe"])
+def test_mode_search_picks_the_exact_mode(which):
+    """Attention concentrated on the key a mode keeps: that mode has MSE ~ 0,
+    so its loss is lam * (1 - S_i); the others miss the key and pay MSE ~ 1."""
+    N, F, d, lam = 2, 3, 8, 0.5
+    L = N * F
+    target = {"diagonal": lambda x: x,
+              "multidiag": lambda x: ((x // F + 1) % N) * F + x % F,
+              "stripe": lambda x: 0}[which]
+    q, k, v = _one_hot_qkv(N, F, d, target)
+    rows = np.arange(L)
+    loss, mode = oracle.mode_search(q, k, v, N, F, rows, 0, 0, 1, lam=lam, eps=1.0)
+    sp = [oracle.mode_sparsity(m, N, F, 0, 0, 1) for m in oracle.SEARCH_MODES]
+    want = {"diagonal": oracle.MODE_DIAGONAL, "multidiag": oracle.MODE_MULTIDIAG, "stripe": oracle.MODE_STRIPE}[which]
+    t = oracle.SEARCH_MODES.index(want)
+    assert loss[0, 0, t] == pytest.approx(lam * (1 - sp[t]), abs=1e-12)
+    assert mode[0, 0] == want
+    # the skip loss is the mean square of the dense output (sparsity 1)
+    o = np.stack([v[0, 0, target(x)] for x in range(L)])
+    assert loss[0, 0, 0] == pytest.approx(np.mean(o**2), rel=1e-12)
+    # below every loss the head stays dense
+    _, mode = oracle.mode_search(q, k, v, N, F, rows, 0, 0, 1, lam=lam, eps=0.01)
+    assert mode[0, 0] == oracle.MODE_FULL
+
+
+def test_mode_search_constant_values_and_full_bands():
+    """V constant over keys: every non-skip mode reproduces the dense output,
+    so L_i = lam * (1 - S_i) and the sparsest one wins (a sign error in the
+    sparsity term would pick the densest); skip costs mean(c^2).  Bands that
+    cover every key give L_i = lam exactly."""
+    N, F, d = 3, 4, 5
+    L = N * F
+    rng = np.random.default_rng(4)
+    q, k = (rng.standard_normal((1, 2, L, d)) for _ in range(2))
+    c = np.array([3.0, -2.0, 1.0, 0.5, 2.5])
+    v = np.broadcast_to(c, (1, 2, L, d)).copy()
+    v[0, 1] *= 1e-3  # second head: output so small that skipping is cheapest
+    rows = np.array([0, 5, 11])
+    loss, mode = oracle.mode_search(q, k, v, N, F, rows, 2, 1, 3, lam=0.5, eps=10.0)
+    sp = [oracle.mode_sparsity(m, N, F, 2, 1, 3) for m in oracle.SEARCH_MODES]
+    for h in range(2):
+        np.testing.assert_allclose(loss[0, h, 1:], 0.5 * (1 - np.array(sp[1:])), atol=1e-12)
+    assert loss[0, 0, 0] == pytest.approx(np.mean(c**2), rel=1e-12)
+    assert mode[0, 0] == oracle.SEARCH_MODES[1 + int(np.argmax(sp[1:]))]
+    assert mode[0, 1] == oracle.MODE_SKIP
+    loss, _ = oracle.mode_search(q, k, rng.standard_normal((1, 2, L, d)), N, F, rows, L, F, L, lam=0.7)
+    np.testing.assert_allclose(loss[0, :, 1:], 0.7, atol=1e-12)

@@ -226,8 +226,12 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, row, bh);
       }
     }
-    } else if (run && nk > 0 && warp == 9 && lane == 0) {
+    } else if (run && nk > 0 && warp == 9) {
       // ------------------------------------------------ MMA issuer
+      // The whole warp runs this loop (waits, descriptor arithmetic) in
+      // lockstep, and one elected lane issues each tcgen05 instruction: the
+      // operands stay warp-uniform, which keeps the per-MMA issue cost low
+      // while the softmax warps on the same sub-partition keep it busy.
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t ring_base = smem_u32(sRing);
@@ -242,40 +246,40 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
-          umma_ss(tmem + C::col_s(i), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss_warp(tmem + C::col_s(i), a + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bar_s[i]);
+        umma_commit_warp(&bar_s[i]);
       };
       auto issue_pv = [&](int i, int slot, bool acc) {
         const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          umma_ts(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8, b + static_cast<uint64_t>((kk * 16 * 128) >> 4),
-                  idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        umma_commit(&bar_o[i]);
+          umma_ts_warp(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
+                       b + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        umma_commit_warp(&bar_o[i]);
       };
-      bool ok = mbar_wait(bar_q, 0, p.wait_ns) && mbar_wait(&bar_full[0], 0, p.wait_ns);
+      bool ok = warp_wait(bar_q, 0, p.wait_ns) && warp_wait(&bar_full[0], 0, p.wait_ns);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
         issue_qk(1, 0);
-        umma_commit(&bar_empty[0]);
+        umma_commit_warp(&bar_empty[0]);
       }
       for (int k = 0; ok && k < nk; ++k) {
         const int nV = 2 * k + 1, nK = 2 * k + 2;
         const int slotV = nV % C::NS, slotK = nK % C::NS;
         const bool has_next = k + 1 < nk;
-        ok = mbar_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
+        ok = warp_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
         for (int i = 0; ok && i < 2; ++i) {
-          ok = mbar_wait(&bar_p[i], k & 1, p.wait_ns);
+          ok = warp_wait(&bar_p[i], k & 1, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_pv(i, slotV, k > 0);
           // V_k is free once both tiles' P V products have read it.
-          if (i == 1) umma_commit(&bar_empty[slotV]);
+          if (i == 1) umma_commit_warp(&bar_empty[slotV]);
           if (has_next) {
             if (i == 0) {
-              ok = mbar_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+              ok = warp_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
               if (!ok) break;
               tc_fence_after();
             }
@@ -283,9 +287,9 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           }
         }
         if (!ok) break;
-        if (has_next) umma_commit(&bar_empty[slotK]);
+        if (has_next) umma_commit_warp(&bar_empty[slotK]);
       }
-      if (!ok) record_timeout(p, abort_flag);
+      if (!ok && lane == 0) record_timeout(p, abort_flag);
     }
   } else {
     if (run) {

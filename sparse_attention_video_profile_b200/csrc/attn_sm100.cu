@@ -84,6 +84,14 @@ struct Cfg {
 #endif
 constexpr int kExpPoly = SVG_EXP_POLY_PAIRS;
 
+// P_i is handed to the MMA issuer in this many column chunks: the first
+// P V products run while the softmax still computes the later keys.
+#ifndef SVG_P_CHUNKS
+#define SVG_P_CHUNKS 2
+#endif
+constexpr int kPChunks = SVG_P_CHUNKS;
+static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P chunks: 1, 2 or 4");
+
 __device__ __forceinline__ void record_timeout(const AttnParams& p, volatile int* abort_flag) {
   *abort_flag = 1;
   atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
@@ -150,8 +158,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   uint64_t* bar_full = bars + 1;
   uint64_t* bar_empty = bars + 1 + C::NS;
   uint64_t* bar_s = bars + 1 + 2 * C::NS;  // [2] S_i ready
-  uint64_t* bar_p = bar_s + 2;             // [2] P_i written (128 arrivals)
-  uint64_t* bar_o = bar_p + 2;             // [2] P_i V done
+  uint64_t* bar_p = bar_s + 2;             // [2][kPChunks] chunk of P_i written (128 arrivals)
+  uint64_t* bar_o = bar_p + 2 * kPChunks;  // [2] P_i V done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_o + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_p[i], 128);
+      for (int j = 0; j < kPChunks; ++j) mbar_init(&bar_p[i * kPChunks + j], 128);
       mbar_init(&bar_o[i], 1);
     }
     fence_barrier_init();
@@ -250,13 +258,16 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         }
         umma_commit_warp(&bar_s[i]);
       };
-      auto issue_pv = [&](int i, int slot, bool acc) {
+      // The P V products of one chunk of P_i (keys [j, j+1) * BK / kPChunks).
+      auto issue_pv_chunk = [&](int i, int slot, bool acc, int j) {
         const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
+        constexpr int KK = C::BK / 16 / kPChunks;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
+        for (int u = 0; u < KK; ++u) {
+          const int kk = j * KK + u;
           umma_ts_warp(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
                        b + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        umma_commit_warp(&bar_o[i]);
+        }
       };
       bool ok = warp_wait(bar_q, 0, p.wait_ns) && warp_wait(&bar_full[0], 0, p.wait_ns);
       if (ok) {
@@ -271,10 +282,15 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         const bool has_next = k + 1 < nk;
         ok = warp_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
         for (int i = 0; ok && i < 2; ++i) {
-          ok = warp_wait(&bar_p[i], k & 1, p.wait_ns);
+#pragma unroll
+          for (int j = 0; j < kPChunks; ++j) {
+            ok = warp_wait(&bar_p[i * kPChunks + j], k & 1, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv_chunk(i, slotV, k > 0, j);
+          }
           if (!ok) break;
-          tc_fence_after();
-          issue_pv(i, slotV, k > 0);
+          umma_commit_warp(&bar_o[i]);
           // V_k is free once both tiles' P V products have read it.
           if (i == 1) umma_commit_warp(&bar_empty[slotV]);
           if (has_next) {
@@ -349,53 +365,60 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         resc = true;
       }
       l *= alpha;
-      const float nb = (m_used == -INFINITY) ? 0.f : -m_used * sl2;
-      const float2 sl2x2 = make_float2(sl2, sl2), nb2 = make_float2(nb, nb);
-      uint32_t pk[2][32];
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
-        float2 pr;
-        if ((c & 7) < kExpPoly) {  // a fixed share of the pairs on the FMA pipe
-          pr = exp2_poly2(x);
-        } else {
-          pr.x = ex2_approx(x.x);
-          pr.y = ex2_approx(x.y);
-        }
-        const uint32_t pp = pack_bf16x2(pr.x, pr.y);
-        // The row sum uses the same bf16-rounded weights the P V product
-        // sees, so each output row is an exact convex combination of V rows.
-        const float2 pw = make_float2(bf16lo_f32(pp), bf16hi_f32(pp));
-        if (c & 1) acc1 = __fadd2_rn(acc1, pw);
-        else acc0 = __fadd2_rn(acc0, pw);
-        pk[c >> 5][c & 31] = pp;
-      }
-      l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
-      __syncwarp();
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
       if (k > 0 && __any_sync(0xffffffffu, resc)) {
-        // O_i must hold P_i(k-1) V before it is rescaled.
+        // O_i holds P_i(k-1) V (its product completed before S_i(k) did);
+        // rescale it before any P_i(k) V product is issued.
         if (!warp_wait(&bar_o[i], (k - 1) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tO + c * 32, ov);
+        // 16 columns at a time: the 128 scores stay live in registers here
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t ov[16];
+          tmem_ld16(tO + c * 16, ov);
           tmem_wait_ld();
-          reg_fence32(ov);
+          reg_fence16(ov);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(tO + c * 32, ov);
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st16(tO + c * 16, ov);
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_p[i]);
+      const float nb = (m_used == -INFINITY) ? 0.f : -m_used * sl2;
+      const float2 sl2x2 = make_float2(sl2, sl2), nb2 = make_float2(nb, nb);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      constexpr int PPC = 64 / kPChunks;  // key pairs (P columns) per chunk
+#pragma unroll
+      for (int j = 0; j < kPChunks; ++j) {
+        uint32_t pk[PPC];
+#pragma unroll
+        for (int cc = 0; cc < PPC; ++cc) {
+          const int c = j * PPC + cc;
+          const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
+          float2 pr;
+          if ((c & 7) < kExpPoly) {  // a fixed share of the pairs on the FMA pipe
+            pr = exp2_poly2(x);
+          } else {
+            pr.x = ex2_approx(x.x);
+            pr.y = ex2_approx(x.y);
+          }
+          const uint32_t pp = pack_bf16x2(pr.x, pr.y);
+          // The row sum uses the same bf16-rounded weights the P V product
+          // sees, so each output row is an exact convex combination of V rows.
+          const float2 pw = make_float2(bf16lo_f32(pp), bf16hi_f32(pp));
+          if (c & 1) acc1 = __fadd2_rn(acc1, pw);
+          else acc0 = __fadd2_rn(acc0, pw);
+          pk[cc] = pp;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < PPC / 16; ++h) tmem_st16(tS + j * PPC + h * 16, pk + h * 16);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p[i * kPChunks + j]);
+      }
+      l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
     }
     if (nk == 0) {
       // skipped head: its output rows are zero

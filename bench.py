@@ -45,6 +45,8 @@ def attn_source_key():
     csrc = os.path.join(ROOT, "sparse_attention_video_profile_b200", "csrc")
     return tuple(hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()[:16]
                  for f in ("attn_sm100.cu", "sm100.cuh"))
+# kernels one bf16 profiling call launches: tcgen05 stage 1, row combine, per-head finalize
+PROFILE_LAUNCHES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -251,7 +253,10 @@ def run_ours(args, wl, rank, world, local):
     rows = torch.from_numpy(rows_np).to(dev)
     N, F = wl.N, wl.F
     o = torch.empty_like(q)
-    qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
+    # token-major copies: only the separate layout path needs them
+    qp = kp = vp = op = None
+    if args.layout == "separate":
+        qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
     mse = torch.empty(wl.B, wl.H, 2, dtype=torch.float32, device=dev)
     label = torch.empty(wl.B, wl.H, dtype=torch.int8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -263,12 +268,24 @@ def run_ours(args, wl, rank, world, local):
         prm = synth.MIXED_PARAMS
         modes_np = synth.head_modes(wl.B, wl.H, rank)
         mode = torch.from_numpy(modes_np).to(dev)
-    names = ("permute", "attn", "unpermute") if mixed else ("profile", "permute", "attn", "unpermute")
+    fused = args.layout == "fused"
+    if mixed:
+        names = ("attn",) if fused else ("permute", "attn", "unpermute")
+    else:
+        names = ("profile", "attn") if fused else ("profile", "permute", "attn", "unpermute")
 
     def new_events():
         return {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
 
     def step_mixed(e=None):
+        if fused:
+            if e:
+                e["attn"][0].record(stream)
+            svg.svg_mixed_attn_fused(q, k, v, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
+                                     status=status)
+            if e:
+                e["attn"][1].record(stream)
+            return
         if e:
             e["permute"][0].record(stream)
         svg.svg_permute_qkv(q, k, v, N, F, md_label, out=(qp, kp, vp))
@@ -290,6 +307,14 @@ def run_ours(args, wl, rank, world, local):
         if e:
             e["profile"][0].record(stream)
         svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws)
+        if fused:
+            if e:
+                e["profile"][1].record(stream)
+                e["attn"][0].record(stream)
+            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status)
+            if e:
+                e["attn"][1].record(stream)
+            return
         if e:
             e["profile"][1].record(stream)
             e["permute"][0].record(stream)
@@ -439,8 +464,10 @@ def run_ours(args, wl, rank, world, local):
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
         "dense_ms": dense_ms,
         "kernel_ms": kern_ms,
-        "permute_gbs": perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal else None,
-        "unpermute_gbs": unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal else None,
+        "layout": ("fused: token-major heads gathered by the attention kernel, no permuted copies" if fused else
+                   "separate: permute -> attention -> unpermute"),
+        "permute_gbs": perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
+        "unpermute_gbs": unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
         "temporal_heads": n_temporal,
         "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
@@ -450,7 +477,7 @@ def run_ours(args, wl, rank, world, local):
         "hbm_peak_gbs": hbm,
         "clocks": clocks.summary(),
         "e2e": e2e,
-        "gpu_launches": (3 if mixed else 5) * args.steps,
+        "gpu_launches": len(names) * args.steps + (0 if mixed else (PROFILE_LAUNCHES - 1) * args.steps),
         "cpu_baseline": cpu,
     }
     if mode_search is not None:
@@ -469,6 +496,8 @@ def main():
     ap.add_argument("--density", type=float, default=None, help="HunyuanVideo sweep density (0.05..0.5)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layout", choices=["fused", "separate"], default="fused",
+                    help="temporal heads' layout transformation fused into attention, or as separate kernels")
     ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per chunk of the host-buffer call")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -263,18 +263,21 @@ SVG_API svg_status svg_dense_attn(const svg_shape* shape, const void* q, const v
                           void* o, int32_t* status_dev, void* stream);
 
 /*
- * svg_sparse_3d_attn_workspace_size -- bytes of device workspace the fused
- * call needs: token-major copies of q, k, v and o plus the profiling
- * workspace (0 on invalid arguments).
+ * svg_sparse_3d_attn_workspace_size -- bytes of device workspace the whole
+ * call needs: the profiling workspace, plus token-major copies of q, k, v
+ * and o for fp32 (bf16 folds the layout transformation into the attention
+ * kernel and needs no copies).  0 on invalid arguments.
  */
 SVG_API size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t S);
 
 /*
- * svg_sparse_3d_attn -- one whole sparse 3D-attention call: profile ->
- * permute temporal heads -> block-sparse attention -> unpermute, all
- * enqueued on `stream` with no host synchronisation.  Outputs o (frame-major
- * [B,H,L,d]) plus the profiling results mse [B,H,2] and label [B,H] (device).
- * Arguments as in the four calls above.
+ * svg_sparse_3d_attn -- one whole sparse 3D-attention call, enqueued on
+ * `stream` with no host synchronisation: profile -> block-sparse attention
+ * with the layout transformation fused in (svg_block_sparse_attn_fused) for
+ * bf16; profile -> permute temporal heads -> block-sparse attention ->
+ * unpermute for fp32.  Outputs o (frame-major [B,H,L,d]) plus the profiling
+ * results mse [B,H,2] and label [B,H] (device).  Arguments as in the calls
+ * above.
  */
 SVG_API svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v,
                               void* o, int32_t a1, int32_t a2, const int32_t* rows, int32_t S,
@@ -382,6 +385,35 @@ SVG_API svg_status svg_mode_search(const svg_shape* shape, const void* q, const 
                                    const int32_t* rows, int32_t S, int32_t window, int32_t md_half,
                                    int32_t stripe, float lambda, float epsilon, float* loss, int8_t* mode,
                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * svg_block_sparse_attn_fused -- svg_block_sparse_attn with the layout
+ * transformation folded into the attention kernel.  The token-major order of
+ * temporal heads ("Sparse VideoGen", Abstract: the hardware-efficient tensor
+ * layout transformation; Sparse VideoGen2 review, 2.A on permuting before
+ * attention and undoing it after) is applied while loading.  The N frames
+ * are split into groups of power-of-two size s; one 128-row tile is s frames
+ * x 128/s consecutive positions, loaded as one box of a 4D view of the
+ * frame-major q/k/v, and already in token-major order.  Keys are visited
+ * group by group (the temporal mask depends on the position only), and each
+ * output row is written to its frame-major position in o.  No permuted
+ * copies exist; o is frame-major for every head.  The key order differs from
+ * the unfused path, so results agree with it to rounding, not bit for bit.
+ * q, k, v, o: device bf16 [B,H,N*F,d] (d = 64 or 128); other arguments as
+ * for svg_block_sparse_attn.  SVG_ERR_UNSUPPORTED for fp32.
+ */
+SVG_API svg_status svg_block_sparse_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v,
+                                               void* o, const int8_t* label, int32_t a1, int32_t a2,
+                                               int32_t* status_dev, void* stream);
+
+/*
+ * svg_mixed_attn_fused -- svg_mixed_attn with the multi-diagonal heads'
+ * token-major layout folded in the same way (no permuted copies, o
+ * frame-major for every head).  The whole mixed-pattern call in one launch.
+ */
+SVG_API svg_status svg_mixed_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                        const int8_t* mode, int32_t window, int32_t md_half, int32_t stripe,
+                                        int32_t* status_dev, void* stream);
 
 /*
  * svg_selftest_wait_bound -- failure-detection self-test (test hook).

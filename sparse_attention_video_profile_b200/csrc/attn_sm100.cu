@@ -38,12 +38,19 @@
 namespace svg {
 
 svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D);
+svg_status make_group_map_bf16(CUtensorMap* map, const void* base, int BH, int N, int F, int D, int size);
 
 namespace {
+
+constexpr int kMaxFrameGroups = 24;
 
 struct AttnParams {
   CUtensorMap tm_q, tm_k, tm_v;     // frame-major [BH, L, D] bf16
   CUtensorMap tm_qp, tm_kp, tm_vp;  // token-major [BH, L, D] bf16
+  // Fused layout transformation: 4D views (d, frame, position, head) of the
+  // frame-major q/k/v whose box is s frames x 128/s positions (s = 2^e, map
+  // index e): one box is a 128-row tile already in token-major order.
+  CUtensorMap tm_fq[8], tm_fk[8], tm_fv[8];
   __nv_bfloat16* o;
   __nv_bfloat16* op;
   const int8_t* label;  // spatial (0) / temporal (1) per head, or nullptr
@@ -56,6 +63,14 @@ struct AttnParams {
   int* status;
   uint64_t wait_ns;
   int withhold_loads;  // self-test only: the producer issues nothing
+  int fused;           // token-major heads load through tm_f* and write O rows to frame-major positions
+  int F;               // tokens per frame (fused only)
+  // Frames split into groups of power-of-two size (largest first):
+  // group g = frames [gfirst[g], gfirst[g] + 2^glog[g]); a CTA of a
+  // token-major head takes 2 Q tiles of one group (2 * 128 / 2^glog[g]
+  // positions), gcta[g] CTAs per group.
+  int ng;
+  int glog[kMaxFrameGroups], gfirst[kMaxFrameGroups], gcta[kMaxFrameGroups];
 };
 
 template <int D>
@@ -193,18 +208,77 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   const int bh = blockIdx.x / p.n_ctiles;
   const HeadBand band = head_band(p, bh);
   const int lab = band.perm;
+  const bool fz = lab && p.fused;  // token-major head, layout transformation fused into the loads
   const int L = p.L;
-  const int q0 = ct * 256;
-  const int q_last = min(q0 + 255, L - 1);
-  int lo_cta, hi_cta, lo_unused, hi_unused;
-  row_interval(band, q0, L, lo_cta, hi_unused);
-  row_interval(band, q_last, L, lo_unused, hi_cta);
-  const int kt0 = lo_cta / C::BK;
-  const int nk = (hi_cta > lo_cta) ? (hi_cta + C::BK - 1) / C::BK - kt0 : 0;  // 0: skipped head
+  bool idle = false;  // no query rows for this CTA
+  int q0 = 0, kt0 = 0, nk = 0;
+  // fused: Q tile group, its first position, and the key position range
+  int gq = 0, pq0 = 0, kp_lo = 0, kp_hi = 0;
+  if (fz) {
+    int rem = ct;
+    while (gq < p.ng && rem >= p.gcta[gq]) rem -= p.gcta[gq++];
+    if (gq == p.ng) {
+      idle = true;
+    } else {
+      const int shq = 7 - p.glog[gq];  // log2 of positions per Q tile
+      pq0 = rem << (shq + 1);
+      const int pq_hi = min(p.F - 1, pq0 + (2 << shq) - 1);
+      kp_lo = max(0, pq0 - band.a + 1);
+      kp_hi = min(p.F - 1, pq_hi + band.a - 1);
+      for (int g = 0; g < p.ng; ++g) {
+        const int sh = 7 - p.glog[g];
+        nk += (kp_hi >> sh) - (kp_lo >> sh) + 1;
+      }
+    }
+  } else if (ct * 256 >= L) {
+    idle = true;
+  } else {
+    q0 = ct * 256;
+    const int q_last = min(q0 + 255, L - 1);
+    int lo_cta, hi_cta, lo_unused, hi_unused;
+    row_interval(band, q0, L, lo_cta, hi_unused);
+    row_interval(band, q_last, L, lo_unused, hi_cta);
+    kt0 = lo_cta / C::BK;
+    nk = (hi_cta > lo_cta) ? (hi_cta + C::BK - 1) / C::BK - kt0 : 0;  // 0: skipped head
+  }
   const bool run = (*abort_flag == 0);
 
   if (warp >= 8) {
-    if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads) {
+    if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads && fz) {
+      // ------------------------------------------------ TMA producer, fused layout transformation
+      // Key tiles go group by group; within group g, tile t holds positions
+      // [t P, (t+1) P) (P = 128 / 2^glog[g]) of the group's frames, one 4D box
+      // per 64-column half.  Positions past F read zeros.
+      tma_prefetch_desc(&p.tm_fq[p.glog[gq]]);
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+      const int shq = 7 - p.glog[gq];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_4d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, &p.tm_fq[p.glog[gq]], bar_q, h * 64,
+                      p.gfirst[gq], pq0 + (i << shq), bh);
+      int g = 0, sh = 7 - p.glog[0], t = kp_lo >> sh, t_end = kp_hi >> sh;
+      for (int n = 0; n < 2 * nk; ++n) {
+        const int slot = n % C::NS;
+        const uint32_t ph = (n / C::NS) & 1;
+        if (!mbar_wait(&bar_empty[slot], ph ^ 1, p.wait_ns)) {
+          record_timeout(p, abort_flag);
+          break;
+        }
+        const CUtensorMap* tm = (n & 1) ? &p.tm_fv[p.glog[g]] : &p.tm_fk[p.glog[g]];
+        mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, p.gfirst[g],
+                      t << sh, bh);
+        if ((n & 1) && ++t > t_end && ++g < p.ng) {  // next key tile after its V
+          sh = 7 - p.glog[g];
+          t = kp_lo >> sh;
+          t_end = kp_hi >> sh;
+        }
+      }
+    } else if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads) {
       // ------------------------------------------------ TMA producer
       {
       const CUtensorMap* tq = lab ? &p.tm_qp : &p.tm_q;
@@ -312,10 +386,20 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     // ------------------------------------------------ softmax / epilogue
     const int i = warp >> 2;
     const int quad = warp & 3;
-    const int r = q0 + i * C::BQ + quad * 32 + lane;  // query row in the head's layout
-    const bool row_ok = r < L;
+    const int r = q0 + i * C::BQ + quad * 32 + lane;  // query row in the head's layout (unfused)
+    // fused: the row's position and frame (rows of a tile: position-major,
+    // the group's frames inside), and its frame-major row x = frame F + pos
+    int pos_q = 0, x_q = r;
+    if (fz) {
+      const int rt = quad * 32 + lane;
+      const int lg = p.glog[gq];
+      pos_q = pq0 + (i << (7 - lg)) + (rt >> lg);
+      x_q = (p.gfirst[gq] + (rt & ((1 << lg) - 1))) * p.F + pos_q;
+    }
+    const bool row_ok = !idle && (fz ? pos_q < p.F : r < L);
     int lo_r = 0, hi_r = 0;
-    if (row_ok) row_interval(band, r, L, lo_r, hi_r);
+    if (row_ok && !fz) row_interval(band, r, L, lo_r, hi_r);
+    int kg = 0, ksh = 7 - p.glog[0], kt = kp_lo >> ksh, kt_end = kp_hi >> ksh;  // fused key-tile iterator
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::col_s(i);
     const uint32_t tO = tmem + lane_bits + C::col_o(i);
@@ -340,13 +424,27 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
 #pragma unroll
         for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(sr[c][e]);
 
-      const int kbase = (kt0 + k) * C::BK;
-      if (kbase < lo_r || kbase + C::BK > hi_r) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int y = kbase + c;
-          if (y < lo_r || y >= hi_r) s[c] = -INFINITY;
+      // keys of this tile the row keeps: columns [lo_c, hi_c)
+      int lo_c, hi_c;
+      if (fz) {
+        // key column c holds position (kt << ksh) + (c >> lg) of the group
+        const int lg = 7 - ksh, p0 = kt << ksh;
+        lo_c = (pos_q - band.a + 1 - p0) * (1 << lg);
+        hi_c = (min(pos_q + band.a, p.F) - p0) * (1 << lg);
+        if (++kt > kt_end && ++kg < p.ng) {
+          ksh = 7 - p.glog[kg];
+          kt = kp_lo >> ksh;
+          kt_end = kp_hi >> ksh;
         }
+      } else {
+        const int kbase = (kt0 + k) * C::BK;
+        lo_c = lo_r - kbase;
+        hi_c = hi_r - kbase;
+      }
+      if (lo_c > 0 || hi_c < C::BK) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c < lo_c || c >= hi_c) s[c] = -INFINITY;
       }
       float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
@@ -420,7 +518,9 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       }
       l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
     }
-    if (nk == 0) {
+    if (idle) {
+      // no query rows here
+    } else if (nk == 0) {
       // skipped head: its output rows are zero
       if (row_ok) {
         uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * L + r) * D);
@@ -430,7 +530,10 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     } else if (ok && warp_wait(&bar_o[i], (nk - 1) & 1, p.wait_ns)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* out = (lab ? p.op : p.o) + (static_cast<size_t>(bh) * L + (row_ok ? r : 0)) * D;
+      // output row: token-major heads write to op, or, fused, straight to
+      // the frame-major position of their row in o
+      const int orow = row_ok ? x_q : 0;
+      __nv_bfloat16* out = (lab && !p.fused ? p.op : p.o) + (static_cast<size_t>(bh) * L + orow) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -475,10 +578,41 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   if ((st = make_tile_map_bf16(&p.tm_q, a.q, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_k, a.k, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_v, a.v, BH, a.L, D)) != SVG_OK) return st;
-  const bool perm = a.label != nullptr || a.modes != nullptr;
+  const bool perm = (a.label != nullptr || a.modes != nullptr) && !a.fused;
   if ((st = make_tile_map_bf16(&p.tm_qp, perm ? a.qp : a.q, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_kp, perm ? a.kp : a.k, BH, a.L, D)) != SVG_OK) return st;
   if ((st = make_tile_map_bf16(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
+  p.fused = a.fused;
+  p.F = a.N > 0 ? a.L / a.N : 0;
+  int perm_ctas = 0;
+  if (a.fused) {
+    if (a.N < 1 || a.L % a.N != 0) return fail(SVG_ERR_INVALID_ARG, "fused layout transformation needs N >= 1");
+    // frame groups: powers of two, largest first, at most 128 frames each
+    int left = a.N, first = 0;
+    p.ng = 0;
+    while (left > 0) {
+      if (p.ng == kMaxFrameGroups) return fail(SVG_ERR_UNSUPPORTED, "too many frames for the fused layout (N = %d)", a.N);
+      int lg = 0;
+      while (lg < 7 && (2 << lg) <= left) ++lg;
+      const int pos_per_cta = 2 * (128 >> lg);
+      p.glog[p.ng] = lg;
+      p.gfirst[p.ng] = first;
+      p.gcta[p.ng] = (p.F + pos_per_cta - 1) / pos_per_cta;
+      perm_ctas += p.gcta[p.ng];
+      first += 1 << lg;
+      left -= 1 << lg;
+      ++p.ng;
+    }
+    bool made[8] = {false, false, false, false, false, false, false, false};
+    for (int g = 0; g < p.ng; ++g) {
+      const int lg = p.glog[g];
+      if (made[lg]) continue;
+      made[lg] = true;
+      if ((st = make_group_map_bf16(&p.tm_fq[lg], a.q, BH, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
+      if ((st = make_group_map_bf16(&p.tm_fk[lg], a.k, BH, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
+      if ((st = make_group_map_bf16(&p.tm_fv[lg], a.v, BH, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
+    }
+  }
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.op = static_cast<__nv_bfloat16*>(perm ? a.op : a.o);
   p.label = a.label;
@@ -490,6 +624,7 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   p.BH = BH;
   p.L = a.L;
   p.n_ctiles = (a.L + 255) / 256;
+  if (perm_ctas > p.n_ctiles) p.n_ctiles = perm_ctas;  // CTAs past a head's own count are idle
   p.G0 = a.G0;
   p.a0 = a.a0;
   p.G1 = a.G1;
@@ -542,6 +677,29 @@ svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SVG_OK;
+}
+
+// 4D view (d, frame, position, head) of a frame-major [BH, N*F, D] bf16
+// tensor with a box of `size` frames x 128/size positions: the box's 128 rows
+// come out position-major, i.e. in the token-major order of those frames.
+// Dimension 1 (frames) has the larger stride, so the strides are not in
+// increasing order; the box walks frames fastest.
+svg_status make_group_map_bf16(CUtensorMap* map, const void* base, int BH, int N, int F, int D, int size) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(F),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(F) * D * 2, static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(N) * F * D * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(size), static_cast<cuuint32_t>(128 / size), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled (frame-group map, %d frames) failed (%d)", size,
+                static_cast<int>(r));
   return SVG_OK;
 }
 

@@ -6,7 +6,9 @@
 // no other head), so the call is cut into chunks of heads.  Two device slots
 // (from the caller's workspace) alternate between chunks:
 //   copy-in stream   H2D of chunk c's q, k, v        (after slot c%2 is free)
-//   caller's stream  profile -> permute -> attention -> unpermute of chunk c
+//   caller's stream  the whole call on chunk c, as svg_sparse_3d_attn does it
+//                    (bf16: profile -> attention with the layout transformation
+//                    fused in; fp32: profile -> permute -> attention -> unpermute)
 //   copy-out stream  D2H of chunk c's o, mse, label  (after its compute)
 // so the copies of one chunk run under the kernels of its neighbours.  The
 // results are bit-identical to svg_sparse_3d_attn on the same data.
@@ -61,6 +63,7 @@ struct SlotLayout {
   size_t prof;     // profiling workspace of a chunk
   size_t mse, label, rows;
   size_t slot;     // bytes per slot
+  int ntensors;
 };
 
 SlotLayout slot_layout(const svg_shape* s, int S, int hc) {
@@ -74,7 +77,8 @@ SlotLayout slot_layout(const svg_shape* s, int S, int hc) {
   l.mse = align256(static_cast<size_t>(hc) * 2 * sizeof(float));
   l.label = align256(static_cast<size_t>(hc));
   l.rows = align256(static_cast<size_t>(S) * sizeof(int32_t));
-  l.slot = 8 * l.tensor + l.prof + l.mse + l.label + l.rows;
+  l.ntensors = s->dtype == SVG_BF16 ? 4 : 8;  // q k v o (+ token-major copies for fp32)
+  l.slot = l.ntensors * l.tensor + l.prof + l.mse + l.label + l.rows;
   return l;
 }
 
@@ -136,7 +140,7 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
     uint8_t *q = slot, *k = slot + lay.tensor, *v = slot + 2 * lay.tensor, *o = slot + 3 * lay.tensor;
     uint8_t *qp = slot + 4 * lay.tensor, *kp = slot + 5 * lay.tensor, *vp = slot + 6 * lay.tensor,
             *op = slot + 7 * lay.tensor;
-    uint8_t* prof = slot + 8 * lay.tensor;
+    uint8_t* prof = slot + lay.ntensors * lay.tensor;
     float* mse = reinterpret_cast<float*>(prof + lay.prof);
     int8_t* lab = reinterpret_cast<int8_t*>(prof + lay.prof + lay.mse);
     int32_t* rows = reinterpret_cast<int32_t*>(prof + lay.prof + lay.mse + lay.label);
@@ -156,10 +160,14 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
     cs.B = 1;
     cs.H = nh;
     if ((st = svg_profile_heads(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, stream)) != SVG_OK) return st;
-    if ((st = svg_permute_qkv(&cs, q, k, v, qp, kp, vp, lab, stream)) != SVG_OK) return st;
-    if ((st = svg_block_sparse_attn(&cs, q, k, v, qp, kp, vp, o, op, lab, a1, a2, status_dev, stream)) != SVG_OK)
-      return st;
-    if ((st = svg_unpermute(&cs, op, o, lab, stream)) != SVG_OK) return st;
+    if (shape->dtype == SVG_BF16) {
+      if ((st = svg_block_sparse_attn_fused(&cs, q, k, v, o, lab, a1, a2, status_dev, stream)) != SVG_OK) return st;
+    } else {
+      if ((st = svg_permute_qkv(&cs, q, k, v, qp, kp, vp, lab, stream)) != SVG_OK) return st;
+      if ((st = svg_block_sparse_attn(&cs, q, k, v, qp, kp, vp, o, op, lab, a1, a2, status_dev, stream)) != SVG_OK)
+        return st;
+      if ((st = svg_unpermute(&cs, op, o, lab, stream)) != SVG_OK) return st;
+    }
     SVG_CU(cudaEventRecord(r->ev_done[s], sc), "event record");
     // copy out
     SVG_CU(cudaStreamWaitEvent(r->s_out, r->ev_done[s], 0), "stream wait");

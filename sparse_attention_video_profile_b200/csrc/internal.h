@@ -49,6 +49,11 @@ struct BandAttnArgs {
   int* status;          // device status word (never null here)
   uint64_t wait_ns;
   int withhold_loads;   // self-test of the bounded waits (tcgen05 kernel only)
+  // Fused layout transformation (tcgen05 kernel only): heads that run
+  // token-major read their rows straight from (q, k, v) by row gathers and
+  // write O rows back to frame-major positions of o; qp..op are unused.
+  // Needs N (frames) > 0.
+  int fused;
 };
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);

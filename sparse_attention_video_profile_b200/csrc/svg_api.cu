@@ -266,6 +266,30 @@ svg_status svg_block_sparse_attn(const svg_shape* shape, const void* q, const vo
   return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
 }
 
+svg_status svg_block_sparse_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                       const int8_t* label, int32_t a1, int32_t a2, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "the fused layout transformation runs in bf16 only");
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (label == nullptr) return fail(SVG_ERR_INVALID_ARG, "label is NULL");
+  if (a1 < 1 || a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a1 and a2 must be >= 1");
+  const int L = shape->N * shape->F;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.label = label;
+  a.G0 = shape->F;
+  a.a0 = clamp_band(a1, shape->F, L);
+  a.G1 = shape->N;
+  a.a1 = clamp_band(a2, shape->N, L);
+  a.N = shape->N;
+  a.fused = 1;
+  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+}
+
 svg_status svg_banded_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o, int32_t G,
                            int32_t a_band, int32_t* status_dev, void* stream) {
   svg_status st = check_shape(shape);
@@ -298,6 +322,7 @@ size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t S) {
   if (check_shape(shape) != SVG_OK) return 0;
   const size_t prof = svg_profile_workspace_size(shape, S);
   if (prof == 0) return 0;
+  if (shape->dtype == SVG_BF16) return prof;  // layout transformation fused: no token-major copies
   const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
   const size_t t_al = (t + 255) / 256 * 256;
   return 4 * t_al + prof;
@@ -315,6 +340,12 @@ svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void*
   if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (shape->dtype == SVG_BF16) {
+    if ((st = svg_profile_heads(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, stream)) !=
+        SVG_OK)
+      return st;
+    return svg_block_sparse_attn_fused(shape, q, k, v, o, label, a1, a2, status_dev, stream);
+  }
   const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
   const size_t t_al = (t + 255) / 256 * 256;
   uint8_t* w = static_cast<uint8_t*>(workspace);
@@ -357,6 +388,34 @@ svg_status svg_mixed_attn(const svg_shape* shape, const void* q, const void* k, 
   a.N = shape->N;
   a.md_a = clamp_band(md_half + 1, shape->N, L);
   a.stripe = stripe < L ? stripe : L;
+  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_mixed_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                const int8_t* mode, int32_t window, int32_t md_half, int32_t stripe,
+                                int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "mixed-pattern attention runs in bf16 only");
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (mode == nullptr) return fail(SVG_ERR_INVALID_ARG, "mode is NULL");
+  if (window < 0 || md_half < 0 || stripe < 1) return fail(SVG_ERR_INVALID_ARG, "window, md_half >= 0 and stripe >= 1");
+  const int L = shape->N * shape->F;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.modes = mode;
+  a.G0 = L;
+  a.a0 = 1;
+  a.G1 = L;
+  a.a1 = 1;
+  a.win = window < L ? window : L;
+  a.N = shape->N;
+  a.md_a = clamp_band(md_half + 1, shape->N, L);
+  a.stripe = stripe < L ? stripe : L;
+  a.fused = 1;
   return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
 }
 

@@ -36,7 +36,8 @@ EXPORTED = (
     "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
     "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
     "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
-    "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search",
+    "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search", "svg_block_sparse_attn_fused",
+    "svg_mixed_attn_fused",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -88,6 +89,8 @@ def _load() -> ctypes.CDLL:
         "svg_sparse_3d_attn_host_workspace_size": (_Z, [_P, _I, _I]),
         "svg_sparse_3d_attn_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _I, _P, _Z, _P, _P]),
         "svg_mode_search_workspace_size": (_Z, [_P, _I]),
+        "svg_block_sparse_attn_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
+        "svg_mixed_attn_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
         "svg_mode_search": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _Z,
                                  _P]),
     }
@@ -257,6 +260,19 @@ def svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N: int, F: int, a1: int, a
     return o, op
 
 
+def svg_block_sparse_attn_fused(q, k, v, label, N: int, F: int, a1: int, a2: int, *, o=None, status=None,
+                                scale: float = 0.0, stream=None):
+    """Block-sparse attention with the layout transformation fused in: every
+    head's output lands frame-major in o (no permuted copies).  bf16."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib.svg_block_sparse_attn_fused(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(label), a1,
+                                           a2, _ptr(status), _stream(stream)))
+    return o
+
+
 def svg_banded_attn(q, k, v, N: int, F: int, G: int, a: int, *, o=None, status=None, scale: float = 0.0,
                     stream=None):
     _same(q, k, v)
@@ -296,6 +312,18 @@ def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Te
                                   _ptr(mse), _ptr(label), _ptr(workspace), workspace.numel(), _ptr(status),
                                   _stream(stream)))
     return o, mse, label
+
+
+def svg_mixed_attn_fused(q, k, v, mode, N: int, F: int, window: int, md_half: int, stripe: int, *, o=None,
+                         status=None, scale: float = 0.0, stream=None):
+    """Mixed-pattern attention with the multi-diagonal heads' layout fused in."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib.svg_mixed_attn_fused(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(mode), window,
+                                    md_half, stripe, _ptr(status), _stream(stream)))
+    return o
 
 
 def svg_mixed_attn(q, k, v, qp, kp, vp, mode, N: int, F: int, window: int, md_half: int, stripe: int, *,

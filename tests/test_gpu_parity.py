@@ -460,3 +460,97 @@ def test_mode_search_mixed_workload():
     ref_loss, ref_mode = oracle.mode_search(f64(q), f64(k), f64(v), wl.N, wl.F, rows_np, *args[2:], sparsity=sp)
     decided = check_mode_search(loss, mode, ref_loss, ref_mode, sp, 0.5, 1.0)
     assert decided.mean() > 0.5
+
+
+# ---------------------------------------------------------------- fused layout transformation
+
+@pytest.mark.parametrize("N,F,d", [(6, 90, 128), (5, 133, 64), (33, 17, 128), (1, 300, 128), (7, 1, 64),
+                                   (3, 29, 128), (13, 45, 64), (21, 20, 128), (130, 3, 64)])
+def test_fused_block_sparse(N, F, d):
+    """Frame-group boxes (s frames x 128/s positions per tile) from the
+    frame-major tensors and the frame-major output scatter: against the
+    oracle, on shapes with 1..8 frame groups, ragged position tails and
+    frames above 128."""
+    L = N * F
+    H = 4
+    q, k, v = rand_qkv(2, H, L, d, torch.bfloat16, 50 + N + F)
+    label = torch.tensor([[1, 0, 1, 1], [0, 1, 0, 1]], dtype=torch.int8, device=DEV)
+    a1, a2 = min(2, N), max(1, min(F, 7))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, a1, a2, status=status)
+    sync_ok(status)
+    ref = oracle.sparse_attention(f64(q), f64(k), f64(v), label.cpu().numpy(), N, F, a1, a2)
+    assert_close(f64(o), ref, torch.bfloat16, "fused")
+
+
+def test_fused_matches_separate_layout_video_shape():
+    """HunyuanVideo shape: the whole call (fused layout) against profile ->
+    permute -> attention -> unpermute; same labels and MSEs bit for bit (same
+    profiling), outputs within twice the bf16 tolerance of each other, and
+    sampled rows against the oracle."""
+    wl = synth.WORKLOADS["hunyuan"]
+    q, k, v = synth.make_qkv(wl, seed=2, device=DEV)
+    rows_np = synth.sample_rows(wl.L, wl.S, 2)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, mse, lab = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, status=status)
+    mse2, lab2 = svg.svg_profile_heads(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows)
+    qp, kp, vp = svg.svg_permute_qkv(q, k, v, wl.N, wl.F, lab2)
+    o2, op = svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, lab2, wl.N, wl.F, wl.a1, wl.a2, status=status)
+    o2 = svg.svg_unpermute(op, wl.N, wl.F, lab2, out=o2)
+    sync_ok(status)
+    del qp, kp, vp, op
+    assert torch.equal(lab, lab2) and torch.equal(mse, mse2)
+    assert int(lab.sum()) > 0  # the token-major path is exercised
+    # each path is within (2e-2 max-abs, 1e-2 rel L2) of the exact result, so
+    # by the triangle inequality they are within twice that of each other
+    diff = (o.float() - o2.float())
+    assert float(diff.abs().max()) <= 4e-2, float(diff.abs().max())
+    assert float(diff.norm() / o2.float().norm()) <= 2e-2
+    idx = torch.from_numpy(sampled_rows(wl, n_extra=16)).to(DEV)
+    for h in range(wl.H):
+        if int(lab[0, h]) == 0:
+            continue
+        qn, kn, vn = (f64(t[:, h:h + 1]) for t in (q, k, v))
+        ref = oracle.sparse_attention(qn, kn, vn, lab[:, h:h + 1].cpu().numpy(), wl.N, wl.F, wl.a1, wl.a2,
+                                      rows=idx.cpu().numpy())
+        assert_close(f64(o[:, h:h + 1, idx]), ref, q.dtype, f"fused head {h}")
+        break
+
+
+@pytest.mark.parametrize("name", ["small", "mixed"])
+def test_fused_mixed(name):
+    if name == "small":
+        N, F, H, d = 6, 90, 10, 128
+        q, k, v = rand_qkv(1, H, N * F, d, torch.bfloat16, 61)
+        modes_np = np.array([[0, 1, 2, 3, 4, 3, 3, 4, 0, 2]], dtype=np.int8)
+        win, mdh, stripe = F, 7, 100
+        rows = None
+    else:
+        wl = synth.WORKLOADS["mixed"]
+        prm = synth.MIXED_PARAMS
+        N, F = wl.N, wl.F
+        q, k, v = synth.make_qkv(wl, seed=1, device=DEV)
+        modes_np = synth.head_modes(wl.B, wl.H, 1)
+        win, mdh, stripe = prm["window"], prm["md_half"], prm["stripe"]
+        rows = sampled_rows(wl, n_extra=12)
+    mode = torch.from_numpy(modes_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = svg.svg_mixed_attn_fused(q, k, v, mode, N, F, win, mdh, stripe, status=status)
+    sync_ok(status)
+    if rows is None:
+        ref = oracle.mixed_attention(f64(q), f64(k), f64(v), modes_np, N, F, win, mdh, stripe)
+        assert_close(f64(o), ref, torch.bfloat16, "fused mixed")
+        return
+    idx = torch.from_numpy(rows).to(DEV)
+    for h in np.nonzero(modes_np[0] == 3)[0][:3]:
+        qn, kn, vn = (f64(t[:, h:h + 1]) for t in (q, k, v))
+        ref = oracle.mixed_attention(qn, kn, vn, modes_np[:, h:h + 1], N, F, win, mdh, stripe, rows=rows)
+        assert_close(f64(o[:, h:h + 1, idx]), ref, q.dtype, f"fused mixed head {h}")
+
+
+def test_fused_rejects_fp32():
+    q, k, v = rand_qkv(1, 1, 64, 64, torch.float32, 3)
+    label = torch.zeros(1, 1, dtype=torch.int8, device=DEV)
+    with pytest.raises(svg.SvgError):
+        svg.svg_block_sparse_attn_fused(q, k, v, label, 4, 16, 1, 1)

@@ -95,7 +95,7 @@ struct Cfg {
 // Pairs (of 8) per softmax row chunk whose exponentials use the FMA-pipe
 // polynomial instead of the MUFU ex2 unit.
 #ifndef SVG_EXP_POLY_PAIRS
-#define SVG_EXP_POLY_PAIRS 2
+#define SVG_EXP_POLY_PAIRS 3
 #endif
 constexpr int kExpPoly = SVG_EXP_POLY_PAIRS;
 
@@ -504,9 +504,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           const uint32_t pp = pack_bf16x2(pr.x, pr.y);
           // The row sum uses the same bf16-rounded weights the P V product
           // sees, so each output row is an exact convex combination of V rows.
-          const float2 pw = make_float2(bf16lo_f32(pp), bf16hi_f32(pp));
-          if (c & 1) acc1 = __fadd2_rn(acc1, pw);
-          else acc0 = __fadd2_rn(acc0, pw);
+          if (c & 1) add_bf16x2_f32(acc1, pp);
+          else add_bf16x2_f32(acc0, pp);
           pk[cc] = pp;
         }
         __syncwarp();

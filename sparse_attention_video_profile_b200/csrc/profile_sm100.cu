@@ -89,9 +89,8 @@ __device__ __forceinline__ float pack_masked(const float (&e)[128], const uint32
     const float p0 = bit128(m, 2 * c) ? e[2 * c] : 0.f;
     const float p1 = bit128(m, 2 * c + 1) ? e[2 * c + 1] : 0.f;
     const uint32_t pp = pack_bf16x2(p0, p1);
-    const float2 pw = make_float2(bf16lo_f32(pp), bf16hi_f32(pp));
-    if (c & 1) a1 = __fadd2_rn(a1, pw);
-    else a0 = __fadd2_rn(a0, pw);
+    if (c & 1) add_bf16x2_f32(a1, pp);
+    else add_bf16x2_f32(a0, pp);
     pk[c] = pp;
   }
   return (a0.x + a1.x) + (a0.y + a1.y);

@@ -328,6 +328,15 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
+// acc.x += low bf16 half of v, acc.y += high half: round-to-nearest fp32
+// adds of the exactly widened bf16 values (the mixed-precision add, so the
+// halves need no separate unpacking).
+__device__ __forceinline__ void add_bf16x2_f32(float2& acc, uint32_t v) {
+  asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %2; add.rn.f32.bf16 %0, lo, %0; add.rn.f32.bf16 %1, hi, %1; }"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "r"(v));
+}
+
 // The two bf16 halves of a packed pair, widened back to fp32 (exact).
 __device__ __forceinline__ float bf16lo_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

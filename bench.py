@@ -255,8 +255,6 @@ def run_ours(args, wl, rank, world, local):
     o = torch.empty_like(q)
     # token-major copies: only the separate layout path needs them
     qp = kp = vp = op = None
-    if args.layout == "separate":
-        qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
     mse = torch.empty(wl.B, wl.H, 2, dtype=torch.float32, device=dev)
     label = torch.empty(wl.B, wl.H, dtype=torch.int8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -268,7 +266,12 @@ def run_ours(args, wl, rank, world, local):
         prm = synth.MIXED_PARAMS
         modes_np = synth.head_modes(wl.B, wl.H, rank)
         mode = torch.from_numpy(modes_np).to(dev)
-    fused = args.layout == "fused"
+    # layout of token-major heads; auto = the whole call's own choice
+    band = prm["md_half"] + 1 if mixed else wl.a2
+    plan_sep, plan_fused, plan_choice = svg.svg_sparse_3d_attn_plan(shape, band)
+    fused = plan_choice if args.layout == "auto" else args.layout == "fused"
+    if not fused:
+        qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
     if mixed:
         names = ("attn",) if fused else ("permute", "attn", "unpermute")
     else:
@@ -418,7 +421,7 @@ def run_ours(args, wl, rank, world, local):
         mseh = torch.empty(mse.shape, dtype=mse.dtype, pin_memory=True)
         labh = torch.empty(label.shape, dtype=label.dtype, pin_memory=True)
         rowsh = torch.from_numpy(rows_np).pin_memory()
-        need = int(svg.lib.svg_sparse_3d_attn_host_workspace_size(svg.ctypes.byref(shape), wl.S, args.e2e_chunk))
+        need = int(svg.lib.svg_sparse_3d_attn_host_workspace_size(svg.ctypes.byref(shape), wl.a2, wl.S, args.e2e_chunk))
         ws_host_call = svg.alloc_workspace(need, dev)
 
         def e2e_step():
@@ -464,8 +467,10 @@ def run_ours(args, wl, rank, world, local):
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
         "dense_ms": dense_ms,
         "kernel_ms": kern_ms,
-        "layout": ("fused: token-major heads gathered by the attention kernel, no permuted copies" if fused else
-                   "separate: permute -> attention -> unpermute"),
+        "layout": ("fused: token-major heads loaded by frame-group boxes in the attention kernel, no permuted copies"
+                   if fused else "separate: permute -> attention -> unpermute"),
+        "layout_plan": {"separate_tiles_per_head": plan_sep, "fused_tiles_per_head": plan_fused,
+                        "choice": "fused" if plan_choice else "separate", "requested": args.layout},
         "permute_gbs": perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
         "unpermute_gbs": unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
         "temporal_heads": n_temporal,
@@ -496,8 +501,9 @@ def main():
     ap.add_argument("--density", type=float, default=None, help="HunyuanVideo sweep density (0.05..0.5)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--layout", choices=["fused", "separate"], default="fused",
-                    help="temporal heads' layout transformation fused into attention, or as separate kernels")
+    ap.add_argument("--layout", choices=["auto", "fused", "separate"], default="auto",
+                    help="temporal heads' layout transformation fused into attention, or as separate kernels; "
+                         "auto = the whole call's own choice")
     ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per chunk of the host-buffer call")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -264,18 +264,32 @@ SVG_API svg_status svg_dense_attn(const svg_shape* shape, const void* q, const v
 
 /*
  * svg_sparse_3d_attn_workspace_size -- bytes of device workspace the whole
- * call needs: the profiling workspace, plus token-major copies of q, k, v
- * and o for fp32 (bf16 folds the layout transformation into the attention
- * kernel and needs no copies).  0 on invalid arguments.
+ * call needs for temporal band a2 and S sampled rows: the profiling
+ * workspace, plus token-major copies of q, k, v and o unless the call folds
+ * the layout transformation into attention (see svg_sparse_3d_attn).  0 on
+ * invalid arguments.
  */
-SVG_API size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t S);
+SVG_API size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t a2, int32_t S);
+
+/*
+ * svg_sparse_3d_attn_plan -- the layout choice svg_sparse_3d_attn makes, on
+ * the host: separate_tiles / fused_tiles = 128-key tiles one temporal head
+ * takes over all its query rows with token-major copies / with the fused
+ * frame-group layout; *fused = 1 if the call folds the layout transformation
+ * into attention.  Host pointers.
+ */
+SVG_API svg_status svg_sparse_3d_attn_plan(const svg_shape* shape, int32_t a2, int64_t* separate_tiles,
+                                           int64_t* fused_tiles, int32_t* fused);
 
 /*
  * svg_sparse_3d_attn -- one whole sparse 3D-attention call, enqueued on
  * `stream` with no host synchronisation: profile -> block-sparse attention
- * with the layout transformation fused in (svg_block_sparse_attn_fused) for
- * bf16; profile -> permute temporal heads -> block-sparse attention ->
- * unpermute for fp32.  Outputs o (frame-major [B,H,L,d]) plus the profiling
+ * with the layout transformation fused in (svg_block_sparse_attn_fused), or
+ * profile -> permute temporal heads -> block-sparse attention -> unpermute.
+ * The fused form is used for bf16 when its frame-group tiling costs at most
+ * 3 % more attention work than the token-major copies (about what the two
+ * permutation passes cost), counted on the host from N, F and a2; fp32
+ * always permutes.  Outputs o (frame-major [B,H,L,d]) plus the profiling
  * results mse [B,H,2] and label [B,H] (device).  Arguments as in the calls
  * above.
  */
@@ -288,9 +302,11 @@ SVG_API svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, con
  * svg_sparse_3d_attn_host_workspace_size -- device workspace of
  * svg_sparse_3d_attn_host for a chunk of `heads_per_chunk` heads (0 on bad
  * arguments): two slots, each with a chunk's q, k, v, o, their token-major
- * copies and the chunk's profiling workspace.
+ * copies when svg_sparse_3d_attn would make them, and the chunk's profiling
+ * workspace.
  */
-SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, int32_t S, int32_t heads_per_chunk);
+SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, int32_t a2, int32_t S,
+                                                      int32_t heads_per_chunk);
 
 /*
  * svg_sparse_3d_attn_host -- svg_sparse_3d_attn on HOST buffers.

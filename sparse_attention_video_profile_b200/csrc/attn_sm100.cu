@@ -32,6 +32,8 @@
 // TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D,256+2D).
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -68,8 +70,10 @@ struct AttnParams {
   // Frames split into groups of power-of-two size (largest first):
   // group g = frames [gfirst[g], gfirst[g] + 2^glog[g]); a CTA of a
   // token-major head takes 2 Q tiles of one group (2 * 128 / 2^glog[g]
-  // positions), gcta[g] CTAs per group.
-  int ng;
+  // positions).  CTAs are ordered by position: block b of bpos positions
+  // has cpb CTAs, gcta[g] of them for group g (in group order), so CTAs that
+  // run together share their key positions in L2.
+  int ng, bpos, cpb;
   int glog[kMaxFrameGroups], gfirst[kMaxFrameGroups], gcta[kMaxFrameGroups];
 };
 
@@ -215,13 +219,14 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   // fused: Q tile group, its first position, and the key position range
   int gq = 0, pq0 = 0, kp_lo = 0, kp_hi = 0;
   if (fz) {
-    int rem = ct;
+    const int blk = ct / p.cpb;
+    int rem = ct - blk * p.cpb;
     while (gq < p.ng && rem >= p.gcta[gq]) rem -= p.gcta[gq++];
-    if (gq == p.ng) {
+    const int shq = 7 - p.glog[gq < p.ng ? gq : 0];  // log2 of positions per Q tile
+    pq0 = blk * p.bpos + (rem << (shq + 1));
+    if (gq == p.ng || pq0 >= p.F) {
       idle = true;
     } else {
-      const int shq = 7 - p.glog[gq];  // log2 of positions per Q tile
-      pq0 = rem << (shq + 1);
       const int pq_hi = min(p.F - 1, pq0 + (2 << shq) - 1);
       kp_lo = max(0, pq0 - band.a + 1);
       kp_hi = min(p.F - 1, pq_hi + band.a - 1);
@@ -586,22 +591,21 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   int perm_ctas = 0;
   if (a.fused) {
     if (a.N < 1 || a.L % a.N != 0) return fail(SVG_ERR_INVALID_ARG, "fused layout transformation needs N >= 1");
-    // frame groups: powers of two, largest first, at most 128 frames each
-    int left = a.N, first = 0;
-    p.ng = 0;
-    while (left > 0) {
-      if (p.ng == kMaxFrameGroups) return fail(SVG_ERR_UNSUPPORTED, "too many frames for the fused layout (N = %d)", a.N);
-      int lg = 0;
-      while (lg < 7 && (2 << lg) <= left) ++lg;
-      const int pos_per_cta = 2 * (128 >> lg);
-      p.glog[p.ng] = lg;
-      p.gfirst[p.ng] = first;
-      p.gcta[p.ng] = (p.F + pos_per_cta - 1) / pos_per_cta;
-      perm_ctas += p.gcta[p.ng];
-      first += 1 << lg;
-      left -= 1 << lg;
-      ++p.ng;
+    p.ng = fused_frame_groups(a.N, p.glog, kMaxFrameGroups);
+    if (p.ng < 0) return fail(SVG_ERR_UNSUPPORTED, "too many frames for the fused layout (N = %d)", a.N);
+    for (int g = 0, first = 0; g < p.ng; ++g) {
+      p.gfirst[g] = first;
+      first += 1 << p.glog[g];
     }
+    // position blocks: as wide as the smallest group's CTA (2 * 128 / 2^lg
+    // positions); group g has bpos / (2 * 128 >> lg) CTAs per block
+    p.bpos = 2 * (128 >> p.glog[p.ng - 1]);
+    p.cpb = 0;
+    for (int g = 0; g < p.ng; ++g) {
+      p.gcta[g] = p.bpos / (2 * (128 >> p.glog[g]));
+      p.cpb += p.gcta[g];
+    }
+    perm_ctas = (p.F + p.bpos - 1) / p.bpos * p.cpb;
     bool made[8] = {false, false, false, false, false, false, false, false};
     for (int g = 0; g < p.ng; ++g) {
       const int lg = p.glog[g];
@@ -700,6 +704,56 @@ svg_status make_group_map_bf16(CUtensorMap* map, const void* base, int BH, int N
     return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled (frame-group map, %d frames) failed (%d)", size,
                 static_cast<int>(r));
   return SVG_OK;
+}
+
+int fused_frame_groups(int N, int* glog, int max_groups) {
+  int ng = 0;
+  for (int left = N; left > 0; ++ng) {
+    if (ng == max_groups) return -1;
+    int lg = 0;
+    while (lg < 7 && (2 << lg) <= left) ++lg;
+    glog[ng] = lg;
+    left -= 1 << lg;
+  }
+  return ng;
+}
+
+void token_major_tile_counts(int N, int F, int a, long long* separate, long long* fused) {
+  const long long L = static_cast<long long>(N) * F;
+  long long sep = 0;
+  for (long long q0 = 0; q0 < L; q0 += 256) {  // 256-row query slabs of the token-major layout
+    const long long q1 = std::min(q0 + 255, L - 1);
+    const long long lo = std::max(0LL, (q0 / N - a + 1) * N), hi = std::min(L, (q1 / N + a) * N);
+    sep += (hi + 127) / 128 - lo / 128;
+  }
+  *separate = sep;
+  int glog[kMaxFrameGroups];
+  const int ng = fused_frame_groups(N, glog, kMaxFrameGroups);
+  if (ng < 0) {
+    *fused = -1;
+    return;
+  }
+  const int bpos = 2 * (128 >> glog[ng - 1]);
+  long long fz = 0;
+  for (int p0 = 0; p0 < F; p0 += bpos)
+    for (int g = 0; g < ng; ++g) {
+      const int per = 2 * (128 >> glog[g]);  // positions per CTA of group g
+      for (int pq0 = p0; pq0 < p0 + bpos && pq0 < F; pq0 += per) {
+        const int pq_hi = std::min(F - 1, pq0 + per - 1);
+        const int kp_lo = std::max(0, pq0 - a + 1), kp_hi = std::min(F - 1, pq_hi + a - 1);
+        for (int gk = 0; gk < ng; ++gk) {
+          const int sh = 7 - glog[gk];
+          fz += (kp_hi >> sh) - (kp_lo >> sh) + 1;
+        }
+      }
+    }
+  *fused = fz;
+}
+
+bool fused_layout_preferred(int N, int F, int a) {
+  long long sep = 0, fz = 0;
+  token_major_tile_counts(N, F, a, &sep, &fz);
+  return fz >= 0 && fz * 100 <= sep * 103;
 }
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream) {

@@ -6,9 +6,9 @@
 // no other head), so the call is cut into chunks of heads.  Two device slots
 // (from the caller's workspace) alternate between chunks:
 //   copy-in stream   H2D of chunk c's q, k, v        (after slot c%2 is free)
-//   caller's stream  the whole call on chunk c, as svg_sparse_3d_attn does it
-//                    (bf16: profile -> attention with the layout transformation
-//                    fused in; fp32: profile -> permute -> attention -> unpermute)
+//   caller's stream  the whole call on chunk c, with svg_sparse_3d_attn's
+//                    choice of layout (fused into attention, or permute ->
+//                    attention -> unpermute)
 //   copy-out stream  D2H of chunk c's o, mse, label  (after its compute)
 // so the copies of one chunk run under the kernels of its neighbours.  The
 // results are bit-identical to svg_sparse_3d_attn on the same data.
@@ -66,7 +66,7 @@ struct SlotLayout {
   int ntensors;
 };
 
-SlotLayout slot_layout(const svg_shape* s, int S, int hc) {
+SlotLayout slot_layout(const svg_shape* s, int S, int hc, bool fused) {
   SlotLayout l{};
   const size_t es = s->dtype == SVG_FP32 ? 4 : 2;
   l.tensor = align256(static_cast<size_t>(hc) * s->N * s->F * s->d * es);
@@ -77,7 +77,7 @@ SlotLayout slot_layout(const svg_shape* s, int S, int hc) {
   l.mse = align256(static_cast<size_t>(hc) * 2 * sizeof(float));
   l.label = align256(static_cast<size_t>(hc));
   l.rows = align256(static_cast<size_t>(S) * sizeof(int32_t));
-  l.ntensors = s->dtype == SVG_BF16 ? 4 : 8;  // q k v o (+ token-major copies for fp32)
+  l.ntensors = fused ? 4 : 8;  // q k v o (+ token-major copies unless the layout is fused)
   l.slot = l.ntensors * l.tensor + l.prof + l.mse + l.label + l.rows;
   return l;
 }
@@ -89,11 +89,12 @@ using namespace svg;
 
 extern "C" {
 
-SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, int32_t S, int32_t heads_per_chunk) {
-  if (shape == nullptr || heads_per_chunk < 1 || S < 1 || S > 128) return 0;
+SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, int32_t a2, int32_t S,
+                                                      int32_t heads_per_chunk) {
+  if (shape == nullptr || heads_per_chunk < 1 || S < 1 || S > 128 || a2 < 1) return 0;
   if (svg_profile_workspace_size(shape, S) == 0) return 0;
   const int hc = heads_per_chunk < shape->B * shape->H ? heads_per_chunk : shape->B * shape->H;
-  return 2 * slot_layout(shape, S, hc).slot;
+  return 2 * slot_layout(shape, S, hc, whole_call_fused(shape, a2)).slot;
 }
 
 SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q_host, const void* k_host,
@@ -105,14 +106,15 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
   if (!q_host || !k_host || !v_host || !o_host || !rows_host || !mse_host || !label_host || !workspace)
     return fail(SVG_ERR_INVALID_ARG, "NULL host buffer or workspace");
   if (heads_per_chunk < 1) return fail(SVG_ERR_INVALID_ARG, "heads_per_chunk must be >= 1");
-  const size_t need = svg_sparse_3d_attn_host_workspace_size(shape, S, heads_per_chunk);
-  if (need == 0) return fail(SVG_ERR_INVALID_ARG, "bad shape or S");
+  const size_t need = svg_sparse_3d_attn_host_workspace_size(shape, a2, S, heads_per_chunk);
+  if (need == 0) return fail(SVG_ERR_INVALID_ARG, "bad shape, S or a2");
   if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   const int BH = shape->B * shape->H;
   const int hc = heads_per_chunk < BH ? heads_per_chunk : BH;
-  const SlotLayout lay = slot_layout(shape, S, hc);
+  const bool fused = whole_call_fused(shape, a2);
+  const SlotLayout lay = slot_layout(shape, S, hc, fused);
   const size_t es = shape->dtype == SVG_FP32 ? 4 : 2;
   const size_t head_bytes = static_cast<size_t>(shape->N) * shape->F * shape->d * es;
 
@@ -160,7 +162,7 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
     cs.B = 1;
     cs.H = nh;
     if ((st = svg_profile_heads(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, stream)) != SVG_OK) return st;
-    if (shape->dtype == SVG_BF16) {
+    if (fused) {
       if ((st = svg_block_sparse_attn_fused(&cs, q, k, v, o, lab, a1, a2, status_dev, stream)) != SVG_OK) return st;
     } else {
       if ((st = svg_permute_qkv(&cs, q, k, v, qp, kp, vp, lab, stream)) != SVG_OK) return st;

@@ -57,6 +57,21 @@ struct BandAttnArgs {
 };
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);
+// Frame groups of the fused layout transformation: powers of two, largest
+// first, at most 128 frames each.  Writes their log2 sizes to glog and
+// returns how many there are, or -1 if more than max_groups are needed.
+int fused_frame_groups(int N, int* glog, int max_groups);
+// Key tiles (128 keys) one token-major head with positional half-width a
+// (keys |j1 - j2| < a, a <= F) takes over all its query rows: with
+// token-major copies (`separate`) and with the fused layout (`fused`, the
+// same CTA geometry as the kernel).
+void token_major_tile_counts(int N, int F, int a, long long* separate, long long* fused);
+// True when the fused layout does at most 3 % more attention work than the
+// token-major copies (about what the permute + unpermute passes cost).
+bool fused_layout_preferred(int N, int F, int a);
+// The choice svg_sparse_3d_attn makes (and its host-buffer form): bf16 and
+// fused_layout_preferred with the clamped temporal band.
+bool whole_call_fused(const svg_shape* s, int a2);
 svg_status launch_attn_simt(const BandAttnArgs& a, cudaStream_t stream);
 // Tile shape of the tcgen05 kernel (rows of Q per tile, keys per tile).
 constexpr int kAttnBq = 128;

@@ -66,6 +66,17 @@ int clamp_band(int a, int G, int L) {
   return a > full ? full : a;
 }
 
+}  // namespace
+
+// The whole bf16 call folds the layout transformation into attention when
+// that costs at most 3 % more attention work than the token-major copies.
+bool whole_call_fused(const svg_shape* s, int a2) {
+  if (s->dtype != SVG_BF16 || a2 < 1) return false;
+  return fused_layout_preferred(s->N, s->F, clamp_band(a2, s->N, s->N * s->F));
+}
+
+namespace {
+
 svg_status status_word(int32_t* user, int** out, cudaStream_t stream) {
   if (user != nullptr) {
     *out = user;
@@ -318,14 +329,28 @@ svg_status svg_dense_attn(const svg_shape* shape, const void* q, const void* k, 
   return svg_banded_attn(shape, q, k, v, o, shape->N * shape->F, 1, status_dev, stream);
 }
 
-size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t S) {
-  if (check_shape(shape) != SVG_OK) return 0;
+size_t svg_sparse_3d_attn_workspace_size(const svg_shape* shape, int32_t a2, int32_t S) {
+  if (check_shape(shape) != SVG_OK || a2 < 1) return 0;
   const size_t prof = svg_profile_workspace_size(shape, S);
   if (prof == 0) return 0;
-  if (shape->dtype == SVG_BF16) return prof;  // layout transformation fused: no token-major copies
+  if (whole_call_fused(shape, a2)) return prof;  // layout transformation fused: no token-major copies
   const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
   const size_t t_al = (t + 255) / 256 * 256;
   return 4 * t_al + prof;
+}
+
+svg_status svg_sparse_3d_attn_plan(const svg_shape* shape, int32_t a2, int64_t* separate_tiles, int64_t* fused_tiles,
+                                   int32_t* fused) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a2 must be >= 1");
+  if (!separate_tiles || !fused_tiles || !fused) return fail(SVG_ERR_INVALID_ARG, "NULL output");
+  long long sep = 0, fz = 0;
+  token_major_tile_counts(shape->N, shape->F, clamp_band(a2, shape->N, shape->N * shape->F), &sep, &fz);
+  *separate_tiles = sep;
+  *fused_tiles = fz;
+  *fused = whole_call_fused(shape, a2) ? 1 : 0;
+  return SVG_OK;
 }
 
 svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o, int32_t a1,
@@ -335,12 +360,12 @@ svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void*
   if (st != SVG_OK) return st;
   if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
   if (!workspace) return fail(SVG_ERR_INVALID_ARG, "workspace is NULL");
-  const size_t need = svg_sparse_3d_attn_workspace_size(shape, S);
-  if (need == 0) return fail(SVG_ERR_INVALID_ARG, "S must be in [1, 128]");
+  const size_t need = svg_sparse_3d_attn_workspace_size(shape, a2, S);
+  if (need == 0) return fail(SVG_ERR_INVALID_ARG, "S must be in [1, 128] and a2 >= 1");
   if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if (shape->dtype == SVG_BF16) {
+  if (whole_call_fused(shape, a2)) {
     if ((st = svg_profile_heads(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, stream)) !=
         SVG_OK)
       return st;

@@ -37,7 +37,7 @@ EXPORTED = (
     "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
     "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
     "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search", "svg_block_sparse_attn_fused",
-    "svg_mixed_attn_fused",
+    "svg_mixed_attn_fused", "svg_sparse_3d_attn_plan",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -79,18 +79,19 @@ def _load() -> ctypes.CDLL:
         "svg_block_sparse_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
         "svg_banded_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _P]),
         "svg_dense_attn": (_I, [_P, _P, _P, _P, _P, _P, _P]),
-        "svg_sparse_3d_attn_workspace_size": (_Z, [_P, _I]),
+        "svg_sparse_3d_attn_workspace_size": (_Z, [_P, _I, _I]),
         "svg_sparse_3d_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P, _P]),
         "svg_profile_heads_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P]),
         "svg_selftest_wait_bound": (_I, [_P, _P, _P, _P, _P, ctypes.c_uint64, _P, _P]),
         "svg_mixed_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
         "svg_mixed_3d_attn_workspace_size": (_Z, [_P]),
         "svg_mixed_3d_attn": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _Z, _P, _P]),
-        "svg_sparse_3d_attn_host_workspace_size": (_Z, [_P, _I, _I]),
+        "svg_sparse_3d_attn_host_workspace_size": (_Z, [_P, _I, _I, _I]),
         "svg_sparse_3d_attn_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _I, _P, _Z, _P, _P]),
         "svg_mode_search_workspace_size": (_Z, [_P, _I]),
         "svg_block_sparse_attn_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
         "svg_mixed_attn_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+        "svg_sparse_3d_attn_plan": (_I, [_P, _I, _P, _P, _P]),
         "svg_mode_search": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _Z,
                                  _P]),
     }
@@ -171,8 +172,15 @@ def svg_profile_workspace_size(shape: svg_shape, S: int) -> int:
     return int(lib.svg_profile_workspace_size(ctypes.byref(shape), S))
 
 
-def svg_sparse_3d_attn_workspace_size(shape: svg_shape, S: int) -> int:
-    return int(lib.svg_sparse_3d_attn_workspace_size(ctypes.byref(shape), S))
+def svg_sparse_3d_attn_plan(shape: svg_shape, a2: int):
+    """(separate_tiles, fused_tiles, fused): the whole call's layout choice."""
+    sep, fz, fu = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+    _check(lib.svg_sparse_3d_attn_plan(ctypes.byref(shape), a2, ctypes.byref(sep), ctypes.byref(fz), ctypes.byref(fu)))
+    return int(sep.value), int(fz.value), bool(fu.value)
+
+
+def svg_sparse_3d_attn_workspace_size(shape: svg_shape, a2: int, S: int) -> int:
+    return int(lib.svg_sparse_3d_attn_workspace_size(ctypes.byref(shape), a2, S))
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
@@ -307,7 +315,7 @@ def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Te
     if label is None:
         label = torch.empty(shape.B, shape.H, dtype=torch.int8, device=q.device)
     if workspace is None:
-        workspace = alloc_workspace(svg_sparse_3d_attn_workspace_size(shape, S), q.device)
+        workspace = alloc_workspace(svg_sparse_3d_attn_workspace_size(shape, a2, S), q.device)
     _check(lib.svg_sparse_3d_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), a1, a2, _ptr(rows), S,
                                   _ptr(mse), _ptr(label), _ptr(workspace), workspace.numel(), _ptr(status),
                                   _stream(stream)))
@@ -376,7 +384,7 @@ def svg_sparse_3d_attn_host(q, k, v, N: int, F: int, a1: int, a2: int, rows, *, 
     if label is None:
         label = torch.empty(shape.B, shape.H, dtype=torch.int8, pin_memory=True)
     if workspace is None:
-        need = int(lib.svg_sparse_3d_attn_host_workspace_size(ctypes.byref(shape), rows.numel(), heads_per_chunk))
+        need = int(lib.svg_sparse_3d_attn_host_workspace_size(ctypes.byref(shape), a2, rows.numel(), heads_per_chunk))
         workspace = alloc_workspace(need, dev)
     _check(lib.svg_sparse_3d_attn_host(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), a1, a2, _ptr(rows),
                                        rows.numel(), _ptr(mse), _ptr(label), heads_per_chunk, _ptr(workspace),
@@ -417,7 +425,8 @@ def svg_selftest_wait_bound(q, k, v, N: int, F: int, status, *, wait_ns: int = 5
 
 class SparseAttention3D:
     """A reusable sparse 3D-attention call for one video shape: keeps its
-    workspace between calls (profile -> permute -> attention -> unpermute)."""
+    workspace between calls (svg_sparse_3d_attn: profiling, then attention
+    with the layout transformation fused in or as separate passes)."""
 
     def __init__(self, N: int, F: int, a1: int, a2: int, scale: float = 0.0):
         self.N, self.F, self.a1, self.a2, self.scale = N, F, a1, a2, scale
@@ -425,7 +434,7 @@ class SparseAttention3D:
 
     def __call__(self, q, k, v, rows, *, o=None, mse=None, label=None, status=None, stream=None):
         shape = make_shape(q, self.N, self.F, self.scale)
-        need = svg_sparse_3d_attn_workspace_size(shape, rows.numel())
+        need = svg_sparse_3d_attn_workspace_size(shape, self.a2, rows.numel())
         if self._ws is None or self._ws.numel() < need or self._ws.device != q.device:
             self._ws = alloc_workspace(need, q.device)
         return svg_sparse_3d_attn(q, k, v, self.N, self.F, self.a1, self.a2, rows, o=o, mse=mse, label=label,

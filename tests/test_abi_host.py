@@ -105,13 +105,58 @@ def test_workspace_sizes():
     s = _shape(B=1, H=24, N=33, F=3600, d=128)
     prof = svg.svg_profile_workspace_size(s, 128)
     assert prof > 0 and prof % 256 == 0
-    # bf16 folds the layout transformation into attention: profiling workspace only
-    assert svg.svg_sparse_3d_attn_workspace_size(s, 128) == prof
+    # the whole call needs token-major copies only when it does not fuse the layout
+    for shp, a2, S in [(s, 281, 128), (_shape(B=1, H=48, N=13, F=1350, d=64), 181, 128), (s, 3, 128)]:
+        _, _, fused = svg.svg_sparse_3d_attn_plan(shp, a2)
+        t = shp.B * shp.H * shp.N * shp.F * shp.d * 2
+        extra = 0 if fused else 4 * ((t + 255) // 256 * 256)
+        assert svg.svg_sparse_3d_attn_workspace_size(shp, a2, S) == svg.svg_profile_workspace_size(shp, S) + extra
     f3 = _shape(B=1, H=2, N=5, F=40, d=64, dtype=svg.SVG_FP32)
     t = 2 * 5 * 40 * 64 * 4
     t_al = (t + 255) // 256 * 256
-    assert svg.svg_sparse_3d_attn_workspace_size(f3, 16) == 4 * t_al + svg.svg_profile_workspace_size(f3, 16)
+    assert svg.svg_sparse_3d_attn_workspace_size(f3, 4, 16) == 4 * t_al + svg.svg_profile_workspace_size(f3, 16)
+    assert svg.svg_sparse_3d_attn_plan(f3, 4)[2] is False  # fp32 always permutes
     assert svg.svg_profile_workspace_size(s, 0) == 0
     assert svg.svg_profile_workspace_size(s, 129) == 0
     f = _shape(dtype=svg.SVG_FP32, d=32)
     assert svg.svg_profile_workspace_size(f, 32) > 0
+
+
+def _brute_tile_counts(N, F, a):
+    """Key tiles a temporal head takes, by enumerating every CTA and every
+    128-key tile and keeping the tiles holding at least one kept key of one
+    of the CTA's rows (tiles between the first and the last such tile count
+    too: the kernels walk one contiguous tile range per frame group)."""
+    L = N * F
+    # token-major copies: CTA = 256 consecutive token-major rows x' = j N + i
+    sep = 0
+    for q0 in range(0, L, 256):
+        js = {x // N for x in range(q0, min(q0 + 256, L))}
+        keys = [y for y in range(L) if any(abs(y // N - j) < a for j in (min(js), max(js)))]
+        sep += keys[-1] // 128 - keys[0] // 128 + 1
+    # fused: frame groups of size 2^e (largest first), a tile = 2^e frames x 128/2^e positions
+    groups, left = [], N
+    while left:
+        s = 1
+        while s * 2 <= left and s < 128:
+            s *= 2
+        groups.append(s)
+        left -= s
+    fz = 0
+    for s_q in groups:
+        per = 2 * 128 // s_q
+        for p0 in range(0, F, per):
+            pos_q = range(p0, min(p0 + per, F))
+            kept = [p for p in range(F) if any(abs(p - j) < a for j in (pos_q[0], pos_q[-1]))]
+            for s_k in groups:
+                P = 128 // s_k
+                fz += kept[-1] // P - kept[0] // P + 1
+    return sep, fz
+
+
+@pytest.mark.parametrize("N,F,a", [(33, 300, 20), (13, 135, 18), (4, 64, 3), (21, 100, 33), (1, 500, 7), (130, 5, 2)])
+def test_layout_plan_tile_counts_match_enumeration(N, F, a):
+    shp = _shape(B=1, H=1, N=N, F=F, d=64)
+    sep, fz, fused = svg.svg_sparse_3d_attn_plan(shp, a)
+    assert (sep, fz) == _brute_tile_counts(N, F, min(a, F))
+    assert fused == (fz * 100 <= sep * 103)

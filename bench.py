@@ -34,10 +34,11 @@ from sparse_attention_video_profile_b200 import metrics, synth  # noqa: E402
 METRIC = "ms per sparse 3D-attention call; effective TFLOPS vs bf16 peak; speedup vs dense"
 
 # DRAM bytes (read + write) per full-size launch of the attention kernel, from
-# an ncu capture (profiles/attn_sm100_hunyuan.md), keyed by the sha256 prefix
-# of the kernel sources it was taken on.  Any other source revision reports
-# traffic as null until it is captured again.
-NCU_TRAFFIC = {("dc678c73ddaa5184", "430a4a7673ed7447"): 2.8216e9}
+# an ncu capture of a 4-head case of the same shape scaled by heads, keyed by
+# the sha256 prefix of the kernel sources it was taken on and by the layout
+# (fused or separate).  Any other revision or layout reports traffic as null
+# until it is captured again.
+NCU_TRAFFIC = {("a92ef83245fe3f99", "d2f4abb45748fc0c", "fused"): 2.8720e9}
 
 
 def attn_source_key():
@@ -477,7 +478,8 @@ def run_ours(args, wl, rank, world, local):
         "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "traffic": args.traffic if args.traffic is not None else (
-                         NCU_TRAFFIC.get(attn_source_key()) if wl.name == "hunyuan" else None),
+                         NCU_TRAFFIC.get(attn_source_key() + ("fused" if fused else "separate",))
+                         if wl.name == "hunyuan" else None),
                      "algorithmic_work": f"{flops:.4e} flops/launch = 4*d*unmasked pairs"},
         "hbm_peak_gbs": hbm,
         "clocks": clocks.summary(),

@@ -442,3 +442,130 @@ def test_mode_search_constant_values_and_full_bands():
     assert mode[0, 1] == oracle.MODE_SKIP
     loss, _ = oracle.mode_search(q, k, rng.standard_normal((1, 2, L, d)), N, F, rows, L, F, L, lam=0.7)
     np.testing.assert_allclose(loss[0, :, 1:], 0.7, atol=1e-12)
+
+
+# ------------------------------------------------------------ SVG2 pins (semantic-aware permutation, top-p)
+
+def _blobs(C, per, d, seed, spread=0.05):
+    """C well-separated blobs of `per` rows each, blob c in rows [c per, (c+1) per)."""
+    rng = np.random.default_rng(seed)
+    centers = rng.standard_normal((C, d)) * 10.0
+    x = np.concatenate([centers[c] + spread * rng.standard_normal((per, d)) for c in range(C)])
+    return x, np.repeat(np.arange(C), per)
+
+
+def test_kmeans_recovers_separated_blobs():
+    """Rows ordered by blob: the start rows floor(c L / C) are one per blob,
+    so one round assigns every row to its blob and the centroids are the
+    blob means."""
+    x, lab = _blobs(6, 20, 5, 1)
+    assign, mu, counts = oracle.kmeans(x, 6, 3)
+    np.testing.assert_array_equal(assign, lab)
+    np.testing.assert_array_equal(counts, np.full(6, 20))
+    for c in range(6):
+        np.testing.assert_allclose(mu[c], x[lab == c].mean(0), rtol=0, atol=1e-12)
+
+
+def test_kmeans_objective_never_increases():
+    x = np.random.default_rng(2).standard_normal((300, 4))
+    prev = np.inf
+    for it in range(1, 9):
+        assign, mu, _ = oracle.kmeans(x, 7, it)
+        obj = oracle.kmeans_objective(x, mu, assign)
+        assert obj <= prev + 1e-9
+        prev = obj
+
+
+def test_kmeans_fixed_point_by_brute_force():
+    """After convergence every row is at its nearest centroid (scalar-loop
+    distances) and every centroid is the mean of its rows (scalar loops)."""
+    x = np.random.default_rng(3).standard_normal((120, 3))
+    assign, mu, counts = oracle.kmeans(x, 5, 60)
+    for r in range(len(x)):
+        dist = [sum((x[r][c] - mu[j][c]) ** 2 for c in range(3)) for j in range(5)]
+        assert dist[assign[r]] <= min(dist) + 1e-12
+    for j in range(5):
+        rows = [r for r in range(len(x)) if assign[r] == j]
+        assert counts[j] == len(rows)
+        for c in range(3):
+            assert abs(mu[j][c] - sum(x[r][c] for r in rows) / len(rows)) < 1e-12
+
+
+def test_kmeans_ties_go_low_and_empty_cluster_keeps_centroid():
+    """Duplicate start rows give equal centroids: every row ties between
+    them and goes to the lower index, so the higher one is empty and keeps
+    its start value."""
+    x = np.array([[0.0, 0.0], [0.0, 0.0], [1.0, 0.0], [5.0, 5.0]])
+    np.testing.assert_array_equal(oracle.nearest_centroid(x, np.array([[1.0, 1.0], [1.0, 1.0]])), [0, 0, 0, 0])
+    x2 = np.array([[3.0, 3.0]] * 4)
+    assign, mu, counts = oracle.kmeans(x2, 2, 2)  # starts rows 0 and 2, both (3, 3)
+    np.testing.assert_array_equal(assign, [0, 0, 0, 0])
+    np.testing.assert_array_equal(counts, [4, 0])
+    np.testing.assert_array_equal(mu[1], [3.0, 3.0])
+
+
+def test_cluster_permutation_is_stable_sort():
+    assign = np.random.default_rng(4).integers(0, 6, size=50)
+    perm, offsets = oracle.cluster_permutation(assign, 7)
+    want = sorted(range(50), key=lambda r: (assign[r], r))
+    np.testing.assert_array_equal(perm, want)
+    for c in range(7):
+        assert list(assign[perm[offsets[c]:offsets[c + 1]]]) == [c] * int((assign == c).sum())
+    assert offsets[-1] == 50 and offsets[6] == offsets[7]  # cluster 6 empty
+
+
+@pytest.mark.parametrize("p", [0.3, 0.7, 0.9, 0.999])
+def test_centroid_topp_is_the_minimal_heaviest_prefix(p):
+    """The kept set (i) has mass >= p, (ii) loses that by dropping its
+    lightest member, (iii) outweighs every cluster it leaves out; with the
+    masses recomputed here from n_k exp(scale mu_q . mu_k) by scalar loops."""
+    rng = np.random.default_rng(5)
+    d = 6
+    mu_q, mu_k = rng.standard_normal((4, d)), rng.standard_normal((9, d))
+    n_k = rng.integers(0, 30, size=9)
+    n_k[3] = 0
+    sel = oracle.centroid_topp(mu_q, mu_k, n_k, p)
+    s = 1.0 / math.sqrt(d)
+    for c in range(4):
+        w = [n_k[j] * math.exp(s * sum(mu_q[c][t] * mu_k[j][t] for t in range(d))) for j in range(9)]
+        z = sum(w)
+        w = [x / z for x in w]
+        kept = [j for j in range(9) if sel[c, j]]
+        left = [j for j in range(9) if not sel[c, j]]
+        assert not sel[c, 3]
+        assert sum(w[j] for j in kept) >= p - 1e-12
+        assert sum(w[j] for j in kept) - min(w[j] for j in kept) < p
+        assert all(w[a] >= w[b] for a in kept for b in left)
+
+
+def test_centroid_topp_sizes_weight_equal_centroids():
+    """Equal centroids: the masses are the size shares (3:1), so p = 0.6
+    keeps only the large cluster and p = 0.8 keeps both; p = 1 keeps every
+    non-empty cluster."""
+    mu_q = np.array([[1.0, 0.0]])
+    mu_k = np.array([[0.5, 0.5], [0.5, 0.5], [0.5, 0.5]])
+    n_k = np.array([30, 10, 0])
+    np.testing.assert_array_equal(oracle.centroid_topp(mu_q, mu_k, n_k, 0.6), [[True, False, False]])
+    np.testing.assert_array_equal(oracle.centroid_topp(mu_q, mu_k, n_k, 0.8), [[True, True, False]])
+    np.testing.assert_array_equal(oracle.centroid_topp(mu_q, mu_k, n_k, 1.0), [[True, True, False]])
+
+
+def test_svg2_attention_special_cases_and_permutation():
+    rng = np.random.default_rng(6)
+    L, d = 40, 4
+    q, k, v = (rng.standard_normal((L, d)) for _ in range(3))
+    aq, ak = rng.integers(0, 3, L), rng.integers(0, 5, L)
+    full = np.ones((3, 5), dtype=bool)
+    np.testing.assert_allclose(oracle.svg2_attention_given(q, k, v, aq, ak, full), oracle.attention(q, k, v),
+                               rtol=1e-12, atol=1e-13)
+    sel = rng.random((3, 5)) < 0.5
+    sel[:, 0] = True
+    sel[2] = False  # query cluster 2 keeps nothing: its rows are zero
+    out = oracle.svg2_attention_given(q, k, v, aq, ak, sel)
+    mask = [[bool(sel[aq[x], ak[y]]) for y in range(L)] for x in range(L)]
+    keep = [x for x in range(L) if aq[x] != 2]
+    ref = _brute_attention(q[keep].tolist(), k.tolist(), v.tolist(), [mask[x] for x in keep], 1 / math.sqrt(d))
+    np.testing.assert_allclose(out[keep], ref, rtol=1e-12, atol=1e-13)
+    assert np.all(out[aq == 2] == 0)
+    via = oracle.svg2_attention_permuted(q, k, v, aq, ak, sel, 3, 5)
+    np.testing.assert_allclose(via, out, rtol=1e-12, atol=1e-13)

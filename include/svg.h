@@ -83,7 +83,8 @@ typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
 
 /* Bits of the device status word. */
 #define SVG_DEV_TIMEOUT 0x1u  /* a pipeline wait exceeded its bound; outputs invalid */
-#define SVG_DEV_RANGE 0x2u    /* profiling: in-band weights underflowed (see svg_profile_heads) */
+#define SVG_DEV_RANGE 0x2u    /* profiling: in-band weights underflowed (see svg_profile_heads);
+                                 semantic attention: a cluster id out of range */
 
 typedef struct svg_shape {
   int32_t B, H, N, F, d;
@@ -430,6 +431,39 @@ SVG_API svg_status svg_block_sparse_attn_fused(const svg_shape* shape, const voi
 SVG_API svg_status svg_mixed_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
                                         const int8_t* mode, int32_t window, int32_t md_half, int32_t stripe,
                                         int32_t* status_dev, void* stream);
+
+/*
+ * svg_semantic_attn_workspace_size -- workspace of svg_semantic_attn (bytes;
+ * 0 on bad arguments, fp32, or cluster counts outside [1, 1024]).
+ */
+SVG_API size_t svg_semantic_attn_workspace_size(const svg_shape* shape, int32_t Cq, int32_t Ck);
+
+/*
+ * svg_semantic_attn -- SVG2-style sparse attention given each token's
+ * cluster (SVG2 explainer, 2.A "Semantic-Aware Permutation", 2.B
+ * "Centroid-Based Top-p Selection", 2.C "Customized Attention Kernel"):
+ *   1. rows of Q are ordered by query cluster and rows of K, V by key
+ *      cluster (stable: clusters in index order, rows in original order);
+ *   2. each cluster's centroid is the mean of its rows;
+ *   3. for query cluster c_q, key cluster c_k gets the mass
+ *      n_k exp(scale mu_q . mu_k) (normalised over c_k; empty clusters 0);
+ *      clusters are taken by mass, descending (ties: lower index), until the
+ *      kept mass reaches p;
+ *   4. each query row attends to every key of the key clusters its cluster
+ *      keeps (one launch of the tcgen05 attention kernel over runs of kept
+ *      clusters), and its output lands at its original row of o.
+ * q, k, v, o: device bf16 [B,H,N*F,d], d = 64 or 128 (o frame-major like q).
+ * assign_q, assign_k: device int32 [B,H,L] cluster ids in [0, Cq) / [0, Ck)
+ *   (an id out of range sets SVG_DEV_RANGE in *status_dev and is read as 0).
+ * p in (0, 1].  selected: device uint32 [B,H,Cq,ceil(Ck/32)], written: bit c_k
+ * of word c_k/32 is set iff query cluster c_q keeps key cluster c_k.
+ * workspace: svg_semantic_attn_workspace_size bytes, 256-byte aligned.
+ * Deterministic: repeated calls return the same bits.
+ */
+SVG_API svg_status svg_semantic_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                     const int32_t* assign_q, const int32_t* assign_k, int32_t Cq, int32_t Ck,
+                                     float p, uint32_t* selected, void* workspace, size_t workspace_bytes,
+                                     int32_t* status_dev, void* stream);
 
 /*
  * svg_selftest_wait_bound -- failure-detection self-test (test hook).

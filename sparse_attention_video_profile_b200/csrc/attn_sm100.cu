@@ -75,7 +75,37 @@ struct AttnParams {
   // run together share their key positions in L2.
   int ng, bpos, cpb;
   int glog[kMaxFrameGroups], gfirst[kMaxFrameGroups], gcta[kMaxFrameGroups];
+  // SVG2 cluster-pair mode: see BandAttnArgs
+  int s2, s2_Cq, s2_Ck, s2_W;
+  const int32_t* s2_cid;
+  const int32_t* s2_perm;
+  const int32_t* s2_koff;
+  const uint32_t* s2_sel;
 };
+
+// SVG2 key tiles: 128-row tiles over the runs of consecutive kept key
+// clusters (empty clusters do not break a run; kept clusters are contiguous
+// in the permuted keys).  `u` is the CTA's union of kept key clusters.
+struct S2Run {
+  int t, end, next;  // current tile row, end of the run, first cluster after it
+};
+
+__device__ __forceinline__ bool s2_bit(const uint32_t* u, int c) { return (u[c >> 5] >> (c & 31)) & 1u; }
+
+// The first run at or after cluster `from`; end == -1 when there is none.
+__device__ __forceinline__ S2Run s2_run(const uint32_t* u, const int32_t* koff, int Ck, int from) {
+  int c = from;
+  while (c < Ck && !(s2_bit(u, c) && koff[c + 1] > koff[c])) ++c;
+  if (c == Ck) return S2Run{0, -1, Ck};
+  int e = c + 1;
+  while (e < Ck && (s2_bit(u, e) || koff[e + 1] == koff[e])) ++e;
+  return S2Run{koff[c], koff[e], e};
+}
+
+__device__ __forceinline__ void s2_next(S2Run& r, const uint32_t* u, const int32_t* koff, int Ck) {
+  r.t += 128;
+  if (r.t >= r.end) r = s2_run(u, koff, Ck, r.next);
+}
 
 template <int D>
 struct Cfg {
@@ -165,7 +195,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
+// S2: the SVG2 cluster-pair mode (its own instantiation, so the other modes
+// keep their register allocation).
+template <int D, bool S2>
 __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -181,6 +213,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   uint64_t* bar_o = bar_p + 2 * kPChunks;  // [2] P_i V done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_o + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* s2u = reinterpret_cast<uint32_t*>(tmem_slot + 2);  // [32] SVG2: union of kept key clusters
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -202,6 +235,17 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (S2 && threadIdx.x < p.s2_W) {
+    // union of the key clusters kept by the query clusters of this CTA's rows
+    const int bh_ = blockIdx.x / p.n_ctiles, q0_ = (blockIdx.x % p.n_ctiles) * 256;
+    uint32_t w = 0;
+    if (q0_ < p.L) {
+      const int32_t* cid = p.s2_cid + static_cast<size_t>(bh_) * p.L;
+      const int c0 = cid[q0_], c1 = cid[min(q0_ + 255, p.L - 1)];
+      for (int c = c0; c <= c1; ++c) w |= p.s2_sel[(static_cast<size_t>(bh_) * p.s2_Cq + c) * p.s2_W + threadIdx.x];
+    }
+    s2u[threadIdx.x] = w;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -212,13 +256,22 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   const int bh = blockIdx.x / p.n_ctiles;
   const HeadBand band = head_band(p, bh);
   const int lab = band.perm;
-  const bool fz = lab && p.fused;  // token-major head, layout transformation fused into the loads
+  const bool fz = lab && p.fused && !S2;  // token-major head, layout transformation fused into the loads
   const int L = p.L;
   bool idle = false;  // no query rows for this CTA
   int q0 = 0, kt0 = 0, nk = 0;
   // fused: Q tile group, its first position, and the key position range
   int gq = 0, pq0 = 0, kp_lo = 0, kp_hi = 0;
-  if (fz) {
+  const int32_t* s2_koff = S2 ? p.s2_koff + static_cast<size_t>(bh) * (p.s2_Ck + 1) : nullptr;
+  if (S2) {
+    if (ct * 256 >= L) {
+      idle = true;
+    } else {
+      q0 = ct * 256;
+      for (S2Run r = s2_run(s2u, s2_koff, p.s2_Ck, 0); r.end >= 0; r = s2_run(s2u, s2_koff, p.s2_Ck, r.next))
+        nk += (r.end - r.t + C::BK - 1) / C::BK;
+    }
+  } else if (fz) {
     const int blk = ct / p.cpb;
     int rem = ct - blk * p.cpb;
     while (gq < p.ng && rem >= p.gcta[gq]) rem -= p.gcta[gq++];
@@ -282,6 +335,32 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           t = kp_lo >> sh;
           t_end = kp_hi >> sh;
         }
+      }
+    } else if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads && S2) {
+      // ------------------------------------------------ TMA producer, SVG2 cluster runs
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_3d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, &p.tm_q, bar_q, h * 64, q0 + i * C::BQ, bh);
+      S2Run kr = s2_run(s2u, s2_koff, p.s2_Ck, 0);
+      for (int n = 0; n < 2 * nk; ++n) {
+        const int slot = n % C::NS;
+        const uint32_t ph = (n / C::NS) & 1;
+        if (!mbar_wait(&bar_empty[slot], ph ^ 1, p.wait_ns)) {
+          record_timeout(p, abort_flag);
+          break;
+        }
+        const CUtensorMap* tm = (n & 1) ? &p.tm_v : &p.tm_k;
+        mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
+#pragma unroll
+        for (int h = 0; h < C::HALVES; ++h)
+          tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, kr.t, bh);
+        if (n & 1) s2_next(kr, s2u, s2_koff, p.s2_Ck);
       }
     } else if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads) {
       // ------------------------------------------------ TMA producer
@@ -403,7 +482,18 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     }
     const bool row_ok = !idle && (fz ? pos_q < p.F : r < L);
     int lo_r = 0, hi_r = 0;
-    if (row_ok && !fz) row_interval(band, r, L, lo_r, hi_r);
+    if (row_ok && !fz && !S2) row_interval(band, r, L, lo_r, hi_r);
+    // SVG2: the row's kept key clusters, the key run iterator, and the first
+    // key cluster that can overlap the current tile
+    const uint32_t* s2_row = nullptr;
+    S2Run s2r{0, -1, 0};
+    int s2_kc = 0;
+    if (S2) {
+      const int cq = row_ok ? p.s2_cid[static_cast<size_t>(bh) * L + r] : 0;
+      s2_row = p.s2_sel + (static_cast<size_t>(bh) * p.s2_Cq + cq) * p.s2_W;
+      if (!idle) s2r = s2_run(s2u, s2_koff, p.s2_Ck, 0);
+      if (S2 && row_ok) x_q = p.s2_perm[static_cast<size_t>(bh) * L + r];
+    }
     int kg = 0, ksh = 7 - p.glog[0], kt = kp_lo >> ksh, kt_end = kp_hi >> ksh;  // fused key-tile iterator
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::col_s(i);
@@ -431,7 +521,34 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
 
       // keys of this tile the row keeps: columns [lo_c, hi_c)
       int lo_c, hi_c;
-      if (fz) {
+      if (S2) {
+        // 128-bit keep mask from the key clusters overlapping [t, t + 128),
+        // cut at the end of the current run: a run's last tile can reach into
+        // the next run, whose keys its own tiles count
+        const int t0 = s2r.t, lim = min(t0 + C::BK, s2r.end);
+        uint32_t km[4] = {0u, 0u, 0u, 0u};
+        while (s2_kc < p.s2_Ck - 1 && s2_koff[s2_kc + 1] <= t0) ++s2_kc;
+        for (int c = s2_kc; c < p.s2_Ck && s2_koff[c] < lim; ++c) {
+          if (!((s2_row[c >> 5] >> (c & 31)) & 1u)) continue;
+          const int a0 = max(s2_koff[c], t0) - t0, a1 = min(s2_koff[c + 1], lim) - t0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int lo = max(a0, 32 * w), hi = min(a1, 32 * w + 32);
+            if (lo < hi) {
+              const uint32_t hi_m = (hi - 32 * w == 32) ? 0xffffffffu : ((1u << (hi - 32 * w)) - 1u);
+              km[w] |= hi_m & ~((1u << (lo - 32 * w)) - 1u);
+            }
+          }
+        }
+        s2_next(s2r, s2u, s2_koff, p.s2_Ck);
+        if ((km[0] & km[1] & km[2] & km[3]) != 0xffffffffu) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((km[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+        }
+        lo_c = 0;
+        hi_c = C::BK;
+      } else if (fz) {
         // key column c holds position (kt << ksh) + (c >> lg) of the group
         const int lg = 7 - ksh, p0 = kt << ksh;
         lo_c = (pos_q - band.a + 1 - p0) * (1 << lg);
@@ -527,7 +644,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     } else if (nk == 0) {
       // skipped head: its output rows are zero
       if (row_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * L + r) * D);
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * L + x_q) * D);
 #pragma unroll
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -537,7 +654,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       // output row: token-major heads write to op, or, fused, straight to
       // the frame-major position of their row in o
       const int orow = row_ok ? x_q : 0;
-      __nv_bfloat16* out = (lab && !p.fused ? p.op : p.o) + (static_cast<size_t>(bh) * L + orow) * D;
+      __nv_bfloat16* out = (lab && !p.fused && !S2 ? p.op : p.o) + (static_cast<size_t>(bh) * L + orow) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -588,6 +705,17 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   if ((st = make_tile_map_bf16(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
   p.fused = a.fused;
   p.F = a.N > 0 ? a.L / a.N : 0;
+  p.s2 = a.s2;
+  if (a.s2) {
+    if (a.s2_Ck < 1 || a.s2_Ck > 1024 || a.s2_Cq < 1) return fail(SVG_ERR_INVALID_ARG, "cluster counts");
+    p.s2_Cq = a.s2_Cq;
+    p.s2_Ck = a.s2_Ck;
+    p.s2_W = (a.s2_Ck + 31) / 32;
+    p.s2_cid = a.s2_cid;
+    p.s2_perm = a.s2_perm;
+    p.s2_koff = a.s2_koff;
+    p.s2_sel = a.s2_sel;
+  }
   int perm_ctas = 0;
   if (a.fused) {
     if (a.N < 1 || a.L % a.N != 0) return fail(SVG_ERR_INVALID_ARG, "fused layout transformation needs N >= 1");
@@ -639,14 +767,19 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   p.withhold_loads = a.withhold_loads;
   const long long grid = static_cast<long long>(BH) * p.n_ctiles;
   if (grid > 0x7fffffffLL) return fail(SVG_ERR_UNSUPPORTED, "grid too large");
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
+  static bool attr_set[2] = {false, false};
+  if (!attr_set[a.s2 ? 1 : 0]) {
+    cudaError_t e = a.s2 ? cudaFuncSetAttribute(attn_sm100_kernel<D, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
+                         : cudaFuncSetAttribute(attn_sm100_kernel<D, false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(attention smem)");
-    attr_set = true;
+    attr_set[a.s2 ? 1 : 0] = true;
   }
-  attn_sm100_kernel<D><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  if (a.s2)
+    attn_sm100_kernel<D, true><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  else
+    attn_sm100_kernel<D, false><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_BYTES, stream>>>(p);
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 

@@ -50,11 +50,35 @@ struct BandAttnArgs {
   uint64_t wait_ns;
   int withhold_loads;   // self-test of the bounded waits (tcgen05 kernel only)
   // Fused layout transformation (tcgen05 kernel only): heads that run
-  // token-major read their rows straight from (q, k, v) by row gathers and
-  // write O rows back to frame-major positions of o; qp..op are unused.
-  // Needs N (frames) > 0.
+  // token-major read their rows straight from (q, k, v) through frame-group
+  // boxes and write O rows back to frame-major positions of o; qp..op are
+  // unused.  Needs N (frames) > 0.
   int fused;
+  // SVG2 cluster-pair mode (tcgen05 kernel only, overrides label and modes):
+  // q, k, v are the cluster-permuted tensors; query row r (permuted) is in
+  // cluster s2_cid[r] and lands at row s2_perm[r] of o; it attends to the key
+  // clusters its cluster keeps (bit ck of s2_sel[cq]), which occupy permuted
+  // key rows [s2_koff[ck], s2_koff[ck + 1]).
+  int s2, s2_Cq, s2_Ck;
+  const int32_t* s2_cid;
+  const int32_t* s2_perm;
+  const int32_t* s2_koff;
+  const uint32_t* s2_sel;
 };
+
+// SVG2 workspace pieces (bytes, 256-aligned) for B*H heads of L rows.
+struct Svg2Sizes {
+  int nblk, W;
+  size_t hist, perm, off_q, off_k, mu_q, mu_k, tensor, total;
+};
+Svg2Sizes svg2_sizes(int BH, int L, int Cq, int Ck, int d);
+svg_status svg2_sort(const int32_t* assign, int BH, int L, int C, int nblk, int32_t* hist, int32_t* perm,
+                     int32_t* cid, int32_t* off, int* status, cudaStream_t stream);
+svg_status svg2_gather(const void* src, const int32_t* perm, void* dst, int BH, int L, int d, cudaStream_t stream);
+svg_status svg2_centroids(const void* xp, const int32_t* off, int BH, int L, int C, int d, float* mu,
+                          cudaStream_t stream);
+svg_status svg2_topp(const float* mu_q, const float* mu_k, const int32_t* off_k, int BH, int Cq, int Ck, int d,
+                     float scale, float p, uint32_t* sel, cudaStream_t stream);
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);
 // Frame groups of the fused layout transformation: powers of two, largest

@@ -479,6 +479,78 @@ svg_status svg_mixed_3d_attn(const svg_shape* shape, const void* q, const void* 
   return launch_permute(1, src1, dst1, BH, shape->N, shape->F, rb, mode, false, s, SVG_MODE_MULTIDIAG);
 }
 
+size_t svg_semantic_attn_workspace_size(const svg_shape* shape, int32_t Cq, int32_t Ck) {
+  if (check_shape(shape) != SVG_OK || shape->dtype != SVG_BF16) return 0;
+  if (Cq < 1 || Ck < 1 || Cq > 1024 || Ck > 1024) return 0;
+  return svg2_sizes(shape->B * shape->H, shape->N * shape->F, Cq, Ck, shape->d).total;
+}
+
+svg_status svg_semantic_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                             const int32_t* assign_q, const int32_t* assign_k, int32_t Cq, int32_t Ck, float p,
+                             uint32_t* selected, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                             void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "semantic-aware attention runs in bf16 only");
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (!assign_q || !assign_k || !selected || !workspace) return fail(SVG_ERR_INVALID_ARG, "NULL argument");
+  if (Cq < 1 || Ck < 1 || Cq > 1024 || Ck > 1024)
+    return fail(SVG_ERR_INVALID_ARG, "cluster counts must be in [1, 1024], got %d, %d", Cq, Ck);
+  if (!(p > 0.f && p <= 1.f)) return fail(SVG_ERR_INVALID_ARG, "p must be in (0, 1]");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const int BH = shape->B * shape->H, L = shape->N * shape->F, d = shape->d;
+  const Svg2Sizes z = svg2_sizes(BH, L, Cq, Ck, d);
+  if (workspace_bytes < z.total) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, z.total);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int32_t* hist = reinterpret_cast<int32_t*>(w);
+  w += z.hist;
+  int32_t* perm_q = reinterpret_cast<int32_t*>(w);
+  int32_t* cid_q = reinterpret_cast<int32_t*>(w + z.perm);
+  int32_t* perm_k = reinterpret_cast<int32_t*>(w + 2 * z.perm);
+  int32_t* cid_k = reinterpret_cast<int32_t*>(w + 3 * z.perm);
+  w += 4 * z.perm;
+  int32_t* off_q = reinterpret_cast<int32_t*>(w);
+  w += z.off_q;
+  int32_t* off_k = reinterpret_cast<int32_t*>(w);
+  w += z.off_k;
+  float* mu_q = reinterpret_cast<float*>(w);
+  w += z.mu_q;
+  float* mu_k = reinterpret_cast<float*>(w);
+  w += z.mu_k;
+  void* qp = w;
+  void* kp = w + z.tensor;
+  void* vp = w + 2 * z.tensor;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* dev_status = nullptr;
+  if ((st = status_word(status_dev, &dev_status, s)) != SVG_OK) return st;
+  if ((st = svg2_sort(assign_q, BH, L, Cq, z.nblk, hist, perm_q, cid_q, off_q, dev_status, s)) != SVG_OK) return st;
+  if ((st = svg2_sort(assign_k, BH, L, Ck, z.nblk, hist, perm_k, cid_k, off_k, dev_status, s)) != SVG_OK) return st;
+  if ((st = svg2_gather(q, perm_q, qp, BH, L, d, s)) != SVG_OK) return st;
+  if ((st = svg2_gather(k, perm_k, kp, BH, L, d, s)) != SVG_OK) return st;
+  if ((st = svg2_gather(v, perm_k, vp, BH, L, d, s)) != SVG_OK) return st;
+  if ((st = svg2_centroids(qp, off_q, BH, L, Cq, d, mu_q, s)) != SVG_OK) return st;
+  if ((st = svg2_centroids(kp, off_k, BH, L, Ck, d, mu_k, s)) != SVG_OK) return st;
+  if ((st = svg2_topp(mu_q, mu_k, off_k, BH, Cq, Ck, d, eff_scale(shape), p, selected, s)) != SVG_OK) return st;
+  BandAttnArgs a{};
+  a.q = qp;
+  a.k = kp;
+  a.v = vp;
+  a.o = o;
+  a.G0 = L;
+  a.a0 = 1;
+  a.G1 = L;
+  a.a1 = 1;
+  a.s2 = 1;
+  a.s2_Cq = Cq;
+  a.s2_Ck = Ck;
+  a.s2_cid = cid_q;
+  a.s2_perm = perm_q;
+  a.s2_koff = off_k;
+  a.s2_sel = selected;
+  return run_attention(shape, a, dev_status, s);
+}
+
 size_t svg_mode_search_workspace_size(const svg_shape* shape, int32_t S) {
   if (check_shape(shape) != SVG_OK || shape->dtype != SVG_BF16) return 0;
   ProfileLayout lay;

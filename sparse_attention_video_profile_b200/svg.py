@@ -28,6 +28,7 @@ SVG_FP32 = 1
 SPATIAL = 0
 TEMPORAL = 1
 SVG_DEV_TIMEOUT = 0x1
+SVG_DEV_RANGE = 0x2
 
 # Every symbol include/svg.h declares.
 EXPORTED = (
@@ -37,7 +38,7 @@ EXPORTED = (
     "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
     "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
     "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search", "svg_block_sparse_attn_fused",
-    "svg_mixed_attn_fused", "svg_sparse_3d_attn_plan",
+    "svg_mixed_attn_fused", "svg_sparse_3d_attn_plan", "svg_semantic_attn_workspace_size", "svg_semantic_attn",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -92,6 +93,8 @@ def _load() -> ctypes.CDLL:
         "svg_block_sparse_attn_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P]),
         "svg_mixed_attn_fused": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
         "svg_sparse_3d_attn_plan": (_I, [_P, _I, _P, _P, _P]),
+        "svg_semantic_attn_workspace_size": (_Z, [_P, _I, _I]),
+        "svg_semantic_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P, _Z, _P, _P]),
         "svg_mode_search": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _Z,
                                  _P]),
     }
@@ -409,6 +412,32 @@ def svg_mode_search(q, k, v, N: int, F: int, rows, window: int, md_half: int, st
                                md_half, stripe, float(lam), float(epsilon), _ptr(loss), _ptr(mode), _ptr(workspace),
                                workspace.numel(), _stream(stream)))
     return loss, mode
+
+
+def svg_semantic_attn(q, k, v, N: int, F: int, assign_q, assign_k, Cq: int, Ck: int, p: float, *, o=None,
+                      selected=None, workspace=None, status=None, scale: float = 0.0, stream=None):
+    """SVG2-style attention given the token clusters (int32 [B,H,L] each).
+    Returns (o, selected [B,H,Cq,ceil(Ck/32)] uint32 bitmask as int32)."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    if o is None:
+        o = torch.empty_like(q)
+    if selected is None:
+        selected = torch.empty(shape.B, shape.H, Cq, (Ck + 31) // 32, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(int(lib.svg_semantic_attn_workspace_size(ctypes.byref(shape), Cq, Ck)), q.device)
+    _check(lib.svg_semantic_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(assign_q),
+                                 _ptr(assign_k), Cq, Ck, float(p), _ptr(selected), _ptr(workspace), workspace.numel(),
+                                 _ptr(status), _stream(stream)))
+    return o, selected
+
+
+def selected_bits(selected, Ck: int):
+    """[B,H,Cq,W] bitmask words -> [B,H,Cq,Ck] bool (host numpy)."""
+    import numpy as np
+    w = selected.cpu().numpy().astype(np.uint32)
+    bits = (w[..., None] >> np.arange(32, dtype=np.uint32)) & 1
+    return bits.reshape(*w.shape[:-1], -1)[..., :Ck].astype(bool)
 
 
 def svg_selftest_wait_bound(q, k, v, N: int, F: int, status, *, wait_ns: int = 50_000_000, o=None,

@@ -554,3 +554,102 @@ def test_fused_rejects_fp32():
     label = torch.zeros(1, 1, dtype=torch.int8, device=DEV)
     with pytest.raises(svg.SvgError):
         svg.svg_block_sparse_attn_fused(q, k, v, label, 4, 16, 1, 1)
+
+
+# ---------------------------------------------------------------- SVG2 semantic-aware attention
+
+def _cluster_means(x, assign, C):
+    mu = np.zeros((C, x.shape[1]))
+    n = np.bincount(assign, minlength=C)
+    np.add.at(mu, assign, x)
+    mu[n > 0] /= n[n > 0, None]
+    return mu, n
+
+
+def _check_topp_valid(sel, mu_q, mu_k, n_k, p, scale, tol=2e-4):
+    """The GPU's kept set for each query cluster against fp64 masses of the
+    same clusters: mass >= p, minimal, and heaviest (each to `tol`, the fp32
+    rounding of the GPU's masses and cumulative sum)."""
+    logits = scale * mu_q @ mu_k.T
+    w = np.where(n_k[None] > 0, n_k[None] * np.exp(logits - logits.max(1, keepdims=True)), 0.0)
+    w = w / w.sum(1, keepdims=True)
+    for c in range(sel.shape[0]):
+        kept, left = np.nonzero(sel[c])[0], np.nonzero(~sel[c])[0]
+        assert len(kept) > 0 and np.all(n_k[kept] > 0)
+        mass = w[c, kept].sum()
+        assert mass >= p - tol, (c, mass)
+        assert mass - w[c, kept].min() < p + tol, (c, mass)
+        if len(left):
+            assert w[c, kept].min() >= w[c, left].max() - tol
+
+
+def _semantic_inputs(B, H, N, F, d, Cq, Ck, seed, iters=3):
+    q, k, v = rand_qkv(B, H, N * F, d, torch.bfloat16, seed)
+    qn, kn = f64(q), f64(k)
+    aq = np.stack([[oracle.kmeans(qn[b, h], Cq, iters)[0] for h in range(H)] for b in range(B)]).astype(np.int32)
+    ak = np.stack([[oracle.kmeans(kn[b, h], Ck, iters)[0] for h in range(H)] for b in range(B)]).astype(np.int32)
+    return q, k, v, aq, ak
+
+
+@pytest.mark.parametrize("N,F,d,Cq,Ck,p", [(4, 300, 128, 8, 24, 0.9), (3, 211, 64, 5, 40, 0.6), (2, 700, 128, 16, 64, 0.95),
+                                           (1, 100, 64, 3, 7, 0.5)])
+def test_semantic_attention(N, F, d, Cq, Ck, p):
+    B, H = 1, 2
+    q, k, v, aq, ak = _semantic_inputs(B, H, N, F, d, Cq, Ck, 70 + F)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    aq_t, ak_t = (torch.from_numpy(a).to(DEV) for a in (aq, ak))
+    o, sel = svg.svg_semantic_attn(q, k, v, N, F, aq_t, ak_t, Cq, Ck, p, status=status)
+    o2, sel2 = svg.svg_semantic_attn(q, k, v, N, F, aq_t, ak_t, Cq, Ck, p, status=status)
+    sync_ok(status)
+    assert torch.equal(o, o2) and torch.equal(sel, sel2)  # deterministic
+    bits = svg.selected_bits(sel, Ck)
+    scale = 1.0 / np.sqrt(d)
+    for h in range(H):
+        qh, kh, vh = f64(q)[0, h], f64(k)[0, h], f64(v)[0, h]
+        mu_q, _ = _cluster_means(qh, aq[0, h], Cq)
+        mu_k, n_k = _cluster_means(kh, ak[0, h], Ck)
+        _check_topp_valid(bits[0, h], mu_q, mu_k, n_k, p, scale)
+        ref = oracle.svg2_attention_given(qh, kh, vh, aq[0, h], ak[0, h], bits[0, h])
+        assert_close(f64(o[0, h]), ref, torch.bfloat16, f"semantic head {h}")
+
+
+def test_semantic_attention_p1_is_dense_and_bad_ids_flagged():
+    N, F, d, Cq, Ck = 3, 200, 128, 6, 20
+    q, k, v, aq, ak = _semantic_inputs(1, 2, N, F, d, Cq, Ck, 81)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, sel = svg.svg_semantic_attn(q, k, v, N, F, torch.from_numpy(aq).to(DEV), torch.from_numpy(ak).to(DEV), Cq, Ck,
+                                   1.0, status=status)
+    sync_ok(status)
+    bits = svg.selected_bits(sel, Ck)
+    nonempty = np.stack([np.bincount(ak[0, h], minlength=Ck) > 0 for h in range(2)])
+    np.testing.assert_array_equal(bits[0], np.repeat(nonempty[:, None, :], Cq, axis=1))
+    assert_close(f64(o), oracle.dense_attention(f64(q), f64(k), f64(v)), torch.bfloat16, "p = 1")
+    bad = aq.copy()
+    bad[0, 1, 17] = Cq + 5
+    status.zero_()
+    svg.svg_semantic_attn(q, k, v, N, F, torch.from_numpy(bad).to(DEV), torch.from_numpy(ak).to(DEV), Cq, Ck, 0.9,
+                          status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & svg.SVG_DEV_RANGE
+
+
+def test_semantic_attention_video_shape_sampled():
+    """HunyuanVideo shape, Cq = 128, Ck = 512, hashed cluster ids: sampled
+    rows of two heads against the oracle under the GPU's selection."""
+    wl = synth.WORKLOADS["hunyuan"]
+    Cq, Ck, p = 128, 512, 0.9
+    q, k, v = synth.make_qkv(wl, seed=3, device=DEV)
+    x = np.arange(wl.L, dtype=np.int64)
+    aq = np.stack([((x * 2654435761 + 97 * h) >> 7) % Cq for h in range(wl.H)]).astype(np.int32)[None]
+    ak = np.stack([((x * 40503 + 31 * h) >> 5) % Ck for h in range(wl.H)]).astype(np.int32)[None]
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, sel = svg.svg_semantic_attn(q, k, v, wl.N, wl.F, torch.from_numpy(aq).to(DEV), torch.from_numpy(ak).to(DEV),
+                                   Cq, Ck, p, status=status)
+    sync_ok(status)
+    bits = svg.selected_bits(sel, Ck)
+    rows = sampled_rows(wl, n_extra=12)
+    idx = torch.from_numpy(rows).to(DEV)
+    for h in (0, 17):
+        qh, kh, vh = f64(q)[0, h], f64(k)[0, h], f64(v)[0, h]
+        ref = oracle.svg2_attention_given(qh, kh, vh, aq[0, h], ak[0, h], bits[0, h], rows=rows)
+        assert_close(f64(o[0, h, idx]), ref, torch.bfloat16, f"semantic video head {h}")

@@ -466,6 +466,37 @@ SVG_API svg_status svg_semantic_attn(const svg_shape* shape, const void* q, cons
                                      int32_t* status_dev, void* stream);
 
 /*
+ * svg_kmeans_workspace_size / svg_kmeans -- k-means of every head's rows of x
+ * (SVG2 explainer, 2.A: Q and K are clustered independently by k-means).
+ * Lloyd's algorithm, `iters` rounds from the rows floor(c L / C): each row
+ * goes to the nearest centroid (squared Euclidean distance, the centroid
+ * rounded to bf16 for the product, ties to the lower index; tcgen05 GEMM with
+ * the argmin in its epilogue), then each centroid becomes the mean of its
+ * rows (fp32, summed in the rows' original order; an empty cluster keeps its
+ * centroid).  Outputs: assign device int32 [B,H,L] (the last round's) and
+ * centroids device float [B,H,C,d] (the means of that assignment).
+ * x: device bf16 [B,H,N*F,d], d = 64 or 128; 1 <= C <= min(512, L).
+ * Deterministic.  The size query returns 0 on bad arguments.
+ */
+SVG_API size_t svg_kmeans_workspace_size(const svg_shape* shape, int32_t C);
+SVG_API svg_status svg_kmeans(const svg_shape* shape, const void* x, int32_t C, int32_t iters, int32_t* assign,
+                              float* centroids, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                              void* stream);
+
+/*
+ * svg_semantic_3d_attn_workspace_size / svg_semantic_3d_attn -- the whole
+ * SVG2-style call: svg_kmeans of Q into Cq clusters and of K into Ck clusters
+ * (`iters` rounds each), then svg_semantic_attn with keep threshold p.
+ * Outputs o, assign_q / assign_k (device int32 [B,H,L]) and selected (as in
+ * svg_semantic_attn).  Cluster counts 1..512.
+ */
+SVG_API size_t svg_semantic_3d_attn_workspace_size(const svg_shape* shape, int32_t Cq, int32_t Ck);
+SVG_API svg_status svg_semantic_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                        int32_t Cq, int32_t Ck, int32_t iters, float p, int32_t* assign_q,
+                                        int32_t* assign_k, uint32_t* selected, void* workspace,
+                                        size_t workspace_bytes, int32_t* status_dev, void* stream);
+
+/*
  * svg_selftest_wait_bound -- failure-detection self-test (test hook).
  *
  * Runs the bf16 attention kernel (one band covering all keys) with its

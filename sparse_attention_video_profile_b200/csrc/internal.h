@@ -79,6 +79,10 @@ svg_status svg2_centroids(const void* xp, const int32_t* off, int BH, int L, int
                           cudaStream_t stream);
 svg_status svg2_topp(const float* mu_q, const float* mu_k, const int32_t* off_k, int BH, int Cq, int Ck, int d,
                      float scale, float p, uint32_t* sel, cudaStream_t stream);
+// k-means (kmeans_sm100.cu): workspace bytes and the Lloyd iterations.
+size_t kmeans_workspace_bytes(int BH, int L, int C, int d);
+svg_status launch_kmeans(const void* x, int BH, int L, int C, int d, int iters, int32_t* assign, float* mu,
+                         void* workspace, int* status, cudaStream_t stream);
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);
 // Frame groups of the fused layout transformation: powers of two, largest

@@ -551,6 +551,65 @@ svg_status svg_semantic_attn(const svg_shape* shape, const void* q, const void* 
   return run_attention(shape, a, dev_status, s);
 }
 
+size_t svg_kmeans_workspace_size(const svg_shape* shape, int32_t C) {
+  if (check_shape(shape) != SVG_OK || shape->dtype != SVG_BF16 || C < 1 || C > 512) return 0;
+  return kmeans_workspace_bytes(shape->B * shape->H, shape->N * shape->F, C, shape->d);
+}
+
+svg_status svg_kmeans(const svg_shape* shape, const void* x, int32_t C, int32_t iters, int32_t* assign,
+                      float* centroids, void* workspace, size_t workspace_bytes, int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "k-means runs on bf16 rows only");
+  if ((st = check_tensors({x})) != SVG_OK) return st;
+  if (!assign || !centroids || !workspace) return fail(SVG_ERR_INVALID_ARG, "NULL assign/centroids/workspace");
+  if (C < 1 || C > 512) return fail(SVG_ERR_INVALID_ARG, "C must be in [1, 512], got %d", C);
+  if (iters < 1) return fail(SVG_ERR_INVALID_ARG, "iters must be >= 1");
+  const int L = shape->N * shape->F;
+  if (C > L) return fail(SVG_ERR_INVALID_ARG, "C = %d exceeds the %d rows", C, L);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = svg_kmeans_workspace_size(shape, C);
+  if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* dev_status = nullptr;
+  if ((st = status_word(status_dev, &dev_status, s)) != SVG_OK) return st;
+  return launch_kmeans(x, shape->B * shape->H, L, C, shape->d, iters, assign, centroids, workspace, dev_status, s);
+}
+
+size_t svg_semantic_3d_attn_workspace_size(const svg_shape* shape, int32_t Cq, int32_t Ck) {
+  const size_t km_q = svg_kmeans_workspace_size(shape, Cq), km_k = svg_kmeans_workspace_size(shape, Ck);
+  const size_t at = svg_semantic_attn_workspace_size(shape, Cq, Ck);
+  if (km_q == 0 || km_k == 0 || at == 0) return 0;
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H;
+  const size_t cent = ((BH * (Cq > Ck ? Cq : Ck) * shape->d * 4) + 255) / 256 * 256;
+  const size_t km = km_q > km_k ? km_q : km_k;
+  return (km > at ? km : at) + cent;
+}
+
+svg_status svg_semantic_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
+                                int32_t Cq, int32_t Ck, int32_t iters, float p, int32_t* assign_q, int32_t* assign_k,
+                                uint32_t* selected, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  const size_t need = svg_semantic_3d_attn_workspace_size(shape, Cq, Ck);
+  if (need == 0) return fail(SVG_ERR_INVALID_ARG, "bad shape (bf16 only) or cluster counts (1..512)");
+  if (!workspace) return fail(SVG_ERR_INVALID_ARG, "workspace is NULL");
+  if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H;
+  const size_t cent = ((BH * (Cq > Ck ? Cq : Ck) * shape->d * 4) + 255) / 256 * 256;
+  float* centroids = static_cast<float*>(workspace);  // scratch: the k-means centroids (unused afterwards)
+  void* rest = static_cast<uint8_t*>(workspace) + cent;
+  const size_t rest_bytes = workspace_bytes - cent;
+  if ((st = svg_kmeans(shape, q, Cq, iters, assign_q, centroids, rest, rest_bytes, status_dev, stream)) != SVG_OK)
+    return st;
+  if ((st = svg_kmeans(shape, k, Ck, iters, assign_k, centroids, rest, rest_bytes, status_dev, stream)) != SVG_OK)
+    return st;
+  return svg_semantic_attn(shape, q, k, v, o, assign_q, assign_k, Cq, Ck, p, selected, rest, rest_bytes, status_dev,
+                           stream);
+}
+
 size_t svg_mode_search_workspace_size(const svg_shape* shape, int32_t S) {
   if (check_shape(shape) != SVG_OK || shape->dtype != SVG_BF16) return 0;
   ProfileLayout lay;

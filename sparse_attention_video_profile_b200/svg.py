@@ -39,6 +39,7 @@ EXPORTED = (
     "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
     "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search", "svg_block_sparse_attn_fused",
     "svg_mixed_attn_fused", "svg_sparse_3d_attn_plan", "svg_semantic_attn_workspace_size", "svg_semantic_attn",
+    "svg_kmeans_workspace_size", "svg_kmeans", "svg_semantic_3d_attn_workspace_size", "svg_semantic_3d_attn",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -95,6 +96,10 @@ def _load() -> ctypes.CDLL:
         "svg_sparse_3d_attn_plan": (_I, [_P, _I, _P, _P, _P]),
         "svg_semantic_attn_workspace_size": (_Z, [_P, _I, _I]),
         "svg_semantic_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, ctypes.c_float, _P, _P, _Z, _P, _P]),
+        "svg_kmeans_workspace_size": (_Z, [_P, _I]),
+        "svg_kmeans": (_I, [_P, _P, _I, _I, _P, _P, _P, _Z, _P, _P]),
+        "svg_semantic_3d_attn_workspace_size": (_Z, [_P, _I, _I]),
+        "svg_semantic_3d_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _Z, _P, _P]),
         "svg_mode_search": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _Z,
                                  _P]),
     }
@@ -430,6 +435,45 @@ def svg_semantic_attn(q, k, v, N: int, F: int, assign_q, assign_k, Cq: int, Ck: 
                                  _ptr(assign_k), Cq, Ck, float(p), _ptr(selected), _ptr(workspace), workspace.numel(),
                                  _ptr(status), _stream(stream)))
     return o, selected
+
+
+def svg_kmeans(x, N: int, F: int, C: int, iters: int, *, assign=None, centroids=None, workspace=None, status=None,
+               stream=None):
+    """k-means of every head's rows.  Returns (assign int32 [B,H,L], centroids float32 [B,H,C,d])."""
+    shape = make_shape(x, N, F, 0.0)
+    if assign is None:
+        assign = torch.empty(shape.B, shape.H, N * F, dtype=torch.int32, device=x.device)
+    if centroids is None:
+        centroids = torch.empty(shape.B, shape.H, C, shape.d, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(int(lib.svg_kmeans_workspace_size(ctypes.byref(shape), C)), x.device)
+    _check(lib.svg_kmeans(ctypes.byref(shape), _ptr(x), C, iters, _ptr(assign), _ptr(centroids), _ptr(workspace),
+                          workspace.numel(), _ptr(status), _stream(stream)))
+    return assign, centroids
+
+
+def svg_semantic_3d_attn(q, k, v, N: int, F: int, Cq: int, Ck: int, iters: int, p: float, *, o=None, assign_q=None,
+                         assign_k=None, selected=None, workspace=None, status=None, scale: float = 0.0, stream=None):
+    """The whole SVG2-style call (k-means of Q and K, top-p, attention).
+    Returns (o, assign_q, assign_k, selected)."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    L = N * F
+    if o is None:
+        o = torch.empty_like(q)
+    if assign_q is None:
+        assign_q = torch.empty(shape.B, shape.H, L, dtype=torch.int32, device=q.device)
+    if assign_k is None:
+        assign_k = torch.empty(shape.B, shape.H, L, dtype=torch.int32, device=q.device)
+    if selected is None:
+        selected = torch.empty(shape.B, shape.H, Cq, (Ck + 31) // 32, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(int(lib.svg_semantic_3d_attn_workspace_size(ctypes.byref(shape), Cq, Ck)),
+                                    q.device)
+    _check(lib.svg_semantic_3d_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), Cq, Ck, iters, float(p),
+                                    _ptr(assign_q), _ptr(assign_k), _ptr(selected), _ptr(workspace),
+                                    workspace.numel(), _ptr(status), _stream(stream)))
+    return o, assign_q, assign_k, selected
 
 
 def selected_bits(selected, Ck: int):

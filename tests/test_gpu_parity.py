@@ -653,3 +653,93 @@ def test_semantic_attention_video_shape_sampled():
         qh, kh, vh = f64(q)[0, h], f64(k)[0, h], f64(v)[0, h]
         ref = oracle.svg2_attention_given(qh, kh, vh, aq[0, h], ak[0, h], bits[0, h], rows=rows)
         assert_close(f64(o[0, h, idx]), ref, torch.bfloat16, f"semantic video head {h}")
+
+
+# ---------------------------------------------------------------- k-means and the whole SVG2-style call
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_kmeans_recovers_blobs(d):
+    """Blobs ordered by row, so the start rows floor(c L / C) are one per
+    blob: every round assigns each row to its blob exactly."""
+    C, per, H = 12, 64, 2
+    rng = np.random.default_rng(d)
+    xs, labs = [], []
+    for h in range(H):
+        centers = rng.standard_normal((C, d)) * 4.0
+        xs.append(np.concatenate([centers[c] + 0.05 * rng.standard_normal((per, d)) for c in range(C)]))
+        labs.append(np.repeat(np.arange(C), per))
+    x = torch.from_numpy(np.stack(xs)[None]).to(torch.bfloat16).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assign, mu = svg.svg_kmeans(x, 1, C * per, C, 3, status=status)
+    sync_ok(status)
+    xn = f64(x)[0]
+    for h in range(H):
+        np.testing.assert_array_equal(assign.cpu().numpy()[0, h], labs[h])
+        for c in range(C):
+            np.testing.assert_allclose(mu.cpu().numpy()[0, h, c], xn[h][labs[h] == c].mean(0), rtol=0, atol=1e-5)
+
+
+@pytest.mark.parametrize("d,C", [(128, 40), (64, 300), (128, 512)])
+def test_kmeans_one_round_and_several(d, C):
+    N, F, H = 3, 700, 2
+    q, _, _ = rand_qkv(1, H, N * F, d, torch.bfloat16, 90 + C)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    a1, mu1 = svg.svg_kmeans(q, N, F, C, 1, status=status)
+    a5, mu5 = svg.svg_kmeans(q, N, F, C, 5, status=status)
+    a5b, mu5b = svg.svg_kmeans(q, N, F, C, 5, status=status)
+    sync_ok(status)
+    assert torch.equal(a5, a5b) and torch.equal(mu5, mu5b)  # deterministic
+    L = N * F
+    init = (np.arange(C) * L) // C
+    for h in range(H):
+        x = f64(q)[0, h]
+        # one round: the nearest start row (bf16 start rows are exact), up to rounding of the scores
+        d2 = ((x[:, None, :] - x[init][None, :, :]) ** 2).sum(-1)
+        g = a1.cpu().numpy()[0, h]
+        gap = d2[np.arange(L), g] - d2.min(1)
+        assert np.all(gap <= 1e-3 * (1.0 + d2.min(1))), float(gap.max())
+        ref_mu, n = _cluster_means(x, g, C)
+        got = mu1.cpu().numpy()[0, h]
+        np.testing.assert_allclose(got[n > 0], ref_mu[n > 0], rtol=0, atol=2e-5)
+        np.testing.assert_array_equal(got[n == 0], x[init][n == 0])  # empty clusters keep their start row
+        # five rounds: close to the oracle's objective from the same start
+        g5 = a5.cpu().numpy()[0, h]
+        obj_gpu = oracle.kmeans_objective(x, _cluster_means(x, g5, C)[0], g5)
+        ga, gmu, _ = oracle.kmeans(x, C, 5)
+        obj_ref = oracle.kmeans_objective(x, gmu, ga)
+        assert abs(obj_gpu - obj_ref) <= 0.02 * obj_ref, (obj_gpu, obj_ref)
+
+
+def test_semantic_3d_attn_whole_call():
+    N, F, d, Cq, Ck, p = 4, 300, 128, 10, 40, 0.9
+    q, k, v = rand_qkv(1, 2, N * F, d, torch.bfloat16, 95)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, aq, ak, sel = svg.svg_semantic_3d_attn(q, k, v, N, F, Cq, Ck, 4, p, status=status)
+    sync_ok(status)
+    aq, ak = aq.cpu().numpy(), ak.cpu().numpy()
+    bits = svg.selected_bits(sel, Ck)
+    for h in range(2):
+        qh, kh, vh = f64(q)[0, h], f64(k)[0, h], f64(v)[0, h]
+        mu_q, _ = _cluster_means(qh, aq[0, h], Cq)
+        mu_k, n_k = _cluster_means(kh, ak[0, h], Ck)
+        _check_topp_valid(bits[0, h], mu_q, mu_k, n_k, p, 1 / np.sqrt(d))
+        ref = oracle.svg2_attention_given(qh, kh, vh, aq[0, h], ak[0, h], bits[0, h])
+        assert_close(f64(o[0, h]), ref, torch.bfloat16, f"svg2 call head {h}")
+
+
+def test_semantic_3d_attn_video_shape_sampled():
+    wl = synth.WORKLOADS["hunyuan"]
+    prm = synth.SVG2_PARAMS
+    q, k, v = synth.make_qkv(wl, seed=4, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, aq, ak, sel = svg.svg_semantic_3d_attn(q, k, v, wl.N, wl.F, prm["Cq"], prm["Ck"], prm["iters"], prm["p"],
+                                              status=status)
+    sync_ok(status)
+    aq, ak = aq.cpu().numpy(), ak.cpu().numpy()
+    bits = svg.selected_bits(sel, prm["Ck"])
+    rows = sampled_rows(wl, n_extra=12)
+    idx = torch.from_numpy(rows).to(DEV)
+    for h in (5, 20):
+        qh, kh, vh = f64(q)[0, h], f64(k)[0, h], f64(v)[0, h]
+        ref = oracle.svg2_attention_given(qh, kh, vh, aq[0, h], ak[0, h], bits[0, h], rows=rows)
+        assert_close(f64(o[0, h, idx]), ref, torch.bfloat16, f"svg2 video head {h}")

@@ -193,6 +193,34 @@ def oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=16, n_attn_rows=16, se
     return per_call_s * 1e3, desc, t_prof + t_attn
 
 
+def oracle_sample_svg2(wl, qkv64, n_attn_rows=16, seed=0):
+    """The fp64 oracle on a bounded sample of one SVG2-style call, scaled
+    linearly: one Lloyd round of k-means of one head's Q and of its K (the
+    call runs `iters` rounds of both on every head), the centroid top-p of
+    that head, and the masked attention of n_attn_rows of its query rows.
+    Returns (ms_per_call_estimate, description, seconds_spent)."""
+    import oracle  # test infrastructure: only this baseline leg runs it
+    prm = synth.SVG2_PARAMS
+    qn, kn, vn = (x[0, 0] for x in qkv64)
+    t0 = time.perf_counter()
+    aq, mu_q, _ = oracle.kmeans(qn, prm["Cq"], 1)
+    ak, mu_k, n_k = oracle.kmeans(kn, prm["Ck"], 1)
+    t_km = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    sel = oracle.centroid_topp(mu_q, mu_k, n_k, prm["p"])
+    t_sel = time.perf_counter() - t0
+    rows = np.sort(np.random.default_rng(seed).choice(wl.L, n_attn_rows, replace=False))
+    t0 = time.perf_counter()
+    oracle.svg2_attention_given(qn, kn, vn, aq, ak, sel, rows=rows)
+    t_attn = time.perf_counter() - t0
+    heads = wl.B * wl.H
+    per_call_s = (t_km * prm["iters"] + t_sel) * heads + t_attn * (wl.L / n_attn_rows) * heads
+    desc = (f"fp64 oracle: one k-means round of Q ({prm['Cq']}) and K ({prm['Ck']}) clusters, the top-p selection, "
+            f"and the attention of {n_attn_rows} of the {wl.L} query rows, all on 1 of the {heads} heads, scaled "
+            f"linearly to the call ({prm['iters']} rounds, all rows and heads)")
+    return per_call_s * 1e3, desc, t_km + t_sel + t_attn
+
+
 def cpu_cores():
     try:
         import threadpoolctl
@@ -215,12 +243,19 @@ def run_reference(args, wl, rank, world):
     labels = synth.head_kinds(wl, 0)
     qkv64 = head_f64(wl, q, k, v)
     del q, k, v
+    svg2 = wl.name == "svg2"
     for w in range(args.warmup):
-        oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=4, n_attn_rows=4, seed=1000 + w)
+        if svg2:
+            oracle_sample_svg2(wl, qkv64, n_attn_rows=4, seed=1000 + w)
+        else:
+            oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=4, n_attn_rows=4, seed=1000 + w)
     ests, secs = [], 0.0
     desc = ""
     for s in range(args.steps):
-        ms, desc, sec = oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=32, n_attn_rows=64, seed=s)
+        if svg2:
+            ms, desc, sec = oracle_sample_svg2(wl, qkv64, n_attn_rows=32, seed=s)
+        else:
+            ms, desc, sec = oracle_sample(wl, qkv64, rows_np, labels, n_prof_rows=32, n_attn_rows=64, seed=s)
         ests.append(ms)
         secs += sec
     value = float(np.mean(ests))
@@ -242,6 +277,120 @@ def config_dict(wl, world):
             "B": wl.B, "H": wl.H, "N": wl.N, "F": wl.F, "L": wl.L, "d": wl.d, "a1": wl.a1, "a2": wl.a2, "S": wl.S,
             "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"replicas{world}" if world > 1 else "single",
             "l2": f"inputs larger than L2 (Q,K,V 3 x {wl.B * wl.H * wl.L * wl.d * 2 / 1e6:.0f} MB); no flush"}
+
+
+def run_svg2(args, wl, rank, world, local):
+    """One SVG2-style call per step on the HunyuanVideo shape: k-means of Q
+    and of K, then the semantic-aware attention (sort, gathers, centroids,
+    top-p, attention)."""
+    from sparse_attention_video_profile_b200 import svg
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    prm = synth.SVG2_PARAMS
+    Cq, Ck, iters, p = prm["Cq"], prm["Ck"], prm["iters"], prm["p"]
+    q, k, v = synth.make_qkv(wl, seed=rank, device=dev)
+    N, F, L = wl.N, wl.F, wl.L
+    shape = svg.make_shape(q, N, F)
+    o = torch.empty_like(q)
+    aq = torch.empty(wl.B, wl.H, L, dtype=torch.int32, device=dev)
+    ak = torch.empty_like(aq)
+    cq = torch.empty(wl.B, wl.H, Cq, wl.d, dtype=torch.float32, device=dev)
+    ck = torch.empty(wl.B, wl.H, Ck, wl.d, dtype=torch.float32, device=dev)
+    sel = torch.empty(wl.B, wl.H, Cq, (Ck + 31) // 32, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    km_ws = svg.alloc_workspace(max(svg.lib.svg_kmeans_workspace_size(svg.ctypes.byref(shape), Cq),
+                                    svg.lib.svg_kmeans_workspace_size(svg.ctypes.byref(shape), Ck)), dev)
+    at_ws = svg.alloc_workspace(svg.lib.svg_semantic_attn_workspace_size(svg.ctypes.byref(shape), Cq, Ck), dev)
+    names = ("kmeans_q", "kmeans_k", "attn")
+
+    def step(e=None):
+        def mark(n, i):
+            if e:
+                e[n][i].record(stream)
+        mark("kmeans_q", 0)
+        svg.svg_kmeans(q, N, F, Cq, iters, assign=aq, centroids=cq, workspace=km_ws, status=status)
+        mark("kmeans_q", 1)
+        mark("kmeans_k", 0)
+        svg.svg_kmeans(k, N, F, Ck, iters, assign=ak, centroids=ck, workspace=km_ws, status=status)
+        mark("kmeans_k", 1)
+        mark("attn", 0)
+        svg.svg_semantic_attn(q, k, v, N, F, aq, ak, Cq, Ck, p, o=o, selected=sel, workspace=at_ws, status=status)
+        mark("attn", 1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    # unmasked pairs: sum over query clusters of |c_q| x |kept keys|
+    bits = svg.selected_bits(sel, Ck)
+    aq_np, ak_np = aq.cpu().numpy(), ak.cpu().numpy()
+    pairs = 0
+    for b in range(wl.B):
+        for h in range(wl.H):
+            nq = np.bincount(aq_np[b, h], minlength=Cq)
+            nk = np.bincount(ak_np[b, h], minlength=Ck)
+            pairs += int((nq * (bits[b, h] @ nk)).sum())
+    density = pairs / (wl.B * wl.H * float(L) * L)
+    flops = metrics.attention_flops(pairs, wl.d)
+    step_events = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
+                   for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for e in step_events:
+            step(e)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status word {int(status.item())} after the timed region")
+    kern_ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in step_events) / args.steps for n in names}
+    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world)
+    value = step_ms / world
+    dense_ms = None
+    if not args.no_dense:
+        od = torch.empty_like(q)
+        svg.svg_dense_attn(q, k, v, N, F, o=od)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(2):
+            svg.svg_dense_attn(q, k, v, N, F, o=od)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = a.elapsed_time(b) / 2
+        del od
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, desc, _ = oracle_sample_svg2(wl, head_f64(wl, q, k, v), n_attn_rows=32)
+        cpu = {"value": ms, "unit": "ms/call", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    attn_tflops = flops / (kern_ms["attn"] * 1e-3) / 1e12
+    km_flops = 2.0 * wl.B * wl.H * L * wl.d * (Cq + Ck) * iters  # distance products of all rounds
+    km_tflops = km_flops / ((kern_ms["kmeans_q"] + kern_ms["kmeans_k"]) * 1e-3) / 1e12
+    line = {
+        "metric": "ms per SVG2-style sparse attention call (k-means of Q and K, top-p, attention)",
+        "value": value, "unit": "ms/call", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": dict(config_dict(wl, world), Cq=Cq, Ck=Ck, iters=iters, p=p),
+        "kernel_ms": kern_ms, "density": density,
+        "effective_tflops_attn_stage": attn_tflops,
+        "kmeans_tflops": km_tflops,
+        "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None, "dense_ms": dense_ms,
+        "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128, cluster-pair> stage (with sort, gathers, "
+                     "centroids, top-p)", "achieved": attn_tflops, "peak": peak,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "traffic": None, "algorithmic_work": f"{flops:.4e} flops = 4*d*kept pairs"},
+        "clocks": clocks.summary(),
+        "e2e": None,
+        "gpu_launches": (2 * (1 + 5 * iters) + 13) * args.steps,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def run_ours(args, wl, rank, world, local):
@@ -530,7 +679,10 @@ def main():
         raise SystemExit("no CUDA device: the benchmark measures the CUDA path only")
     rank, world, local = dist_setup(args.gpus)
     try:
-        run_ours(args, wl, rank, world, local)
+        if wl.name == "svg2":
+            run_svg2(args, wl, rank, world, local)
+        else:
+            run_ours(args, wl, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -81,6 +81,8 @@ MIXED_PARAMS = {"window": 1560, "md_half": 32, "stripe": 512}
 # SVG2-style semantic-aware attention on the HunyuanVideo shape: query / key
 # cluster counts, Lloyd rounds from the deterministic start, keep threshold.
 SVG2_PARAMS = {"Cq": 128, "Ck": 512, "iters": 8, "p": 0.9}
+WORKLOADS["svg2"] = Workload("svg2", B=1, H=24, N=33, F=3600, d=128, dtype="bf16", a1=3, a2=281, S=128,
+                             kinds="coin", weight=("uniform", 1.0, 4.0))
 # Mode shares for heads after the first five (which take modes 0..4 in order
 # so every mode is present): full, skip, diagonal, multi-diagonal, stripe.
 MIXED_MODE_P = (0.10, 0.05, 0.35, 0.30, 0.20)

@@ -13,9 +13,9 @@
 //           ring, and the score accumulator alternates between two 256-column
 //           TMEM slots so the epilogue of one overlaps the MMAs of the next.
 //   update  each centroid to the mean of its rows: the counting sort by
-//           cluster (svg2_sort), then one warp per cluster summing its rows
-//           in their original order in fp32 (deterministic); an empty
-//           cluster keeps its centroid.
+//           cluster (svg2_sort), then eight warps per cluster summing its
+//           rows in fp32 in a fixed order (deterministic); an empty cluster
+//           keeps its centroid.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -223,36 +223,65 @@ __global__ void __launch_bounds__(32) kmeans_init_kernel(const __nv_bfloat16* __
   if (lane == 0) norm[static_cast<size_t>(bh) * C + c] = n2;
 }
 
-// Each centroid becomes the mean of its rows (read through the permutation,
-// in their original order); an empty cluster keeps its centroid.
+// Each centroid becomes the mean of its rows (read through the permutation);
+// an empty cluster keeps its centroid.  kUpdWarps warps per cluster: warp w
+// sums rows w, w + W, w + 2W, ... (two rows in flight), and the partial sums
+// are added in warp order: a fixed order, so the result is deterministic.
+constexpr int kUpdWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(32) kmeans_update_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           const int32_t* __restrict__ perm,
-                                                           const int32_t* __restrict__ off, int L, int C,
-                                                           float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_b,
-                                                           float* __restrict__ norm) {
+__global__ void __launch_bounds__(kUpdWarps * 32) kmeans_update_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const int32_t* __restrict__ perm,
+                                                            const int32_t* __restrict__ off, int L, int C,
+                                                            float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_b,
+                                                            float* __restrict__ norm) {
   constexpr int PER = D / 32;
-  const int c = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+  __shared__ float part[kUpdWarps][D];
+  const int c = blockIdx.x, bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* o = off + static_cast<size_t>(bh) * (C + 1);
   const int r0 = o[c], r1 = o[c + 1];
   const size_t mo = (static_cast<size_t>(bh) * C + c) * D;
+  float s[PER], t[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) s[e] = t[e] = 0.f;
+  const __nv_bfloat16* xh = x + static_cast<size_t>(bh) * L * D;
+  const int32_t* pm = perm + static_cast<size_t>(bh) * L;
+  int r = r0 + warp;
+  for (; r + kUpdWarps < r1; r += 2 * kUpdWarps) {  // two independent rows per step
+    const __nv_bfloat16* xa = xh + static_cast<size_t>(pm[r]) * D;
+    const __nv_bfloat16* xb = xh + static_cast<size_t>(pm[r + kUpdWarps]) * D;
+    __nv_bfloat16 va[PER], vb[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      va[e] = xa[e * 32 + lane];
+      vb[e] = xb[e * 32 + lane];
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      s[e] += __bfloat162float(va[e]);
+      t[e] += __bfloat162float(vb[e]);
+    }
+  }
+  if (r < r1) {
+    const __nv_bfloat16* xa = xh + static_cast<size_t>(pm[r]) * D;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) s[e] += __bfloat162float(xa[e * 32 + lane]);
+  }
+#pragma unroll
+  for (int e = 0; e < PER; ++e) part[warp][e * 32 + lane] = s[e] + t[e];
+  __syncthreads();
+  if (warp != 0) return;
   float m[PER];
   if (r1 > r0) {
-    float s[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) s[e] = 0.f;
-    const __nv_bfloat16* xh = x + static_cast<size_t>(bh) * L * D;
-    const int32_t* pm = perm + static_cast<size_t>(bh) * L;
-    for (int r = r0; r < r1; ++r) {
-      const __nv_bfloat16* xr = xh + static_cast<size_t>(pm[r]) * D;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) s[e] += __bfloat162float(xr[e * 32 + lane]);
-    }
     const float inv = 1.f / static_cast<float>(r1 - r0);
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
-      m[e] = s[e] * inv;
-      mu[mo + e * 32 + lane] = m[e];
+      const int col = e * 32 + lane;
+      float acc = part[0][col];
+#pragma unroll
+      for (int w = 1; w < kUpdWarps; ++w) acc += part[w][col];
+      m[e] = acc * inv;
+      mu[mo + col] = m[e];
     }
   } else {
 #pragma unroll
@@ -345,9 +374,9 @@ svg_status launch_kmeans(const void* x, int BH, int L, int C, int d, int iters, 
     if (st != SVG_OK) break;
     if ((st = svg2_sort(assign, BH, L, C, nblk, hist, perm, cid, off, status, stream)) != SVG_OK) break;
     if (d == 128)
-      kmeans_update_kernel<128><<<dim3(C, BH), 32, 0, stream>>>(xb, perm, off, L, C, mu, mu_b, norm);
+      kmeans_update_kernel<128><<<dim3(C, BH), kUpdWarps * 32, 0, stream>>>(xb, perm, off, L, C, mu, mu_b, norm);
     else
-      kmeans_update_kernel<64><<<dim3(C, BH), 32, 0, stream>>>(xb, perm, off, L, C, mu, mu_b, norm);
+      kmeans_update_kernel<64><<<dim3(C, BH), kUpdWarps * 32, 0, stream>>>(xb, perm, off, L, C, mu, mu_b, norm);
     st = cuda_check(cudaGetLastError(), "k-means update launch");
   }
   return st;

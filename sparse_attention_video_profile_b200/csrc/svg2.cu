@@ -125,25 +125,36 @@ __global__ void __launch_bounds__(256) svg2_gather_kernel(const uint4* __restric
   }
 }
 
-// One warp per (cluster, head): fp32 mean of the cluster's permuted rows.
+// Four warps per (cluster, head): fp32 mean of the cluster's permuted rows;
+// warp w sums rows w, w + 4, ... and the partial sums are added in warp
+// order (deterministic).
 template <int D>
-__global__ void __launch_bounds__(32) svg2_centroid_kernel(const __nv_bfloat16* __restrict__ xp, const int32_t* __restrict__ off,
-                                                           int L, int C, float* __restrict__ mu) {
+__global__ void __launch_bounds__(128) svg2_centroid_kernel(const __nv_bfloat16* __restrict__ xp,
+                                                            const int32_t* __restrict__ off, int L, int C,
+                                                            float* __restrict__ mu) {
   constexpr int PER = D / 32;
-  const int c = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
+  __shared__ float part[4][D];
+  const int c = blockIdx.x, bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* o = off + static_cast<size_t>(bh) * (C + 1);
   const int r0 = o[c], r1 = o[c + 1];
   float s[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) s[e] = 0.f;
   const __nv_bfloat16* x = xp + static_cast<size_t>(bh) * L * D;
-  for (int r = r0; r < r1; ++r)
+  for (int r = r0 + warp; r < r1; r += 4)
 #pragma unroll
     for (int e = 0; e < PER; ++e) s[e] += __bfloat162float(x[static_cast<size_t>(r) * D + e * 32 + lane]);
+#pragma unroll
+  for (int e = 0; e < PER; ++e) part[warp][e * 32 + lane] = s[e];
+  __syncthreads();
+  if (warp != 0) return;
   const float inv = r1 > r0 ? 1.f / static_cast<float>(r1 - r0) : 0.f;
   float* m = mu + (static_cast<size_t>(bh) * C + c) * D;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) m[e * 32 + lane] = s[e] * inv;
+  for (int e = 0; e < PER; ++e) {
+    const int col = e * 32 + lane;
+    m[col] = (((part[0][col] + part[1][col]) + part[2][col]) + part[3][col]) * inv;
+  }
 }
 
 // One CTA per (query cluster, head): the kept key clusters as a bitmask.
@@ -275,9 +286,9 @@ svg_status svg2_gather(const void* src, const int32_t* perm, void* dst, int BH, 
 svg_status svg2_centroids(const void* xp, const int32_t* off, int BH, int L, int C, int d, float* mu,
                           cudaStream_t stream) {
   if (d == 128)
-    svg2_centroid_kernel<128><<<dim3(C, BH), 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(xp), off, L, C, mu);
+    svg2_centroid_kernel<128><<<dim3(C, BH), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(xp), off, L, C, mu);
   else
-    svg2_centroid_kernel<64><<<dim3(C, BH), 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(xp), off, L, C, mu);
+    svg2_centroid_kernel<64><<<dim3(C, BH), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(xp), off, L, C, mu);
   return cuda_check(cudaGetLastError(), "centroid launch");
 }
 

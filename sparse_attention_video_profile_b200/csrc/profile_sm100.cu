@@ -189,8 +189,10 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
         tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64,
                     (kt0 + (n >> 1)) * 128, bh);
     }
-  } else if (run && warp == 5 && lane == 0) {
+  } else if (run && warp == 5) {
     // ------------------------------------------------ MMA issuer
+    // The whole warp runs the loop with warp-uniform operands; one elected
+    // lane issues each tcgen05 instruction.
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
     const uint32_t ring_base = smem_u32(sRing);
@@ -201,14 +203,14 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
       const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_ts(tmem + C::col_o(v), tmem + pcol + kk * 8, b + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                (acc || kk > 0) ? 1u : 0u);
+        umma_ts_warp(tmem + C::col_o(v), tmem + pcol + kk * 8, b + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                     (acc || kk > 0) ? 1u : 0u);
     };
-    bool ok = mbar_wait(bar_q, 0, p.wait_ns);
+    bool ok = warp_wait_p(bar_q, 0, p.wait_ns);
     for (int k = 0; ok && k < nk; ++k) {
       const int nK = 2 * k, nV = 2 * k + 1;
       const int slotK = nK % C::NS, slotV = nV % C::NS;
-      ok = mbar_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+      ok = warp_wait_p(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       {
@@ -216,25 +218,25 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
-          umma_ss(tmem + C::COL_S, dq + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss_warp(tmem + C::COL_S, dq + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       }
-      umma_commit(bar_s);
-      umma_commit(&bar_empty[slotK]);
-      ok = mbar_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns) && mbar_wait(bar_p01, k & 1, p.wait_ns);
+      umma_commit_warp(bar_s);
+      umma_commit_warp(&bar_empty[slotK]);
+      ok = warp_wait_p(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns) && warp_wait_p(bar_p01, k & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       pv(0, C::COL_S, slotV, k > 0);       // O_d += P_d V
       pv(1, C::COL_S + 64, slotV, k > 0);  // O_s += P_s V
-      umma_commit(bar_o01);
-      ok = mbar_wait(bar_pt, k & 1, p.wait_ns);
+      umma_commit_warp(bar_o01);
+      ok = warp_wait_p(bar_pt, k & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       pv(2, C::COL_S, slotV, k > 0);  // O_t += P_t V
-      umma_commit(bar_ot);
-      umma_commit(&bar_empty[slotV]);
+      umma_commit_warp(bar_ot);
+      umma_commit_warp(&bar_empty[slotV]);
     }
-    if (!ok) {
+    if (!ok && lane == 0) {
       *abort_flag = 1;
       atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
     }

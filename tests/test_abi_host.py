@@ -160,3 +160,42 @@ def test_layout_plan_tile_counts_match_enumeration(N, F, a):
     sep, fz, fused = svg.svg_sparse_3d_attn_plan(shp, a)
     assert (sep, fz) == _brute_tile_counts(N, F, min(a, F))
     assert fused == (fz * 100 <= sep * 103)
+
+
+def test_semantic_and_kmeans_validation_and_sizes():
+    """Argument checks of the SVG2-style entry points fail before any launch
+    (the pointers below are never dereferenced)."""
+    s = _shape(B=1, H=2, N=4, F=100, d=128)
+    f = _shape(B=1, H=2, N=4, F=100, d=64, dtype=svg.SVG_FP32)
+    lib = svg.lib
+    assert lib.svg_semantic_attn_workspace_size(ctypes.byref(s), 16, 64) > 0
+    assert lib.svg_semantic_attn_workspace_size(ctypes.byref(f), 16, 64) == 0       # fp32
+    assert lib.svg_semantic_attn_workspace_size(ctypes.byref(s), 16, 1025) == 0     # Ck > 1024
+    assert lib.svg_semantic_attn_workspace_size(ctypes.byref(s), 0, 64) == 0
+    assert lib.svg_kmeans_workspace_size(ctypes.byref(s), 512) > 0
+    assert lib.svg_kmeans_workspace_size(ctypes.byref(s), 513) == 0                 # C > 512
+    assert lib.svg_kmeans_workspace_size(ctypes.byref(f), 8) == 0
+    ws3 = lib.svg_semantic_3d_attn_workspace_size(ctypes.byref(s), 16, 64)
+    assert ws3 >= lib.svg_semantic_attn_workspace_size(ctypes.byref(s), 16, 64)
+    assert ws3 >= lib.svg_kmeans_workspace_size(ctypes.byref(s), 64)
+    p = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 24)
+    big = ctypes.c_size_t(1 << 40)
+    sem = lib.svg_semantic_attn
+    assert sem(ctypes.byref(s), p, p, p, p, p, p, 16, 64, ctypes.c_float(0.0), p, ws, big, None, None) == 1  # p = 0
+    assert sem(ctypes.byref(s), p, p, p, p, p, p, 16, 64, ctypes.c_float(1.5), p, ws, big, None, None) == 1  # p > 1
+    assert sem(ctypes.byref(s), p, p, p, p, None, p, 16, 64, ctypes.c_float(0.9), p, ws, big, None, None) == 1
+    assert sem(ctypes.byref(s), p, p, p, p, p, p, 16, 64, ctypes.c_float(0.9), p, ctypes.c_void_p((1 << 24) + 16),
+               big, None, None) == 1  # misaligned workspace
+    assert sem(ctypes.byref(s), p, p, p, p, p, p, 16, 64, ctypes.c_float(0.9), p, ws, ctypes.c_size_t(64), None,
+               None) == 5  # short workspace
+    assert sem(ctypes.byref(f), p, p, p, p, p, p, 16, 64, ctypes.c_float(0.9), p, ws, big, None, None) == 2  # fp32
+    km = lib.svg_kmeans
+    assert km(ctypes.byref(s), p, 401, 3, p, p, ws, big, None, None) == 1    # C > L (400 rows)
+    assert km(ctypes.byref(s), p, 16, 0, p, p, ws, big, None, None) == 1     # iters < 1
+    assert km(ctypes.byref(s), p, 16, 3, None, p, ws, big, None, None) == 1
+    assert km(ctypes.byref(f), p, 16, 3, p, p, ws, big, None, None) == 2     # fp32
+    fused = lib.svg_block_sparse_attn_fused
+    assert fused(ctypes.byref(f), p, p, p, p, p, 1, 1, None, None) == 2      # fp32: unsupported
+    assert fused(ctypes.byref(s), p, p, p, p, None, 1, 1, None, None) == 1   # no labels
+    assert lib.svg_mixed_attn_fused(ctypes.byref(s), p, p, p, p, p, -1, 0, 1, None, None) == 1

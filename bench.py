@@ -221,6 +221,13 @@ def oracle_sample_svg2(wl, qkv64, n_attn_rows=16, seed=0):
     return per_call_s * 1e3, desc, t_km + t_sel + t_attn
 
 
+def step_spread(step_events, names):
+    """p10 / median / p90 of the per-call device time (first kernel's start
+    to the last kernel's end of each timed call)."""
+    t = np.array([e[names[0]][0].elapsed_time(e[names[-1]][1]) for e in step_events])
+    return {"p10": float(np.percentile(t, 10)), "p50": float(np.median(t)), "p90": float(np.percentile(t, 90))}
+
+
 def cpu_cores():
     try:
         import threadpoolctl
@@ -347,6 +354,7 @@ def run_svg2(args, wl, rank, world, local):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item())} after the timed region")
     kern_ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in step_events) / args.steps for n in names}
+    spread = step_spread(step_events, names)
     step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world)
     value = step_ms / world
     dense_ms = None
@@ -376,7 +384,7 @@ def run_svg2(args, wl, rank, world, local):
         "value": value, "unit": "ms/call", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": dict(config_dict(wl, world), Cq=Cq, Ck=Ck, iters=iters, p=p),
-        "kernel_ms": kern_ms, "density": density,
+        "kernel_ms": kern_ms, "call_ms_spread": spread, "density": density,
         "effective_tflops_attn_stage": attn_tflops,
         "kmeans_tflops": km_tflops,
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None, "dense_ms": dense_ms,
@@ -510,6 +518,7 @@ def run_ours(args, wl, rank, world, local):
         torch.cuda.synchronize()
         barrier(world)
     acc = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in step_events) for n in names}
+    spread = step_spread(step_events, names)
     step_ms_local = t_start.elapsed_time(t_end) / args.steps
     if int(status.item()) != 0:
         raise RuntimeError(f"device status word {int(status.item())} after the timed region")
@@ -617,6 +626,7 @@ def run_ours(args, wl, rank, world, local):
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
         "dense_ms": dense_ms,
         "kernel_ms": kern_ms,
+        "call_ms_spread": spread,
         "layout": ("fused: token-major heads loaded by frame-group boxes in the attention kernel, no permuted copies"
                    if fused else "separate: permute -> attention -> unpermute"),
         "layout_plan": {"separate_tiles_per_head": plan_sep, "fused_tiles_per_head": plan_fused,
@@ -624,6 +634,7 @@ def run_ours(args, wl, rank, world, local):
         "permute_gbs": perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
         "unpermute_gbs": unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
         "temporal_heads": n_temporal,
+        "density": pairs / (wl.B * wl.H * float(wl.L) * wl.L),
         "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
                      "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "traffic": args.traffic if args.traffic is not None else (

@@ -127,11 +127,12 @@ struct Cfg {
 };
 
 // Pairs (of 8) per softmax row chunk whose exponentials use the FMA-pipe
-// polynomial instead of the MUFU ex2 unit.
-#ifndef SVG_EXP_POLY_PAIRS
-#define SVG_EXP_POLY_PAIRS 3
-#endif
-constexpr int kExpPoly = SVG_EXP_POLY_PAIRS;
+// polynomial instead of the MUFU ex2 unit.  A d = 64 tile has half the MMA
+// work of a d = 128 tile for the same exponentials; its best share is lower.
+template <int D>
+constexpr int exp_poly_pairs() {
+  return D == 64 ? 2 : 3;
+}
 
 // P_i is handed to the MMA issuer in this many column chunks: the first
 // P V products run while the softmax still computes the later keys.
@@ -617,7 +618,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           const int c = j * PPC + cc;
           const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
           float2 pr;
-          if ((c & 7) < kExpPoly) {  // a fixed share of the pairs on the FMA pipe
+          if ((c & 7) < exp_poly_pairs<D>()) {  // a fixed share of the pairs on the FMA pipe
             pr = exp2_poly2(x);
           } else {
             pr.x = ex2_approx(x.x);

@@ -19,8 +19,10 @@
 // go to the workspace; the combine kernels merge the chunks.
 // TMEM: S [0,128), O_d [128,128+D), O_s [128+D,128+2D), O_t [128+2D,128+3D).
 //
-// Warps 0-3: one thread per sampled row (Q gather, masks, three softmaxes,
-// epilogue).  Warp 4: TMA producer of K and V.  Warp 5: MMA issuer.
+// Warps 0-7: two threads per sampled row, one per 64-key half of each tile
+// (Q gather, masks, three softmaxes, epilogue); the halves exchange their
+// maxima through shared memory once per tile.  Warp 8: TMA producer of K and
+// V.  Warp 9: MMA issuer.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -54,8 +56,11 @@ struct PCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int NS = (D == 128) ? 5 : 8;
   static constexpr int SMEM_BAR = TILE_BYTES + NS * TILE_BYTES;
-  static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int SMEM_X = SMEM_BAR + 512;  // row-max exchange [2][2][128] + final sums [5][128] (fp32)
+  static constexpr int SMEM_BYTES = SMEM_X + 5120 + 1024;
+  // 10 warps: softmax 0-7 (warp w: rows 32 (w & 3) .. +31, key columns
+  // 64 (w >> 2) .. +63 of each tile), TMA producer 8, MMA issuer 9.
+  static constexpr int THREADS = 320;
   static constexpr uint32_t COL_S = 0;
   static constexpr uint32_t col_o(int v) { return 128u + D * v; }
 };
@@ -65,13 +70,10 @@ __device__ __forceinline__ bool warp_wait_p(uint64_t* bar, uint32_t parity, uint
   return __all_sync(0xffffffffu, ok);
 }
 
-// Bit c of a 128-bit mask (four 32-bit words), c a compile-time constant.
-__device__ __forceinline__ bool bit128(const uint32_t (&m)[4], int c) { return (m[c >> 5] >> (c & 31)) & 1u; }
-
-// Sets bits [lo, hi) of a 128-bit mask (0 <= lo, hi <= 128).
-__device__ __forceinline__ void set_range128(uint32_t (&m)[4], int lo, int hi) {
+// Sets bits [lo, hi) of a 64-bit mask held as two words (0 <= lo, hi <= 64).
+__device__ __forceinline__ void set_range64(uint32_t (&m)[2], int lo, int hi) {
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = 0; w < 2; ++w) {
     const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 32);
     if (a < b) {
       const uint32_t hi_bits = (b >= 32) ? 0xFFFFFFFFu : ((1u << b) - 1u);
@@ -80,26 +82,63 @@ __device__ __forceinline__ void set_range128(uint32_t (&m)[4], int lo, int hi) {
   }
 }
 
-// Packs P = e for the keys whose mask bit is set (0 elsewhere) as bf16 pairs
-// and returns the sum of the rounded weights.
-__device__ __forceinline__ float pack_masked(const float (&e)[128], const uint32_t (&m)[4], uint32_t (&pk)[64]) {
-  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+// P_d of one half row: the weights e (already 0 for keys outside the chunk)
+// as bf16 pairs, and the sum of the rounded weights of each 32-key word.
+__device__ __forceinline__ void pack_plain(const float (&e)[64], uint32_t (&pk)[32], float (&wsum)[2]) {
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
-    const float p0 = bit128(m, 2 * c) ? e[2 * c] : 0.f;
-    const float p1 = bit128(m, 2 * c + 1) ? e[2 * c + 1] : 0.f;
-    const uint32_t pp = pack_bf16x2(p0, p1);
-    if (c & 1) add_bf16x2_f32(a1, pp);
-    else add_bf16x2_f32(a0, pp);
-    pk[c] = pp;
+  for (int wi = 0; wi < 2; ++wi) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = wi * 16 + c;
+      const uint32_t pp = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+      if (c & 1) add_bf16x2_f32(a1, pp);
+      else add_bf16x2_f32(a0, pp);
+      pk[i] = pp;
+    }
+    wsum[wi] = (a0.x + a1.x) + (a0.y + a1.y);
   }
-  return (a0.x + a1.x) + (a0.y + a1.y);
 }
 
-template <int D>
-__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
+// A restricted variant's P of one half row: the P_d pairs with the halves
+// whose mask bit is clear set to +0; returns the sum of its rounded weights.
+// A 32-key word that the mask keeps whole reuses P_d's word sum, one it drops
+// is zero.
+__device__ __forceinline__ float pack_variant(const uint32_t (&pkd)[32], const float (&wsum)[2], const uint32_t (&m)[2],
+                                              uint32_t (&pk)[32]) {
+  float sum = 0.f;
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int wi = 0; wi < 2; ++wi) {
+    const uint32_t mw = m[wi];
+    if (mw == 0xFFFFFFFFu) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) pk[wi * 16 + c] = pkd[wi * 16 + c];
+      sum += wsum[wi];
+    } else if (mw == 0u) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) pk[wi * 16 + c] = 0u;
+    } else {
+      float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int i = wi * 16 + c;
+        const uint32_t lo = (mw >> (2 * c)) & 1u, hi = (mw >> (2 * c + 1)) & 1u;
+        const uint32_t pp = pkd[i] & (((0u - lo) & 0x0000FFFFu) | ((0u - hi) << 16));
+        if (c & 1) add_bf16x2_f32(a1, pp);
+        else add_bf16x2_f32(a0, pp);
+        pk[i] = pp;
+      }
+      sum += (a0.x + a1.x) + (a0.y + a1.y);
+    }
+  }
+  return sum;
+}
+
+// Multiplies D/2 columns of an O accumulator (this thread's TMEM lane) by alpha.
+template <int D>
+__device__ __forceinline__ void rescale_o_half(uint32_t t_o, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
     uint32_t ov[32];
     tmem_ld32(t_o + c * 32, ov);
     tmem_wait_ld();
@@ -110,19 +149,8 @@ __device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
   }
 }
 
-__device__ __forceinline__ void st_p64(uint32_t taddr, const uint32_t (&pk)[64]) {
-  uint32_t a[32], b[32];
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    a[e] = pk[e];
-    b[e] = pk[32 + e];
-  }
-  tmem_st32(taddr, a);
-  tmem_st32(taddr + 32, b);
-}
-
 template <int D>
-__global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_constant__ ProfSm100Params p) {
+__global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_constant__ ProfSm100Params p) {
   using C = PCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -133,12 +161,15 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
   uint64_t* bar_full = bars + 1;                // [NS]
   uint64_t* bar_empty = bars + 1 + C::NS;       // [NS]
   uint64_t* bar_s = bars + 1 + 2 * C::NS;       // S ready
-  uint64_t* bar_p01 = bar_s + 1;                // 128 arrivals: P_d, P_s written
+  uint64_t* bar_p01 = bar_s + 1;                // 256 arrivals: P_d, P_s written
   uint64_t* bar_o01 = bar_s + 2;                // P_d V, P_s V done
-  uint64_t* bar_pt = bar_s + 3;                 // 128 arrivals: P_t written
+  uint64_t* bar_pt = bar_s + 3;                 // 256 arrivals: P_t written
   uint64_t* bar_ot = bar_s + 4;                 // P_t V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 5);
+  uint64_t* bar_x = bar_s + 5;                  // [4] 64 arrivals: the two halves of 32 rows exchanged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_x + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xm = reinterpret_cast<float*>(smem + C::SMEM_X);  // [2 parity][2 half][128 rows] half-row maxima
+  float* fin = xm + 512;                                    // [5][128] second half's sums and counts
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x, bh = blockIdx.y;
@@ -155,13 +186,14 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(bar_s, 1);
-    mbar_init(bar_p01, 128);
+    mbar_init(bar_p01, 256);
     mbar_init(bar_o01, 1);
-    mbar_init(bar_pt, 128);
+    mbar_init(bar_pt, 256);
     mbar_init(bar_ot, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bar_x[q], 64);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -171,7 +203,7 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
   const uint32_t tmem = *tmem_slot;
   const bool run = (*abort_flag == 0);
 
-  if (run && warp == 4 && lane == 0) {
+  if (run && warp == 8 && lane == 0) {
     // ------------------------------------------------ TMA producer (K, V)
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
@@ -189,7 +221,7 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
         tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64,
                     (kt0 + (n >> 1)) * 128, bh);
     }
-  } else if (run && warp == 5) {
+  } else if (run && warp == 9) {
     // ------------------------------------------------ MMA issuer
     // The whole warp runs the loop with warp-uniform operands; one elected
     // lane issues each tcgen05 instruction.
@@ -240,18 +272,22 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
       *abort_flag = 1;
       atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
     }
-  } else if (run && warp < 4) {
+  } else if (run && warp < 8) {
     // ------------------------------------------------ rows: gather, softmax, epilogue
-    const int r = threadIdx.x;  // row of the tile = sampled-row index (padded)
+    // Two threads per sampled row: half h handles key columns [64 h, 64 h + 64)
+    // of every tile.  The halves exchange their maxima once per tile so both
+    // scale their weights by the same reference.
+    const int q = warp & 3, h = warp >> 2;
+    const int r = q * 32 + lane;  // row of the tile = sampled-row index (padded)
     const int x = min(max(p.rows[min(r, p.S - 1)], 0), p.L - 1);
-    {
+    if (h == 0) {
       // gather Q row x into the 128-byte-swizzled K-major tile layout
       const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.L + x) * D);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
         const uint4 val = __ldg(src + c);
-        const int h = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(sQ + h * C::HALF_BYTES + r * 128 + ((cc ^ (r & 7)) << 4)) = val;
+        const int hh = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(sQ + hh * C::HALF_BYTES + r * 128 + ((cc ^ (r & 7)) << 4)) = val;
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(bar_q);
@@ -275,11 +311,12 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
         hi_v[v] = min(p.L, a);
       }
     }
-    const uint32_t lane_bits = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t lane_bits = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::COL_S;
+    const uint32_t tO = tmem + lane_bits + h * (D / 2);  // + col_o(v): this half's output columns
     const float sl2 = p.sl2;
-    // One softmax reference (the running max over all kept keys) serves the
-    // three variants: P_s and P_t are P_d restricted to their masks.
+    // One softmax reference (the running max over all kept keys of the row)
+    // serves the three variants: P_s and P_t are P_d restricted to their masks.
     float m_ref = -INFINITY, l_d = 0.f, l_s = 0.f, l_t = 0.f;
     int inband_s = 0, inband_t = 0;
     bool ok = true;
@@ -289,59 +326,68 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
         break;
       }
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      uint32_t sr[2][32];
+      tmem_ld32(tS + h * 64, sr[0]);
+      tmem_ld32(tS + h * 64 + 32, sr[1]);
       tmem_wait_ld();
+      reg_fence32(sr[0]);
+      reg_fence32(sr[1]);
+      float s[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(sr[c][e]);
+      for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
 
-      const int kbase = (kt0 + k) * 128;
-      const int nvalid = min(128, y_end - kbase);  // keys of this chunk in the tile
-      // Key masks of the tile: dense (chunk end); each restricted variant
-      // either one key interval or, for the in-frame-position band, |j - j_r| < a
-      // within each frame segment of the tile.
-      uint32_t md[4] = {0u, 0u, 0u, 0u}, ms[4] = {0u, 0u, 0u, 0u}, mt[4] = {0u, 0u, 0u, 0u};
-      set_range128(md, 0, nvalid);
+      const int kbase = (kt0 + k) * 128 + h * 64;  // key of this half's first column
+      const int nv = min(64, y_end - kbase);        // keys of the chunk in this half (may be <= 0)
+      // Key masks of the restricted variants: one key interval or, for the
+      // in-frame-position band, |j - j_r| < a within each frame segment.
+      uint32_t ms[2] = {0u, 0u}, mt[2] = {0u, 0u};
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
-        uint32_t(&mv)[4] = v ? mt : ms;
+        uint32_t(&mv)[2] = v ? mt : ms;
         if (p.kind[v] == kMaskPositionBand) {
           const int a = p.par[v];
           int c = 0;
           int j0 = kbase % p.F;
-          while (c < nvalid) {  // one frame segment per pass: keys c .. c + (F - j0) - 1
-            const int seg_end = min(nvalid, c + (p.F - j0));
+          while (c < nv) {  // one frame segment per pass: keys c .. c + (F - j0) - 1
+            const int seg_end = min(nv, c + (p.F - j0));
             const int lo = max(c, c + (jr - a + 1 - j0));
             const int hi = min(seg_end, c + (jr + a - j0));
-            if (lo < hi) set_range128(mv, lo, hi);
+            if (lo < hi) set_range64(mv, lo, hi);
             c = seg_end;
             j0 = 0;
           }
         } else {
-          set_range128(mv, max(lo_v[v] - kbase, 0), min(hi_v[v] - kbase, nvalid));
+          set_range64(mv, max(lo_v[v] - kbase, 0), min(hi_v[v] - kbase, nv));
         }
       }
-      // one max over the kept keys; every variant uses it as its reference
-      if (nvalid < 128) {
+      // keys past the chunk end get weight 0 in every variant
+      if (nv < 64) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (!bit128(md, c)) s[c] = -INFINITY;
+        for (int c = 0; c < 64; ++c)
+          if (c >= nv) s[c] = -INFINITY;
       }
       float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]), m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
 #pragma unroll
-      for (int c = 8; c < 128; c += 8) {
+      for (int c = 8; c < 64; c += 8) {
         m0 = fmax3f(m0, s[c], s[c + 1]);
         m1 = fmax3f(m1, s[c + 2], s[c + 3]);
         m2 = fmax3f(m2, s[c + 4], s[c + 5]);
         m3 = fmax3f(m3, s[c + 6], s[c + 7]);
       }
-      const float m_new = fmax3f(m_ref, fmax3f(m0, m1, m2), m3);
+      const float mh = fmaxf(fmax3f(m0, m1, m2), m3);
+      // The row's maximum over the whole tile, from both halves.  The
+      // exchange also orders both halves' score loads before either half's P
+      // stores, which overwrite score columns the other half reads.
+      float* xk = xm + (k & 1) * 256;
+      xk[h * 128 + r] = mh;
+      tc_fence_before();
+      mbar_arrive(&bar_x[q]);
+      if (!warp_wait_p(&bar_x[q], k & 1, p.wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float m_new = fmax3f(m_ref, mh, xk[(h ^ 1) * 128 + r]);
       float alpha = 1.f;
       bool resc = false;
       if (m_new > m_ref + p.lazy_th) {
@@ -353,21 +399,24 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
       {
         const float2 sl2x2 = make_float2(sl2, sl2), nb2 = make_float2(nb, nb);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
-          s[2 * c] = ex2_approx(x.x);  // s now holds the weights e
-          s[2 * c + 1] = ex2_approx(x.y);
+        for (int c = 0; c < 32; ++c) {
+          const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
+          s[2 * c] = ex2_approx(xx.x);  // s now holds the weights e
+          s[2 * c + 1] = ex2_approx(xx.y);
         }
       }
-      inband_s += __popc(ms[0]) + __popc(ms[1]) + __popc(ms[2]) + __popc(ms[3]);
-      inband_t += __popc(mt[0]) + __popc(mt[1]) + __popc(mt[2]) + __popc(mt[3]);
-      uint32_t pk[64];
-      l_d = l_d * alpha + pack_masked(s, md, pk);
+      inband_s += __popc(ms[0]) + __popc(ms[1]);
+      inband_t += __popc(mt[0]) + __popc(mt[1]);
+      uint32_t pkd[32], pk[32];
+      float wsum[2];
+      pack_plain(s, pkd, wsum);
+      l_d = l_d * alpha + (wsum[0] + wsum[1]);
       __syncwarp();
-      st_p64(tS, pk);
-      l_s = l_s * alpha + pack_masked(s, ms, pk);
+      tmem_st32(tS + h * 32, pkd);  // P_d: packed columns [0, 64)
+      l_s = l_s * alpha + pack_variant(pkd, wsum, ms, pk);
       __syncwarp();
-      st_p64(tS + 64, pk);
+      tmem_st32(tS + 64 + h * 32, pk);  // P_s: packed columns [64, 128)
+      // both halves of a row take the same decision (same reference)
       const bool any_resc = k > 0 && __any_sync(0xffffffffu, resc);
       if (any_resc) {
         if (!warp_wait_p(bar_o01, (k - 1) & 1, p.wait_ns)) {
@@ -375,47 +424,66 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
           break;
         }
         tc_fence_after();
-        rescale_o<D>(tmem + lane_bits + C::col_o(0), alpha);
-        rescale_o<D>(tmem + lane_bits + C::col_o(1), alpha);
+        rescale_o_half<D>(tO + C::col_o(0), alpha);
+        rescale_o_half<D>(tO + C::col_o(1), alpha);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p01);
-      l_t = l_t * alpha + pack_masked(s, mt, pk);
+      l_t = l_t * alpha + pack_variant(pkd, wsum, mt, pk);
       // P_t goes over P_d once P_d V has read it
       if (!warp_wait_p(bar_o01, k & 1, p.wait_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      st_p64(tS, pk);
+      tmem_st32(tS + h * 32, pk);
       if (any_resc) {
         if (!warp_wait_p(bar_ot, (k - 1) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        rescale_o<D>(tmem + lane_bits + C::col_o(2), alpha);
+        rescale_o_half<D>(tO + C::col_o(2), alpha);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_pt);
     }
-    // Kept keys whose weights all underflowed relative to the shared reference
-    // (in-band logits more than ~126 / (scale log2 e) below the row max):
-    // report it rather than return a wrong label.
-    if ((inband_s > 0 && !(l_s > 0.f)) || (inband_t > 0 && !(l_t > 0.f))) atomicOr(p.status, SVG_DEV_RANGE);
+    // the first half of each row collects the second half's sums and counts
+    if (ok) {
+      if (h == 1) {
+        fin[r] = l_d;
+        fin[128 + r] = l_s;
+        fin[256 + r] = l_t;
+        fin[384 + r] = __int_as_float(inband_s);
+        fin[512 + r] = __int_as_float(inband_t);
+      }
+      mbar_arrive(&bar_x[q]);
+      ok = warp_wait_p(&bar_x[q], nk & 1, p.wait_ns);
+    }
+    if (ok && h == 0) {
+      l_d += fin[r];
+      l_s += fin[128 + r];
+      l_t += fin[256 + r];
+      inband_s += __float_as_int(fin[384 + r]);
+      inband_t += __float_as_int(fin[512 + r]);
+      // Kept keys whose weights all underflowed relative to the shared
+      // reference (in-band logits more than ~126 / (scale log2 e) below the
+      // row max): report it rather than return a wrong label.
+      if ((inband_s > 0 && !(l_s > 0.f)) || (inband_t > 0 && !(l_t > 0.f))) atomicOr(p.status, SVG_DEV_RANGE);
+    }
     if (ok && warp_wait_p(bar_ot, (nk - 1) & 1, p.wait_ns)) {
       tc_fence_after();
 #pragma unroll
       for (int v = 0; v < 3; ++v) {
         const size_t base = ((static_cast<size_t>(bh) * p.nch + chunk) * 3 + v) * 128 + r;
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + base * D);
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + base * D + h * (D / 2));
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t ov[32];
           __syncwarp();
-          tmem_ld32(tmem + lane_bits + C::col_o(v) + c * 32, ov);
+          tmem_ld32(tO + C::col_o(v) + c * 32, ov);
           tmem_wait_ld();
           reg_fence32(ov);
 #pragma unroll
@@ -423,11 +491,13 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
             dst[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
                                          __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
         }
-        const float lv = (v == 0) ? l_d : (v == 1 ? l_s : l_t);
-        const int nin = (v == 0) ? 1 : (v == 1 ? inband_s : inband_t);
-        // max in log2 units; a variant with no kept key in this chunk has none
-        p.ws_ml[base * 2 + 0] = (m_ref == -INFINITY || nin == 0) ? -INFINITY : m_ref * sl2;
-        p.ws_ml[base * 2 + 1] = lv;
+        if (h == 0) {
+          const float lv = (v == 0) ? l_d : (v == 1 ? l_s : l_t);
+          const int nin = (v == 0) ? 1 : (v == 1 ? inband_s : inband_t);
+          // max in log2 units; a variant with no kept key in this chunk has none
+          p.ws_ml[base * 2 + 0] = (m_ref == -INFINITY || nin == 0) ? -INFINITY : m_ref * sl2;
+          p.ws_ml[base * 2 + 1] = lv;
+        }
       }
     } else {
       *abort_flag = 1;
@@ -437,7 +507,7 @@ __global__ void __launch_bounds__(192, 1) profile_sm100_kernel(const __grid_cons
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -65,6 +65,13 @@ struct PCfg {
   static constexpr uint32_t col_o(int v) { return 128u + D * v; }
 };
 
+// Pairs (of 8) of each half row's exponentials computed by the FMA-pipe
+// polynomial instead of the MUFU ex2 unit.
+#ifndef SVG_PROF_POLY_PAIRS
+#define SVG_PROF_POLY_PAIRS 2
+#endif
+constexpr int kProfPolyPairs = SVG_PROF_POLY_PAIRS;
+
 __device__ __forceinline__ bool warp_wait_p(uint64_t* bar, uint32_t parity, uint64_t limit) {
   const bool ok = mbar_wait(bar, parity, limit);
   return __all_sync(0xffffffffu, ok);
@@ -165,7 +172,8 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
   uint64_t* bar_o01 = bar_s + 2;                // P_d V, P_s V done
   uint64_t* bar_pt = bar_s + 3;                 // 256 arrivals: P_t written
   uint64_t* bar_ot = bar_s + 4;                 // P_t V done
-  uint64_t* bar_x = bar_s + 5;                  // [4] 64 arrivals: the two halves of 32 rows exchanged
+  uint64_t* bar_od = bar_s + 5;                 // P_d V done (P_t may overwrite P_d)
+  uint64_t* bar_x = bar_s + 6;                  // [4] 64 arrivals: the two halves of 32 rows exchanged
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_x + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xm = reinterpret_cast<float*>(smem + C::SMEM_X);  // [2 parity][2 half][128 rows] half-row maxima
@@ -190,6 +198,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     mbar_init(bar_o01, 1);
     mbar_init(bar_pt, 256);
     mbar_init(bar_ot, 1);
+    mbar_init(bar_od, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&bar_x[q], 64);
     fence_barrier_init();
   }
@@ -258,7 +267,8 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       ok = warp_wait_p(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns) && warp_wait_p(bar_p01, k & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      pv(0, C::COL_S, slotV, k > 0);       // O_d += P_d V
+      pv(0, C::COL_S, slotV, k > 0);  // O_d += P_d V
+      umma_commit_warp(bar_od);
       pv(1, C::COL_S + 64, slotV, k > 0);  // O_s += P_s V
       umma_commit_warp(bar_o01);
       ok = warp_wait_p(bar_pt, k & 1, p.wait_ns);
@@ -401,8 +411,20 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float2 xx = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2x2, nb2);
-          s[2 * c] = ex2_approx(xx.x);  // s now holds the weights e
-          s[2 * c + 1] = ex2_approx(xx.y);
+          float2 e;
+          if ((c & 7) < kProfPolyPairs) {
+            // FMA-pipe polynomial (both halves of a row share one MUFU unit);
+            // it clamps its argument, so weights that underflow, masked keys
+            // and keys past the chunk end included, are set to 0 as ex2 does
+            e = exp2_poly2(xx);
+            e.x = xx.x < -126.f ? 0.f : e.x;
+            e.y = xx.y < -126.f ? 0.f : e.y;
+          } else {
+            e.x = ex2_approx(xx.x);
+            e.y = ex2_approx(xx.y);
+          }
+          s[2 * c] = e.x;  // s now holds the weights e
+          s[2 * c + 1] = e.y;
         }
       }
       inband_s += __popc(ms[0]) + __popc(ms[1]);
@@ -431,8 +453,8 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       tc_fence_before();
       mbar_arrive(bar_p01);
       l_t = l_t * alpha + pack_variant(pkd, wsum, mt, pk);
-      // P_t goes over P_d once P_d V has read it
-      if (!warp_wait_p(bar_o01, k & 1, p.wait_ns)) {
+      // P_t goes over P_d once P_d V has read it (P_s V may still run)
+      if (!warp_wait_p(bar_od, k & 1, p.wait_ns)) {
         ok = false;
         break;
       }

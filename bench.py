@@ -286,6 +286,27 @@ def config_dict(wl, world):
             "l2": f"inputs larger than L2 (Q,K,V 3 x {wl.B * wl.H * wl.L * wl.d * 2 / 1e6:.0f} MB); no flush"}
 
 
+def s2_computed_pairs(cid_sorted, keep, nk, rows_per_cta=256, bk=128):
+    """(query, key) pairs the cluster-pair attention kernel computes for one
+    head: each CTA of 256 cluster-sorted query rows walks the union of the key
+    clusters its query clusters keep, as runs of consecutive kept clusters in
+    the cluster-sorted key order (empty clusters do not break a run), in
+    128-key tiles; every tile is computed for all 256 rows."""
+    ne = nk > 0
+    sizes = nk[ne]
+    csum = np.concatenate(([0], np.cumsum(sizes)))
+    total = 0
+    L = cid_sorted.shape[0]
+    for q0 in range(0, L, rows_per_cta):
+        c0, c1 = cid_sorted[q0], cid_sorted[min(q0 + rows_per_cta, L) - 1]
+        u = keep[c0:c1 + 1].any(axis=0)[ne].astype(np.int8)
+        edges = np.diff(np.concatenate(([0], u, [0])))
+        starts, ends = np.flatnonzero(edges == 1), np.flatnonzero(edges == -1)
+        lens = csum[ends] - csum[starts]
+        total += int(((lens + bk - 1) // bk).sum()) * bk * rows_per_cta
+    return total
+
+
 def run_svg2(args, wl, rank, world, local):
     """One SVG2-style call per step on the HunyuanVideo shape: k-means of Q
     and of K, then the semantic-aware attention (sort, gathers, centroids,
@@ -332,11 +353,13 @@ def run_svg2(args, wl, rank, world, local):
     bits = svg.selected_bits(sel, Ck)
     aq_np, ak_np = aq.cpu().numpy(), ak.cpu().numpy()
     pairs = 0
+    computed = 0
     for b in range(wl.B):
         for h in range(wl.H):
             nq = np.bincount(aq_np[b, h], minlength=Cq)
             nk = np.bincount(ak_np[b, h], minlength=Ck)
             pairs += int((nq * (bits[b, h] @ nk)).sum())
+            computed += s2_computed_pairs(np.sort(aq_np[b, h]), bits[b, h].astype(bool), nk)
     density = pairs / (wl.B * wl.H * float(L) * L)
     flops = metrics.attention_flops(pairs, wl.d)
     step_events = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
@@ -385,6 +408,7 @@ def run_svg2(args, wl, rank, world, local):
         "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": dict(config_dict(wl, world), Cq=Cq, Ck=Ck, iters=iters, p=p),
         "kernel_ms": kern_ms, "call_ms_spread": spread, "density": density,
+        "computed_pairs": computed, "tile_efficiency": pairs / computed if computed else None,
         "effective_tflops_attn_stage": attn_tflops,
         "kmeans_tflops": km_tflops,
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None, "dense_ms": dense_ms,

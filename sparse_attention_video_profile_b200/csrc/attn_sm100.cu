@@ -107,6 +107,30 @@ __device__ __forceinline__ void s2_next(S2Run& r, const uint32_t* u, const int32
   if (r.t >= r.end) r = s2_run(u, koff, Ck, r.next);
 }
 
+// 128-bit keep mask of one row for the tile [r.t, r.t + 128) of run r: the
+// keys of the clusters the row's query cluster keeps (`row`, one bit per key
+// cluster), cut at the end of the run (a run's last tile can reach into the
+// next run, whose keys its own tiles count).  `kc` is the first key cluster
+// that can overlap the tile; it only moves forward.
+__device__ __forceinline__ void s2_tile_mask(const S2Run& r, const int32_t* koff, const uint32_t* row, int Ck,
+                                             int& kc, uint32_t (&km)[4]) {
+  const int t0 = r.t, lim = min(t0 + 128, r.end);
+  km[0] = km[1] = km[2] = km[3] = 0u;
+  while (kc < Ck - 1 && koff[kc + 1] <= t0) ++kc;
+  for (int c = kc; c < Ck && koff[c] < lim; ++c) {
+    if (!((row[c >> 5] >> (c & 31)) & 1u)) continue;
+    const int a0 = max(koff[c], t0) - t0, a1 = min(koff[c + 1], lim) - t0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int lo = max(a0, 32 * w), hi = min(a1, 32 * w + 32);
+      if (lo < hi) {
+        const uint32_t hi_m = (hi - 32 * w == 32) ? 0xffffffffu : ((1u << (hi - 32 * w)) - 1u);
+        km[w] |= hi_m & ~((1u << (lo - 32 * w)) - 1u);
+      }
+    }
+  }
+}
+
 template <int D>
 struct Cfg {
   static constexpr int BQ = 128;          // rows per Q tile (MMA M)
@@ -489,11 +513,13 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     const uint32_t* s2_row = nullptr;
     S2Run s2r{0, -1, 0};
     int s2_kc = 0;
+    uint32_t s2_km[4] = {0u, 0u, 0u, 0u};  // keep mask of the next tile, built ahead of its scores
     if (S2) {
       const int cq = row_ok ? p.s2_cid[static_cast<size_t>(bh) * L + r] : 0;
       s2_row = p.s2_sel + (static_cast<size_t>(bh) * p.s2_Cq + cq) * p.s2_W;
       if (!idle) s2r = s2_run(s2u, s2_koff, p.s2_Ck, 0);
       if (S2 && row_ok) x_q = p.s2_perm[static_cast<size_t>(bh) * L + r];
+      if (nk > 0) s2_tile_mask(s2r, s2_koff, s2_row, p.s2_Ck, s2_kc, s2_km);
     }
     int kg = 0, ksh = 7 - p.glog[0], kt = kp_lo >> ksh, kt_end = kp_hi >> ksh;  // fused key-tile iterator
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
@@ -523,29 +549,11 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       // keys of this tile the row keeps: columns [lo_c, hi_c)
       int lo_c, hi_c;
       if (S2) {
-        // 128-bit keep mask from the key clusters overlapping [t, t + 128),
-        // cut at the end of the current run: a run's last tile can reach into
-        // the next run, whose keys its own tiles count
-        const int t0 = s2r.t, lim = min(t0 + C::BK, s2r.end);
-        uint32_t km[4] = {0u, 0u, 0u, 0u};
-        while (s2_kc < p.s2_Ck - 1 && s2_koff[s2_kc + 1] <= t0) ++s2_kc;
-        for (int c = s2_kc; c < p.s2_Ck && s2_koff[c] < lim; ++c) {
-          if (!((s2_row[c >> 5] >> (c & 31)) & 1u)) continue;
-          const int a0 = max(s2_koff[c], t0) - t0, a1 = min(s2_koff[c + 1], lim) - t0;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int lo = max(a0, 32 * w), hi = min(a1, 32 * w + 32);
-            if (lo < hi) {
-              const uint32_t hi_m = (hi - 32 * w == 32) ? 0xffffffffu : ((1u << (hi - 32 * w)) - 1u);
-              km[w] |= hi_m & ~((1u << (lo - 32 * w)) - 1u);
-            }
-          }
-        }
-        s2_next(s2r, s2u, s2_koff, p.s2_Ck);
-        if ((km[0] & km[1] & km[2] & km[3]) != 0xffffffffu) {
+        // the keep mask of this tile was built while its scores were computed
+        if ((s2_km[0] & s2_km[1] & s2_km[2] & s2_km[3]) != 0xffffffffu) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (!((km[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+            if (!((s2_km[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
         }
         lo_c = 0;
         hi_c = C::BK;
@@ -639,6 +647,11 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         mbar_arrive(&bar_p[i * kPChunks + j]);
       }
       l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
+      if (S2 && k + 1 < nk) {
+        // the next tile's keep mask, while the tensor cores compute its scores
+        s2_next(s2r, s2u, s2_koff, p.s2_Ck);
+        s2_tile_mask(s2r, s2_koff, s2_row, p.s2_Ck, s2_kc, s2_km);
+      }
     }
     if (idle) {
       // no query rows here

@@ -311,6 +311,34 @@ def test_video_shape_sampled(name):
     assert set(np.unique(label_np)) <= {0, 1}
 
 
+@pytest.mark.parametrize("density", [0.05, 0.5])
+def test_density_sweep_extremes_sampled(density):
+    """HunyuanVideo shape at the ends of the 5-50 % sweep: at 5 % the whole
+    call keeps the separate layout, at 50 % the fused one with a wide band
+    (a2 = 1055).  One spatial and one temporal head: profiling against the
+    oracle, and sampled output rows against the oracle."""
+    a1, a2 = synth.HUNYUAN_SWEEP[density]
+    wl = synth.WORKLOADS["hunyuan"].with_bands(a1, a2)
+    q, k, v = synth.make_qkv(wl, seed=3, device=DEV)
+    rows_np = synth.sample_rows(wl.L, wl.S, 3)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, mse, label = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, status=status)
+    sync_ok(status)
+    label_np = label.cpu().numpy()
+    mse_np = mse.cpu().numpy()
+    heads = [int(np.flatnonzero(label_np[0] == kind)[0]) for kind in (0, 1) if (label_np[0] == kind).any()]
+    check_rows = sampled_rows(wl, n_extra=16)
+    for h in heads:
+        qn, kn, vn = (f64(t[:, h:h + 1]) for t in (q, k, v))
+        ref_mse, ref_label = oracle.profile_heads(qn, kn, vn, wl.N, wl.F, wl.a1, wl.a2, rows_np)
+        check_profile(torch.from_numpy(mse_np[:, h:h + 1]), torch.from_numpy(label_np[:, h:h + 1]),
+                      ref_mse, ref_label, q.dtype)
+        ref = oracle.sparse_attention(qn, kn, vn, label_np[:, h:h + 1], wl.N, wl.F, wl.a1, wl.a2, rows=check_rows)
+        got = f64(o[:, h:h + 1, torch.from_numpy(check_rows).to(DEV)])
+        assert_close(got, ref, q.dtype, f"density {density} head {h}")
+
+
 # ---------------------------------------------------------------- failure detection
 
 def test_bounded_waits_report_timeout_and_context_stays_usable():

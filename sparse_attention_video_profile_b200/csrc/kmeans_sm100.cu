@@ -84,8 +84,9 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
     }
     fence_barrier_init();
   }
+  // padding centroids score +inf, so they never win the argmin
   for (int c = threadIdx.x; c < p.C_pad; c += kKmThreads)
-    sNorm[c] = c < p.C ? p.norm[static_cast<size_t>(bh) * p.C + c] : 0.f;
+    sNorm[c] = c < p.C ? p.norm[static_cast<size_t>(bh) * p.C + c] : INFINITY;
   if (warp == 5) {
     tmem_alloc(tmem_slot, 2 * p.slot_cols);
     tmem_relinquish();
@@ -163,20 +164,37 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
         }
         tc_fence_after();
         const int width = min(kKmSlotCols, p.C_pad - j * kKmSlotCols);
-        for (int c0 = 0; c0 < width; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_bits + s * p.slot_cols + c0, v);
-          tmem_wait_ld();
-          reg_fence32(v);
-          const int cbase = j * kKmSlotCols + c0;
+        const uint32_t ts = tmem + lane_bits + s * p.slot_cols;
+        // 32 columns at a time, the next load in flight while this one is reduced
+        uint32_t v[2][32];
+        tmem_ld32(ts, v[0]);
+        tmem_wait_ld();
+        reg_fence32(v[0]);
+        for (int c0 = 0; c0 < width; c0 += 64) {
+          tmem_ld32(ts + c0 + 32, v[1]);  // width is a multiple of 128
+          const float* nrm = sNorm + j * kKmSlotCols + c0;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int c = cbase + e;
-            const float score = fmaf(-2.f, __uint_as_float(v[e]), sNorm[c]);
-            if (c < p.C && score < best) {
+            const float score = fmaf(-2.f, __uint_as_float(v[0][e]), nrm[e]);
+            if (score < best) {  // ascending columns: ties keep the lower index
               best = score;
-              bi = c;
+              bi = j * kKmSlotCols + c0 + e;
             }
+          }
+          tmem_wait_ld();
+          reg_fence32(v[1]);
+          if (c0 + 64 < width) tmem_ld32(ts + c0 + 64, v[0]);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float score = fmaf(-2.f, __uint_as_float(v[1][e]), nrm[32 + e]);
+            if (score < best) {
+              best = score;
+              bi = j * kKmSlotCols + c0 + 32 + e;
+            }
+          }
+          if (c0 + 64 < width) {
+            tmem_wait_ld();
+            reg_fence32(v[0]);
           }
         }
         tc_fence_before();

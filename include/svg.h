@@ -134,6 +134,21 @@ SVG_API svg_status svg_block_list(int32_t L, int32_t G, int32_t a, int32_t Bq, i
 SVG_API size_t svg_profile_workspace_size(const svg_shape* shape, int32_t S);
 
 /*
+ * svg_workspace_size -- bytes of device workspace the step-by-step call needs
+ * (svg_profile_heads -> svg_permute_qkv -> svg_block_sparse_attn ->
+ * svg_unpermute) besides the caller's q, k, v and o, for any sample count
+ * S <= 128 and at most n_temporal_heads_max temporal heads.  Layout, each part
+ * starting on a 256-byte boundary: [profiling workspace | qp | kp | vp | op].
+ * The four token-major tensors are present only when n_temporal_heads_max > 0,
+ * each the size of q: a temporal head's token-major copy sits at its own head
+ * index of a [B,H,L,d] tensor, so they do not shrink with fewer temporal heads.
+ * The whole call sizes its own workspace (svg_sparse_3d_attn_workspace_size).
+ * Returns 0 on invalid arguments (invalid shape, n_temporal_heads_max < 0 or
+ * > B*H).
+ */
+SVG_API size_t svg_workspace_size(const svg_shape* shape, int32_t n_temporal_heads_max);
+
+/*
  * svg_profile_heads -- online profiling ("Sparse Video-Gen", Weakness 1
  * answer on online profiling; "Sparse VideoGen ...", Abstract).
  *

@@ -193,6 +193,18 @@ size_t svg_profile_workspace_size(const svg_shape* shape, int32_t S) {
   return lay.total;
 }
 
+size_t svg_workspace_size(const svg_shape* shape, int32_t n_temporal_heads_max) {
+  if (check_shape(shape) != SVG_OK) return 0;
+  if (n_temporal_heads_max < 0 || n_temporal_heads_max > shape->B * shape->H) return 0;
+  const int L = shape->N * shape->F;
+  const size_t prof = svg_profile_workspace_size(shape, L < 128 ? L : 128);
+  if (prof == 0) return 0;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t elt = shape->dtype == SVG_FP32 ? 4 : 2;
+  const size_t tensor = al(static_cast<size_t>(shape->B) * shape->H * L * shape->d * elt);
+  return al(prof) + (n_temporal_heads_max > 0 ? 4 * tensor : 0);
+}
+
 svg_status svg_profile_heads(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
                              size_t workspace_bytes, void* stream) {

@@ -33,7 +33,7 @@ SVG_DEV_RANGE = 0x2
 # Every symbol include/svg.h declares.
 EXPORTED = (
     "svg_abi_version", "svg_status_string", "svg_last_error", "svg_attn_tile", "svg_block_list",
-    "svg_profile_workspace_size", "svg_profile_heads", "svg_permute", "svg_permute_qkv", "svg_unpermute",
+    "svg_profile_workspace_size", "svg_workspace_size", "svg_profile_heads", "svg_permute", "svg_permute_qkv", "svg_unpermute",
     "svg_block_sparse_attn", "svg_banded_attn", "svg_dense_attn", "svg_sparse_3d_attn_workspace_size",
     "svg_sparse_3d_attn", "svg_profile_heads_noalloc", "svg_selftest_wait_bound", "svg_mixed_attn",
     "svg_mixed_3d_attn_workspace_size", "svg_mixed_3d_attn", "svg_sparse_3d_attn_host_workspace_size",
@@ -74,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "svg_attn_tile": (_I, [_I, _I, _P, _P]),
         "svg_block_list": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P]),
         "svg_profile_workspace_size": (_Z, [_P, _I]),
+        "svg_workspace_size": (_Z, [_P, _I]),
         "svg_profile_heads": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
         "svg_permute": (_I, [_P, _P, _P, _P, _P]),
         "svg_permute_qkv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -178,6 +179,11 @@ def svg_block_list(L: int, G: int, a: int, Bq: int, Bk: int):
 
 def svg_profile_workspace_size(shape: svg_shape, S: int) -> int:
     return int(lib.svg_profile_workspace_size(ctypes.byref(shape), S))
+
+
+def svg_workspace_size(shape: svg_shape, n_temporal_heads_max: int) -> int:
+    """Workspace of the step-by-step call: [profiling | qp | kp | vp | op]."""
+    return int(lib.svg_workspace_size(ctypes.byref(shape), n_temporal_heads_max))
 
 
 def svg_sparse_3d_attn_plan(shape: svg_shape, a2: int):

@@ -120,6 +120,16 @@ def test_workspace_sizes():
     assert svg.svg_profile_workspace_size(s, 129) == 0
     f = _shape(dtype=svg.SVG_FP32, d=32)
     assert svg.svg_profile_workspace_size(f, 32) > 0
+    # the step-by-step call: [profiling workspace at S = 128 | qp | kp | vp | op]
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    t = al(s.B * s.H * s.N * s.F * s.d * 2)
+    assert svg.svg_workspace_size(s, 0) == al(prof)
+    assert svg.svg_workspace_size(s, 1) == al(prof) + 4 * t
+    assert svg.svg_workspace_size(s, 24) == al(prof) + 4 * t
+    assert svg.svg_workspace_size(s, -1) == 0 and svg.svg_workspace_size(s, 25) == 0
+    small = _shape(B=1, H=2, N=2, F=32, d=64)  # L = 64 < 128: profiling sized for S = L
+    assert svg.svg_workspace_size(small, 2) == al(svg.svg_profile_workspace_size(small, 64)) + 4 * al(2 * 64 * 64 * 2)
+    assert svg.svg_workspace_size(f3, 1) == al(svg.svg_profile_workspace_size(f3, 128)) + 4 * t_al
 
 
 def _brute_tile_counts(N, F, a):

@@ -569,3 +569,64 @@ def test_svg2_attention_special_cases_and_permutation():
     assert np.all(out[aq == 2] == 0)
     via = oracle.svg2_attention_permuted(q, k, v, aq, ak, sel, 3, 5)
     np.testing.assert_allclose(via, out, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- mixed-pattern masks, row attention, SVG2 end to end
+
+@pytest.mark.parametrize("L,W", [(7, 0), (7, 2), (12, 5), (9, 8), (9, 20)])
+def test_window_mask_bruteforce_and_count(L, W):
+    """|x - y| <= W by scalar loops; count L(2W+1) - W(W+1) while W < L."""
+    m = oracle.window_mask(L, W)
+    ref = [[abs(x - y) <= W for y in range(L)] for x in range(L)]
+    np.testing.assert_array_equal(m, np.array(ref))
+    expect = L * L if W >= L - 1 else L * (2 * W + 1) - W * (W + 1)
+    assert int(m.sum()) == expect
+    rows = [0, L // 2, L - 1]
+    np.testing.assert_array_equal(oracle.window_mask(L, W, rows), m[rows])
+
+
+@pytest.mark.parametrize("L,P", [(8, 0), (8, 3), (8, 8), (8, 11)])
+def test_prefix_mask_bruteforce_and_count(L, P):
+    """y < P by scalar loops; count L min(P, L); the same for every row."""
+    m = oracle.prefix_mask(L, P)
+    np.testing.assert_array_equal(m, np.array([[y < P for y in range(L)] for _ in range(L)]))
+    assert int(m.sum()) == L * min(P, L)
+    np.testing.assert_array_equal(oracle.prefix_mask(L, P, [1, 5]), m[[1, 5]])
+
+
+def test_head_mask_follows_the_label():
+    """Label 0 is the frame band |i1 - i2| < a1, label 1 the position band
+    |j1 - j2| < a2 (scalar loops over (i, j))."""
+    N, F, a1, a2 = 4, 5, 2, 2
+    coords = [(x // F, x % F) for x in range(N * F)]
+    sp = [[abs(i1 - i2) < a1 for (i2, _) in coords] for (i1, _) in coords]
+    tp = [[abs(j1 - j2) < a2 for (_, j2) in coords] for (_, j1) in coords]
+    np.testing.assert_array_equal(oracle.head_mask(oracle.SPATIAL, N, F, a1, a2), np.array(sp))
+    np.testing.assert_array_equal(oracle.head_mask(oracle.TEMPORAL, N, F, a1, a2), np.array(tp))
+
+
+def test_attention_rows_uniform_weights_give_window_means():
+    """With q = 0 every kept key has the same weight, so each output row is
+    the plain mean of V over its window |x - y| <= W."""
+    rng = np.random.default_rng(11)
+    L, d, W = 50, 6, 4
+    q = np.zeros((L, d))
+    k, v = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    rows = np.array([0, 1, 3, 25, 47, 49])
+    out = oracle.attention_rows(q, k, v, rows, lambda rr: oracle.window_mask(L, W, rr), chunk=4)
+    ref = np.array([v[max(0, x - W):min(L, x + W + 1)].mean(axis=0) for x in rows])
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-14)
+
+
+def test_svg2_attention_with_p_one_is_dense():
+    """Top-p with p = 1 keeps every non-empty key cluster for every query
+    cluster, so the whole SVG2 step is dense attention, whatever the
+    clustering."""
+    rng = np.random.default_rng(12)
+    L, d = 60, 8
+    q, k, v = (rng.standard_normal((L, d)) for _ in range(3))
+    out, aq, ak, sel = oracle.svg2_attention(q, k, v, 4, 6, 3, 1.0)
+    probs = np.exp(q @ k.T / math.sqrt(d))
+    probs /= probs.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(out, probs @ v, rtol=1e-11, atol=1e-12)
+    assert aq.shape == (L,) and ak.shape == (L,) and sel.shape == (4, 6)

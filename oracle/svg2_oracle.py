@@ -16,7 +16,7 @@ Source: the SVG2 explainer (gist.science), section 2 "Methodology":
   2.C "Customized Attention Kernel" -- contiguous query clusters attend to
       the selected (variable-size) key clusters.
 
-Readings taken where the page is silent (each also listed in the design doc):
+Readings taken where the page is silent:
   * k-means is Lloyd's algorithm with Euclidean distance, run for a fixed
     number of iterations from a deterministic start: centroid c is the row
     floor(c * L / C).  A row goes to its nearest centroid (ties: the lowest

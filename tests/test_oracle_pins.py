@@ -466,6 +466,30 @@ def test_kmeans_recovers_separated_blobs():
         np.testing.assert_allclose(mu[c], x[lab == c].mean(0), rtol=0, atol=1e-12)
 
 
+def test_kmeans_objective_pins():
+    """kmeans_objective is the sum of squared row-to-centroid distances: equal
+    to a scalar-loop sum, zero when every row sits at its centroid, and the
+    hand-computed value of a two-cluster case."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((37, 5))
+    mu = rng.standard_normal((4, 5))
+    assign = rng.integers(0, 4, size=37)
+    loop = sum((x[r][c] - mu[assign[r]][c]) ** 2 for r in range(37) for c in range(5))
+    assert abs(oracle.kmeans_objective(x, mu, assign) - loop) <= 1e-12 * loop
+    # every row at its centroid: objective 0 exactly
+    assert oracle.kmeans_objective(mu[assign], mu, assign) == 0.0
+    # rows (0,0), (2,0) with centroid (1,0); rows (0,3), (0,5) with centroid (0,4):
+    # 1 + 1 + 1 + 1 = 4
+    x2 = np.array([[0.0, 0.0], [2.0, 0.0], [0.0, 3.0], [0.0, 5.0]])
+    mu2 = np.array([[1.0, 0.0], [0.0, 4.0]])
+    assert oracle.kmeans_objective(x2, mu2, [0, 0, 1, 1]) == 4.0
+    # with the assignment swapped: (0,0)-(0,4): 16, (2,0)-(0,4): 4+16, (0,3)-(1,0): 1+9, (0,5)-(1,0): 1+25
+    assert oracle.kmeans_objective(x2, mu2, [1, 1, 0, 0]) == 16.0 + 20.0 + 10.0 + 26.0
+    # it weighs only the assigned centroid: an unused centroid changes nothing
+    mu3 = np.vstack([mu2, [[100.0, 100.0]]])
+    assert oracle.kmeans_objective(x2, mu3, [0, 0, 1, 1]) == 4.0
+
+
 def test_kmeans_objective_never_increases():
     x = np.random.default_rng(2).standard_normal((300, 4))
     prev = np.inf

@@ -46,8 +46,12 @@
  *             enqueued, and launch errors (SVG_ERR_CUDA) after.  Errors that
  *             happen on the device (a bounded wait that ran out) are OR-ed
  *             into the optional device word `status_dev` as SVG_DEV_* bits;
- *             read it after the stream has synchronised.  svg_last_error()
- *             gives a message for the last failing call on this host thread.
+ *             read it after the stream has synchronised.  With status_dev
+ *             NULL they go to one word per device that every such call
+ *             shares (and zeroes first), so calls that overlap on the GPU
+ *             can clear each other's bits: pass a word of your own to rely
+ *             on them.  svg_last_error() gives a message for the last
+ *             failing call on this host thread.
  *   Support.  bf16: d in {64, 128}.  fp32: d in {32, 64, 128}.  a1 >= 1,
  *             a2 >= 1 (a1 >= N or a2 >= F keep every pair of that kind).
  */
@@ -129,7 +133,9 @@ SVG_API svg_status svg_block_list(int32_t L, int32_t G, int32_t a, int32_t Bq, i
 
 /*
  * svg_profile_workspace_size -- bytes of device workspace svg_profile_heads
- * needs for this shape and sample count (0 on invalid arguments).
+ * needs for this shape and sample count (0 on invalid arguments): the
+ * per-chunk partial results, the per-row sums and the call's own device
+ * status word.
  */
 SVG_API size_t svg_profile_workspace_size(const svg_shape* shape, int32_t S);
 
@@ -161,11 +167,19 @@ SVG_API size_t svg_workspace_size(const svg_shape* shape, int32_t n_temporal_hea
  *   label[b,h] = SVG_TEMPORAL if mse[b,h,1] < mse[b,h,0] else SVG_SPATIAL.
  * The reduction order is fixed, so repeated calls give identical bits.
  * The three softmaxes of a row share one reference (the row's running max
- * over all keys), so every key needs one exponential.  If a row's in-band
- * logits all lie more than about 126 / (scale * log2(e)) below its largest
- * logit (about 990 raw units for d = 128), their weights underflow.  That
+ * over the keys of a key chunk, a contiguous range of keys the kernel takes
+ * as one unit of work), so every key needs one exponential.  If, within one
+ * chunk, a row's in-band logits all lie more than about 126 / (scale *
+ * log2(e)) below its largest logit of that chunk (about 990 raw units for
+ * d = 128), their weights underflow.  That
  * case, like a device-side wait that ran out, is reported rather than
- * returned: every label is set to -1 and every MSE to NaN.
+ * returned: every label is set to -1 and every MSE to NaN.  The call keeps
+ * its status word inside the workspace (zeroed at the start of the call), so
+ * calls with separate workspaces never see each other's failures; the whole
+ * calls (svg_sparse_3d_attn, svg_sparse_3d_attn_host) also OR the failure
+ * bits (SVG_DEV_RANGE, SVG_DEV_TIMEOUT) into their status_dev.  The
+ * attention entry points run a head whose label is not SVG_TEMPORAL (-1
+ * included) with the spatial band.
  *
  * q, k, v   device, [B,H,L,d] frame-major, dtype of shape.
  * rows      device, int32 [S], each in [0, L) (duplicates allowed), shared by
@@ -199,7 +213,10 @@ SVG_API svg_status svg_profile_heads(const svg_shape* shape, const void* q, cons
  *
  * Set-up: the first call on a device looks up the array's device address
  * (which also loads the library's kernels on that device) and remembers it.
- * Make that first call before any stream capture on that device.
+ * Make that first call before any stream capture on that device.  The
+ * remembered address belongs to the device's current CUDA context: after
+ * cudaDeviceReset the call must not be used again in the process.
+ * Failures on the device are recorded in a status word inside the array.
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents.  Nothing in it needs to start at zero, because each call
  * writes every byte it later reads.  Calls whose kernels overlap on the GPU,
@@ -249,7 +266,10 @@ SVG_API svg_status svg_unpermute(const svg_shape* shape, const void* xp, void* x
  *                  transformation.
  * All heads run in one launch; the key range of each query tile is computed
  * on the fly from (G, a); no mask tensor is read.  Rows of temporal heads in
- * o and of spatial heads in op are not written.
+ * o and of spatial heads in op are not written.  A label other than
+ * SVG_TEMPORAL (for instance the -1 of a failed profiling call) is treated
+ * as SVG_SPATIAL, as by the permute and unpermute calls, which move only
+ * SVG_TEMPORAL heads.
  *
  * q,k,v,o      device [B,H,L,d] frame-major.
  * qp,kp,vp,op  device [B,H,L,d] token-major (temporal heads' slices are used);
@@ -306,8 +326,10 @@ SVG_API svg_status svg_sparse_3d_attn_plan(const svg_shape* shape, int32_t a2, i
  * 3 % more attention work than the token-major copies (about what the two
  * permutation passes cost), counted on the host from N, F and a2; fp32
  * always permutes.  Outputs o (frame-major [B,H,L,d]) plus the profiling
- * results mse [B,H,2] and label [B,H] (device).  Arguments as in the calls
- * above.
+ * results mse [B,H,2] and label [B,H] (device).  If profiling fails on the
+ * device (see svg_profile_heads), its SVG_DEV_* bits are OR-ed into
+ * status_dev and every head, labelled -1, gets the spatial attention; both
+ * layouts give that same output.  Arguments as in the calls above.
  */
 SVG_API svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void* k, const void* v,
                               void* o, int32_t a1, int32_t a2, const int32_t* rows, int32_t S,
@@ -335,15 +357,48 @@ SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, in
  * device-to-host copies of a third overlap on two internal streams plus the
  * caller's stream.  The results are bit-identical to svg_sparse_3d_attn.
  * The call is asynchronous: `stream` resumes after the last copy-out, so
- * synchronise it before reading the host outputs.  Calls on one device must
- * not run concurrently from several host threads (the internal streams and
- * events are shared per device).
+ * synchronise it before reading the host outputs.  The internal streams
+ * and events are shared per device, so calls on one device from several
+ * host threads take a per-device lock while they enqueue (their work then
+ * runs in that order on the shared copy streams).
  */
 SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q_host, const void* k_host,
                                            const void* v_host, void* o_host, int32_t a1, int32_t a2,
                                            const int32_t* rows_host, int32_t S, float* mse_host,
                                            int8_t* label_host, int32_t heads_per_chunk, void* workspace,
                                            size_t workspace_bytes, int32_t* status_dev, void* stream);
+
+/*
+ * Head sharding across GPUs.  Every head's profiling, layout transformation
+ * and attention touch no other head, so one call splits over `world` ranks
+ * (one process per GPU) by head with no exchange on the data path.  Heads are
+ * numbered over (b, h) as g = b * H + h; rank r takes the contiguous block
+ * [first, first + count) with count = n / world or n / world + 1 (the first
+ * n % world ranks take one more), so the blocks cover every head exactly once.
+ *
+ * svg_head_shard -- that block for n_heads heads (host only; 0 <= rank <
+ * world; count may be 0 when world > n_heads).
+ */
+SVG_API svg_status svg_head_shard(int32_t n_heads, int32_t rank, int32_t world, int32_t* first, int32_t* count);
+
+/*
+ * svg_sparse_3d_attn_shard_workspace_size / svg_sparse_3d_attn_shard --
+ * svg_sparse_3d_attn on this rank's block of heads only.  q, k, v, o, mse and
+ * label are the FULL [B, H, ...] tensors on this rank's device (the same
+ * addresses' layout as for svg_sparse_3d_attn); only the block's heads are
+ * read and written, so a caller that wants the whole output gathers the
+ * blocks from the other ranks afterwards (one all-gather over NVLink), and a
+ * caller that keeps heads sharded never does.  The workspace is sized for
+ * the block.  With no heads on this rank the call does nothing and returns
+ * SVG_OK.
+ */
+SVG_API size_t svg_sparse_3d_attn_shard_workspace_size(const svg_shape* shape, int32_t rank, int32_t world,
+                                                       int32_t a2, int32_t S);
+SVG_API svg_status svg_sparse_3d_attn_shard(const svg_shape* shape, int32_t rank, int32_t world, const void* q,
+                                            const void* k, const void* v, void* o, int32_t a1, int32_t a2,
+                                            const int32_t* rows, int32_t S, float* mse, int8_t* label,
+                                            void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                            void* stream);
 
 /*
  * Mixed sparse patterns ("Sparse-vDiT" review, pith.science, "What carries

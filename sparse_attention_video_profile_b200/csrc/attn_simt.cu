@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
   if (gid >= static_cast<long long>(BH) * L) return;
   const int bh = static_cast<int>(gid / L);
   const int x = static_cast<int>(gid - static_cast<long long>(bh) * L);
-  const int lab = label ? label[bh] : 0;
+  const int lab = (label != nullptr && label[bh] == SVG_TEMPORAL) ? 1 : 0;  // any other label runs spatial
   const int G = lab ? G1 : G0, a = lab ? a1 : a0;
   const size_t hoff = static_cast<size_t>(bh) * L * D;
   const float* q = (lab ? q1 : q0) + hoff;

@@ -210,8 +210,12 @@ __device__ __forceinline__ HeadBand head_band(const AttnParams& p, int bh) {
       default: return HeadBand{kSkip, 1, 0, 0};
     }
   }
-  const int lab = p.label ? static_cast<int>(p.label[bh]) : 0;
-  return lab ? HeadBand{kGroup, p.G1, p.a1, 1} : HeadBand{kGroup, p.G0, p.a0, 0};
+  // Only SVG_TEMPORAL selects the token-major band; any other value (the -1
+  // a failed profiling call writes included) runs the spatial band on the
+  // frame-major tensors, as the permute and unpermute kernels move only
+  // SVG_TEMPORAL heads.
+  const bool temporal = p.label != nullptr && p.label[bh] == SVG_TEMPORAL;
+  return temporal ? HeadBand{kGroup, p.G1, p.a1, 1} : HeadBand{kGroup, p.G0, p.a0, 0};
 }
 
 // Warp-uniform bounded wait.

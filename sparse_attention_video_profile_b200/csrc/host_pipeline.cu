@@ -30,13 +30,17 @@ struct PipeResources {
 
 std::mutex g_pipe_mutex;
 PipeResources g_pipe[kMaxDevices];
+// Held by a call for its whole enqueue: the streams and events of a device
+// are shared, so two host threads must not interleave their records and waits.
+std::mutex g_enqueue_mutex[kMaxDevices];
 
 // Streams and events of the current device, created on first use and kept.
-svg_status pipe_resources(PipeResources** out) {
+svg_status pipe_resources(PipeResources** out, int* dev_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_check(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(SVG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  *dev_out = dev;
   std::lock_guard<std::mutex> lock(g_pipe_mutex);
   PipeResources& r = g_pipe[dev];
   if (!r.ready) {
@@ -119,8 +123,10 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
   const size_t head_bytes = static_cast<size_t>(shape->N) * shape->F * shape->d * es;
 
   PipeResources* r = nullptr;
-  svg_status st = pipe_resources(&r);
+  int dev = 0;
+  svg_status st = pipe_resources(&r, &dev);
   if (st != SVG_OK) return st;
+  std::lock_guard<std::mutex> enqueue_lock(g_enqueue_mutex[dev]);
   const cudaStream_t sc = static_cast<cudaStream_t>(stream);
   cudaError_t e;
 #define SVG_CU(call, what)                                   \
@@ -161,7 +167,8 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
     svg_shape cs = *shape;
     cs.B = 1;
     cs.H = nh;
-    if ((st = svg_profile_heads(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, stream)) != SVG_OK) return st;
+    if ((st = profile_heads_impl(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, status_dev, sc)) != SVG_OK)
+      return st;
     if (fused) {
       if ((st = svg_block_sparse_attn_fused(&cs, q, k, v, o, lab, a1, a2, status_dev, stream)) != SVG_OK) return st;
     } else {

@@ -114,17 +114,25 @@ struct ProfileLayout {
   size_t o_bytes;     // partial outputs  [BH][n_chunks][3][S_pad][d] f32
   size_t ml_bytes;    // partial max/sum  [BH][n_chunks][3][S_pad][2] f32
   size_t part_bytes;  // per-row sums [BH][S_pad][3] f64: (O_1 - O_d)^2, (O_2 - O_d)^2, O_d^2
-  size_t total;
+  size_t status_bytes;  // the call's own device status word (int32, zeroed by the call), padded to 256 bytes
+  size_t total;         // o_bytes + ml_bytes + part_bytes + status_bytes
 };
+
+// Offset of the call's status word inside a profiling workspace.
+inline size_t profile_status_offset(const ProfileLayout& lay) { return lay.o_bytes + lay.ml_bytes + lay.part_bytes; }
 
 // Workspace layout of the profiling kernels.  max_chunks > 0 caps the number
 // of key chunks (fewer chunks need less workspace); fp32 always uses one.
 bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks = 0);
 
+// Online profiling.  Device-side failures (a wait that ran out, in-band
+// weights that underflowed) are recorded in the status word inside `ws`
+// (zeroed first, so calls with separate workspaces do not interfere) and,
+// when status_out is not NULL, also OR-ed into *status_out.
 svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
                           const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
                           float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
-                          cudaStream_t stream);
+                          int* status_out, cudaStream_t stream);
 
 // Masks of the two restricted variants of a profiling pass.
 constexpr int kProfFrameBand = 0;     // |i_x - i_y| < a           (spatial)
@@ -154,6 +162,13 @@ svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, co
                               const ProfileLayout& lay, double* part2, cudaStream_t stream);
 
 // A zeroed per-device status word for kernels whose entry point takes none.
+// It is shared by every such call on the device.
 svg_status internal_status_word(int** out, cudaStream_t stream);
+
+// svg_profile_heads with the failure bits also OR-ed into status_out (may be
+// NULL); the whole calls use it to carry a profiling failure to the caller.
+svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
+                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
+                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream);
 
 }  // namespace svg

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 // writes the two MSEs and the label.
 __global__ void __launch_bounds__(kCombineThreads)
     profile_finalize_kernel(const double* __restrict__ part, int S, int S_pad, int D, float* __restrict__ mse,
-                            int8_t* __restrict__ label, const int* __restrict__ status) {
+                            int8_t* __restrict__ label, const int* __restrict__ status, int* __restrict__ status_out) {
   __shared__ double red[2][kCombineThreads];
   const int bh = blockIdx.x;
   double a = 0.0, b = 0.0;
@@ -218,7 +218,9 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (threadIdx.x == 0) {
     const double n = static_cast<double>(S) * D;
     const float ms = static_cast<float>(red[0][0] / n), mt = static_cast<float>(red[1][0] / n);
-    const bool failed = status != nullptr && (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE));
+    const int bits = status != nullptr ? (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE)) : 0;
+    const bool failed = bits != 0;
+    if (failed && status_out != nullptr && bh == 0) atomicOr(status_out, bits);
     mse[bh * 2 + 0] = failed ? __int_as_float(0x7fc00000) : ms;
     mse[bh * 2 + 1] = failed ? __int_as_float(0x7fc00000) : mt;
     label[bh] = failed ? static_cast<int8_t>(-1) : ((mt < ms) ? SVG_TEMPORAL : SVG_SPATIAL);
@@ -298,9 +300,10 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
     lay.n_chunks = 1;
     lay.chunk = L;
   } else {
-    // One CTA per (chunk, head), one CTA per SM.  Pick the chunk count that
-    // minimises waves x (key tiles per chunk + a fixed per-CTA cost of about
-    // two tiles for setup, Q gather and the partials' store).
+    // A pair of CTAs per (chunk, head) (one per restricted variant), one CTA
+    // per SM.  Pick the chunk count that minimises waves x (key tiles per
+    // chunk + a fixed per-CTA cost of about two tiles for setup, Q gather and
+    // the partials' store).
     const long long heads = static_cast<long long>(B) * H;
     const long long tiles = (L + kKT - 1) / kKT;
     long long limit = tiles;
@@ -323,7 +326,8 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
   lay.o_bytes = (rows_total * d * sizeof(float) + 255) / 256 * 256;
   lay.ml_bytes = (rows_total * 2 * sizeof(float) + 255) / 256 * 256;
   lay.part_bytes = (static_cast<size_t>(B) * H * lay.S_pad * 3 * sizeof(double) + 255) / 256 * 256;
-  lay.total = lay.o_bytes + lay.ml_bytes + lay.part_bytes;
+  lay.status_bytes = 256;
+  lay.total = lay.o_bytes + lay.ml_bytes + lay.part_bytes + lay.status_bytes;
   *out = lay;
   return true;
 }
@@ -369,19 +373,28 @@ svg_status launch_profile_pass(int B, int H, int N, int F, int d, int dtype, flo
   return cuda_check(cudaGetLastError(), "profile combine launch");
 }
 
+static svg_status call_status_word(void* ws, const ProfileLayout& lay, int** out, cudaStream_t stream) {
+  int* w = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + profile_status_offset(lay));
+  cudaError_t e = cudaMemsetAsync(w, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_check(e, "cudaMemsetAsync(profiling status)");
+  *out = w;
+  return SVG_OK;
+}
+
 svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
                           const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
                           float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
-                          cudaStream_t stream) {
+                          int* status_out, cudaStream_t stream) {
   int* status = nullptr;
-  svg_status st = internal_status_word(&status, stream);
+  svg_status st = call_status_word(ws, lay, &status, stream);
   if (st != SVG_OK) return st;
   double* part = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
   const int kind[2] = {kProfFrameBand, kProfPositionBand}, par[2] = {a1, a2};
   if ((st = launch_profile_pass(B, H, N, F, d, dtype, scale, q, k, v, kind, par, rows, S, ws, lay, part, status,
                                 stream)) != SVG_OK)
     return st;
-  profile_finalize_kernel<<<B * H, kCombineThreads, 0, stream>>>(part, S, lay.S_pad, d, mse, label, status);
+  profile_finalize_kernel<<<B * H, kCombineThreads, 0, stream>>>(part, S, lay.S_pad, d, mse, label, status,
+                                                                   status_out);
   return cuda_check(cudaGetLastError(), "profile finalize launch");
 }
 
@@ -390,7 +403,7 @@ svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, co
                               float lambda, float epsilon, float* loss, int8_t* mode, void* ws,
                               const ProfileLayout& lay, double* part2, cudaStream_t stream) {
   int* status = nullptr;
-  svg_status st = internal_status_word(&status, stream);
+  svg_status st = call_status_word(ws, lay, &status, stream);
   if (st != SVG_OK) return st;
   double* part1 = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
   const int kind1[2] = {kProfWindow, kProfPositionBand}, par1[2] = {window, md_half + 1};

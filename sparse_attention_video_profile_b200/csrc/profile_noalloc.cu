@@ -79,7 +79,7 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
     ProfileLayout one;
     profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &one, 1);
     const size_t per_chunk = one.o_bytes + one.ml_bytes;  // bytes that scale with the chunk count
-    const long long fit = static_cast<long long>((kMax - one.part_bytes - 512) / per_chunk);
+    const long long fit = static_cast<long long>((kMax - one.part_bytes - one.status_bytes - 512) / per_chunk);
     if (shape->dtype != SVG_BF16 || one.total > kMax || fit < 1)
       return fail(SVG_ERR_WORKSPACE,
                   "profiling this shape needs at least %zu bytes of scratch, more than the %zu-byte static "
@@ -96,5 +96,5 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
   const int a2c = a2 < shape->F ? a2 : shape->F;
   // the same kernels as svg_profile_heads, on the static scratch
   return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, scale, q, k, v, a1c, a2c,
-                        rows, S, mse, label, scratch, lay, static_cast<cudaStream_t>(stream));
+                        rows, S, mse, label, scratch, lay, nullptr, static_cast<cudaStream_t>(stream));
 }

@@ -308,22 +308,27 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
 // 2^x for a pair of arguments on the FMA pipe, leaving the MUFU unit free.
 // Round-to-nearest range reduction x = j + f with f in [-1/2, 1/2] (adding
 // 1.5 * 2^23 puts round(x) in the low mantissa bits), a cubic for 2^f, and j
-// added straight into the exponent field.  The cubic's coefficients are a
-// minimax fit (Lawson-weighted least squares) of 2^f on [-1/2, 1/2] in relative error:
-// max relative error 8.4e-5, against the 2^-9 half-ulp of the bf16 value the
-// result is rounded to.  Arguments below -125 are clamped, returning 2^-125
-// in place of a smaller (or zero) value.
+// added straight into the exponent field.  The cubic is a minimax fit of 2^f
+// on [-1/2, 1/2] in relative error (a linear program on a dense grid) with
+// its constant term held at exactly 1: max relative error 1.01e-4, against
+// the 2^-9 half-ulp of the bf16 value the result is rounded to.
+// Arguments are clamped at -127.  There f = 0 and the cubic returns exactly
+// 1.0f (bits 127 << 23), so adding -127 to the exponent field gives the bits
+// of +0: a masked key (argument -inf) weighs exactly 0, as with ex2.approx.
+// Arguments in (-127, -126) give subnormal results below 2^-126; no argument
+// drives the exponent field negative (j = -127 only for f >= 0, where the
+// cubic is >= 1).
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99991959799f, c1 = 0.69326216025f, c2 = 0.24271414047f, c3 = 0.05521299318f;
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
+  constexpr float c1 = 0.6932829022f, c2 = 0.2422109544f, c3 = 0.05500892922f;
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
   const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
   const float2 j = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
   const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
   float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
   q = __ffma2_rn(q, f, make_float2(c1, c1));
-  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
   return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }

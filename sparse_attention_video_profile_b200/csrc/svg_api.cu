@@ -208,6 +208,17 @@ size_t svg_workspace_size(const svg_shape* shape, int32_t n_temporal_heads_max) 
 svg_status svg_profile_heads(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
                              size_t workspace_bytes, void* stream) {
+  return profile_heads_impl(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, nullptr,
+                            static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace svg {
+
+svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
+                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
+                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream) {
   svg_status st = check_shape(shape);
   if (st != SVG_OK) return st;
   if ((st = check_tensors({q, k, v})) != SVG_OK) return st;
@@ -223,8 +234,12 @@ svg_status svg_profile_heads(const svg_shape* shape, const void* q, const void* 
     return fail(SVG_ERR_WORKSPACE, "profile workspace %zu bytes < %zu required", workspace_bytes, lay.total);
   return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, eff_scale(shape), q, k, v,
                         clamp_band(a1, 1, shape->N), clamp_band(a2, 1, shape->F), rows, S, mse, label, workspace, lay,
-                        static_cast<cudaStream_t>(stream));
+                        status_out, stream);
 }
+
+}  // namespace svg
+
+extern "C" {
 
 svg_status svg_permute(const svg_shape* shape, const void* x, void* xp, const int8_t* label, void* stream) {
   svg_status st = check_shape(shape);
@@ -378,8 +393,8 @@ svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void*
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if (whole_call_fused(shape, a2)) {
-    if ((st = svg_profile_heads(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, stream)) !=
-        SVG_OK)
+    if ((st = profile_heads_impl(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, status_dev,
+                                 static_cast<cudaStream_t>(stream))) != SVG_OK)
       return st;
     return svg_block_sparse_attn_fused(shape, q, k, v, o, label, a1, a2, status_dev, stream);
   }
@@ -389,12 +404,61 @@ svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void*
   void *qp = w, *kp = w + t_al, *vp = w + 2 * t_al, *op = w + 3 * t_al;
   void* prof_ws = w + 4 * t_al;
   const size_t prof_bytes = workspace_bytes - 4 * t_al;
-  if ((st = svg_profile_heads(shape, q, k, v, a1, a2, rows, S, mse, label, prof_ws, prof_bytes, stream)) != SVG_OK)
+  if ((st = profile_heads_impl(shape, q, k, v, a1, a2, rows, S, mse, label, prof_ws, prof_bytes, status_dev,
+                               static_cast<cudaStream_t>(stream))) != SVG_OK)
     return st;
   if ((st = svg_permute_qkv(shape, q, k, v, qp, kp, vp, label, stream)) != SVG_OK) return st;
   if ((st = svg_block_sparse_attn(shape, q, k, v, qp, kp, vp, o, op, label, a1, a2, status_dev, stream)) != SVG_OK)
     return st;
   return svg_unpermute(shape, op, o, label, stream);
+}
+
+svg_status svg_head_shard(int32_t n_heads, int32_t rank, int32_t world, int32_t* first, int32_t* count) {
+  if (first == nullptr || count == nullptr) return fail(SVG_ERR_INVALID_ARG, "NULL output");
+  if (n_heads < 0 || world < 1 || rank < 0 || rank >= world)
+    return fail(SVG_ERR_INVALID_ARG, "need n_heads >= 0, world >= 1 and 0 <= rank < world (got %d, %d, %d)", n_heads,
+                rank, world);
+  const int32_t base = n_heads / world, extra = n_heads % world;
+  *count = base + (rank < extra ? 1 : 0);
+  *first = rank * base + (rank < extra ? rank : extra);
+  return SVG_OK;
+}
+
+size_t svg_sparse_3d_attn_shard_workspace_size(const svg_shape* shape, int32_t rank, int32_t world, int32_t a2,
+                                               int32_t S) {
+  if (check_shape(shape) != SVG_OK) return 0;
+  int32_t first = 0, count = 0;
+  if (svg_head_shard(shape->B * shape->H, rank, world, &first, &count) != SVG_OK) return 0;
+  if (count == 0) return 256;  // nothing to compute; a token workspace keeps the size query non-zero
+  svg_shape local = *shape;
+  local.B = 1;
+  local.H = count;
+  return svg_sparse_3d_attn_workspace_size(&local, a2, S);
+}
+
+svg_status svg_sparse_3d_attn_shard(const svg_shape* shape, int32_t rank, int32_t world, const void* q, const void* k,
+                                    const void* v, void* o, int32_t a1, int32_t a2, const int32_t* rows, int32_t S,
+                                    float* mse, int8_t* label, void* workspace, size_t workspace_bytes,
+                                    int32_t* status_dev, void* stream) {
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  int32_t first = 0, count = 0;
+  if ((st = svg_head_shard(shape->B * shape->H, rank, world, &first, &count)) != SVG_OK) return st;
+  if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
+  if (!mse || !label) return fail(SVG_ERR_INVALID_ARG, "NULL mse/label");
+  if (count == 0) return SVG_OK;  // more ranks than heads: this rank has none
+  // heads are flattened over (b, h): this rank's heads are one contiguous
+  // block of every [B, H, ...] array, so the shard is the whole call on that
+  // block
+  svg_shape local = *shape;
+  local.B = 1;
+  local.H = count;
+  const size_t head_bytes = static_cast<size_t>(shape->N) * shape->F * shape->d * elem_size(shape->dtype);
+  const size_t off = static_cast<size_t>(first) * head_bytes;
+  auto at = [off](const void* p) { return static_cast<const uint8_t*>(p) + off; };
+  return svg_sparse_3d_attn(&local, at(q), at(k), at(v), static_cast<uint8_t*>(o) + off, a1, a2, rows, S,
+                            mse + 2 * static_cast<size_t>(first), label + first, workspace, workspace_bytes,
+                            status_dev, stream);
 }
 
 svg_status svg_mixed_attn(const svg_shape* shape, const void* q, const void* k, const void* v, const void* qp,

@@ -40,6 +40,7 @@ EXPORTED = (
     "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search", "svg_block_sparse_attn_fused",
     "svg_mixed_attn_fused", "svg_sparse_3d_attn_plan", "svg_semantic_attn_workspace_size", "svg_semantic_attn",
     "svg_kmeans_workspace_size", "svg_kmeans", "svg_semantic_3d_attn_workspace_size", "svg_semantic_3d_attn",
+    "svg_head_shard", "svg_sparse_3d_attn_shard_workspace_size", "svg_sparse_3d_attn_shard",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -103,6 +104,9 @@ def _load() -> ctypes.CDLL:
         "svg_semantic_3d_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _Z, _P, _P]),
         "svg_mode_search": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _Z,
                                  _P]),
+        "svg_head_shard": (_I, [_I, _I, _I, _P, _P]),
+        "svg_sparse_3d_attn_shard_workspace_size": (_Z, [_P, _I, _I, _I, _I]),
+        "svg_sparse_3d_attn_shard": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _Z, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -333,6 +337,62 @@ def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Te
     _check(lib.svg_sparse_3d_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), a1, a2, _ptr(rows), S,
                                   _ptr(mse), _ptr(label), _ptr(workspace), workspace.numel(), _ptr(status),
                                   _stream(stream)))
+    return o, mse, label
+
+
+def svg_head_shard(n_heads: int, rank: int, world: int):
+    """(first, count): rank's contiguous block of the heads numbered over (b, h)."""
+    first, count = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.svg_head_shard(n_heads, rank, world, ctypes.byref(first), ctypes.byref(count)))
+    return int(first.value), int(count.value)
+
+
+def gather_heads(x: torch.Tensor, n_heads: int, rank: int, world: int, group=None) -> torch.Tensor:
+    """Fills every rank's block of heads of x (shape [B, H, ...], this rank's
+    block already written) from the other ranks, in place: one all-gather of
+    blocks padded to the largest block.  Works on any torch.distributed
+    backend (NCCL for device tensors, gloo for host tensors)."""
+    import torch.distributed as dist
+    flat = x.view(n_heads, -1)
+    first, count = svg_head_shard(n_heads, rank, world)
+    width = -(-n_heads // world)
+    buf = torch.zeros(width, flat.shape[1], dtype=x.dtype, device=x.device)
+    buf[:count] = flat[first:first + count]
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf, group=group)
+    for r in range(world):
+        f, c = svg_head_shard(n_heads, r, world)
+        if r != rank and c:
+            flat[f:f + c] = parts[r][:c]
+    return x
+
+
+def svg_sparse_3d_attn_shard(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, rank: int, world: int, *,
+                             o=None, mse=None, label=None, workspace=None, status=None, scale: float = 0.0,
+                             stream=None, gather: bool = False, group=None):
+    """This rank's block of heads of one whole call (q, k, v are the full
+    tensors).  Returns (o, mse, label) full-size; only this rank's heads are
+    written unless gather=True, which then fills the rest from the other
+    ranks (torch.distributed must be initialised)."""
+    _same(q, k, v)
+    shape = make_shape(q, N, F, scale)
+    S = rows.numel()
+    if o is None:
+        o = torch.empty_like(q)
+    if mse is None:
+        mse = torch.empty(shape.B, shape.H, 2, dtype=torch.float32, device=q.device)
+    if label is None:
+        label = torch.empty(shape.B, shape.H, dtype=torch.int8, device=q.device)
+    if workspace is None:
+        need = int(lib.svg_sparse_3d_attn_shard_workspace_size(ctypes.byref(shape), rank, world, a2, S))
+        workspace = alloc_workspace(need, q.device)
+    _check(lib.svg_sparse_3d_attn_shard(ctypes.byref(shape), rank, world, _ptr(q), _ptr(k), _ptr(v), _ptr(o), a1, a2,
+                                        _ptr(rows), S, _ptr(mse), _ptr(label), _ptr(workspace), workspace.numel(),
+                                        _ptr(status), _stream(stream)))
+    if gather and world > 1:
+        n = shape.B * shape.H
+        for t in (o, mse, label):
+            gather_heads(t, n, rank, world, group)
     return o, mse, label
 
 

@@ -270,7 +270,7 @@ def run_reference(args, wl, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "ms/call", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(wl, world),
+        "config": config_dict(wl, world, args.shard),
         "cpu_baseline": {"value": value, "unit": "ms/call", "cores": cpu_cores(), "kind": "oracle",
                          "sample": desc + " (per step)"},
         "e2e": {"value": value, "unit": "ms/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -278,11 +278,12 @@ def run_reference(args, wl, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(wl, world):
+def config_dict(wl, world, shard="replicas"):
     shape_name = "mixed sparse-pattern" if wl.name.startswith("mixed") else "HunyuanVideo-shaped"
     return {"workload": f"{shape_name} {wl.name}: B={wl.B} H={wl.H} N={wl.N} F={wl.F} L={wl.L} d={wl.d}",
             "B": wl.B, "H": wl.H, "N": wl.N, "F": wl.F, "L": wl.L, "d": wl.d, "a1": wl.a1, "a2": wl.a2, "S": wl.S,
-            "global_batch": wl.B * world, "seq_len": wl.L, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "global_batch": wl.B * (world if shard == "replicas" else 1), "seq_len": wl.L,
+            "parallelism": f"{shard}{world}" if world > 1 else "single",
             "l2": f"inputs larger than L2 (Q,K,V 3 x {wl.B * wl.H * wl.L * wl.d * 2 / 1e6:.0f} MB); no flush"}
 
 
@@ -427,13 +428,120 @@ def run_svg2(args, wl, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def time_calls(fn, reps, stream, warm=2):
+    """Mean device time (ms) of `reps` back-to-back calls of fn on `stream`,
+    after `warm` untimed calls (CUDA events on the launching stream)."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def measure_config(wl, dev, stream, peak, seed=0, steps=5, warm=2):
+    """One workload timed outside the headline's timed region: the whole call
+    step by step (profile -> attention with the layout the call picks, or
+    permute -> attention -> unpermute), CUDA events around each stage.
+    Returns ms per call, attention-kernel ms, effective TFLOPS and the
+    fraction of the bf16 peak."""
+    from sparse_attention_video_profile_b200 import svg
+    q, k, v = synth.make_qkv(wl, seed=seed, device=dev)
+    rows = torch.from_numpy(synth.sample_rows(wl.L, wl.S, seed)).to(dev)
+    N, F = wl.N, wl.F
+    shape = svg.make_shape(q, N, F)
+    o = torch.empty_like(q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    mixed = wl.name.startswith("mixed")
+    prm = synth.MIXED_PARAMS
+    band = prm["md_half"] + 1 if mixed else wl.a2
+    fused = svg.svg_sparse_3d_attn_plan(shape, band)[2]
+    if mixed:
+        modes_np = synth.head_modes(wl.B, wl.H, seed)
+        mode = torch.from_numpy(modes_np).to(dev)
+        md_label = torch.from_numpy((modes_np == 3).astype(np.int8)).to(dev)
+    else:
+        mse = torch.empty(wl.B, wl.H, 2, dtype=torch.float32, device=dev)
+        label = torch.empty(wl.B, wl.H, dtype=torch.int8, device=dev)
+        prof_ws = svg.alloc_workspace(svg.svg_profile_workspace_size(shape, wl.S), dev)
+    if not fused:
+        qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
+
+    def step(ev):
+        ev[0].record(stream)
+        if not mixed:
+            svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws)
+        lab = md_label if mixed else label
+        if not fused:
+            svg.svg_permute_qkv(q, k, v, N, F, lab, out=(qp, kp, vp))
+        ev[1].record(stream)
+        if mixed and fused:
+            svg.svg_mixed_attn_fused(q, k, v, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
+                                     status=status)
+        elif mixed:
+            svg.svg_mixed_attn(q, k, v, qp, kp, vp, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
+                               op=op, status=status)
+        elif fused:
+            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status)
+        else:
+            svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status)
+        ev[2].record(stream)
+        if not fused:
+            svg.svg_unpermute(op, N, F, lab, out=o)
+        ev[3].record(stream)
+
+    def events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    for _ in range(warm):
+        step(events())
+    torch.cuda.synchronize()
+    evs = [events() for _ in range(steps)]
+    for ev in evs:
+        step(ev)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status word {int(status.item())} in the {wl.name} config")
+    call_ms = float(np.mean([ev[0].elapsed_time(ev[3]) for ev in evs]))
+    attn_ms = float(np.mean([ev[1].elapsed_time(ev[2]) for ev in evs]))
+    if mixed:
+        pairs = metrics.mixed_pairs(N, F, modes_np, prm["window"], prm["md_half"], prm["stripe"])
+    else:
+        pairs = metrics.effective_pairs(N, F, wl.a1, wl.a2, label.cpu().numpy())
+    tflops = metrics.attention_flops(pairs, wl.d) / (attn_ms * 1e-3) / 1e12
+    return {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={N} F={F} L={wl.L} d={wl.d} a1={wl.a1} a2={wl.a2}",
+            "ms": call_ms, "attn_ms": attn_ms, "effective_tflops": tflops, "frac_bf16_peak": tflops / peak,
+            "density": pairs / (wl.B * wl.H * float(wl.L) * wl.L),
+            "layout": "fused" if fused else "separate", "steps": steps}
+
+
 def run_ours(args, wl, rank, world, local):
     from sparse_attention_video_profile_b200 import svg
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    q, k, v = synth.make_qkv(wl, seed=rank, device=dev)
-    rows_np = synth.sample_rows(wl.L, wl.S, rank)
+    # N > 1: every rank takes its block of the heads of ONE call (the head
+    # partition of svg_head_shard, as svg_sparse_3d_attn_shard runs it: views
+    # of the block, no copies), or with --shard replicas runs its own call
+    shard_heads = world > 1 and args.shard == "heads"
+    job_wl = wl
+    if shard_heads:
+        import dataclasses
+        n_heads = wl.B * wl.H
+        first, count = svg.svg_head_shard(n_heads, rank, world)
+        if count == 0:
+            raise SystemExit(f"--shard heads needs at least one head per rank ({n_heads} heads, {world} ranks)")
+        q, k, v = (t.view(n_heads, wl.L, wl.d)[first:first + count].view(1, count, wl.L, wl.d)
+                   for t in synth.make_qkv(wl, seed=0, device=dev))
+        wl = dataclasses.replace(wl, B=1, H=count)
+        rows_np = synth.sample_rows(wl.L, wl.S, 0)
+    else:
+        q, k, v = synth.make_qkv(wl, seed=rank, device=dev)
+        rows_np = synth.sample_rows(wl.L, wl.S, rank)
     rows = torch.from_numpy(rows_np).to(dev)
     N, F = wl.N, wl.F
     o = torch.empty_like(q)
@@ -550,7 +658,9 @@ def run_ours(args, wl, rank, world, local):
         raise RuntimeError(f"device status word {int(status.item())} after the timed region")
     step_ms = max_over_ranks(step_ms_local, world)
     kern_ms = {n: acc[n] / args.steps for n in acc}
-    value = step_ms / world  # ms per call, whole job (world calls per step): job_ms_per_call
+    # ms per call, whole job: head shards finish one call per step (the
+    # slowest rank's step); replicas finish `world` calls per step
+    value = step_ms if shard_heads else step_ms / world
 
     # dense reference on the same inputs (speedup vs dense), outside the timed region
     dense_ms = None
@@ -623,7 +733,7 @@ def run_ours(args, wl, rank, world, local):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world) / world
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world) / (1 if shard_heads else world)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, rowsh))
         d2h = sum(t.numel() * t.element_size() for t in (oh, mseh, labh))
         e2e = {"value": e2e_ms, "unit": "ms/call", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -631,13 +741,50 @@ def run_ours(args, wl, rank, world, local):
         del qh, kh, vh, oh, ws_host_call
 
     peaks, peak_kind = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     attn_tflops = flops / (kern_ms["attn"] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    # the seconds-long power-capped figure, shown beside the burst one
-    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     perm_bytes = 2 * 3 * n_temporal * wl.B * wl.L * wl.d * 2
     unperm_bytes = 2 * n_temporal * wl.B * wl.L * wl.d * 2
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    # the layout-transformation kernels on this call's labels, timed on their
+    # own after the timed region (when the call fuses the layout they are not
+    # part of it); each moves more than L2 holds, so no flush is needed
+    layout_kernels = None
+    if not mixed and n_temporal and not args.no_configs:
+        if fused:
+            qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
+        t_perm = time_calls(lambda: svg.svg_permute_qkv(q, k, v, N, F, label, out=(qp, kp, vp)), 5, stream)
+        t_unperm = time_calls(lambda: svg.svg_unpermute(op, N, F, label, out=o), 5, stream)
+        layout_kernels = {
+            "permute_ms": t_perm, "permute_gbs": perm_bytes / (t_perm * 1e-3) / 1e9,
+            "permute_frac_hbm": perm_bytes / (t_perm * 1e-3) / 1e9 / hbm,
+            "unpermute_ms": t_unperm, "unpermute_gbs": unperm_bytes / (t_unperm * 1e-3) / 1e9,
+            "unpermute_frac_hbm": unperm_bytes / (t_unperm * 1e-3) / 1e9 / hbm,
+            "bytes": {"permute": perm_bytes, "unpermute": unperm_bytes},
+            "note": "svg_permute_qkv / svg_unpermute on this call's temporal heads, 2 warm + 5 timed calls each"}
+        if fused:
+            qp = kp = vp = op = None
+    prof_bytes = 2 * wl.B * wl.H * wl.L * wl.d * 2  # K and V read once
+    roofline_profile = None
+    if not mixed:
+        prof_gbs = prof_bytes / (kern_ms["profile"] * 1e-3) / 1e9
+        roofline_profile = {"bound": "hbm", "kernel": "svg_profile_heads: profile_sm100_kernel + "
+                            "profile_combine_rows_kernel + profile_finalize_kernel (whole call timed)",
+                            "achieved": prof_gbs, "peak": hbm, "peak_kind": f"{peak_kind} hbm_gbs",
+                            "unit": "GB/s", "frac": prof_gbs / hbm, "traffic": None,
+                            "algorithmic_work": f"{prof_bytes:.4e} bytes/launch = K and V of every head once"}
+    configs = None
+    if not args.no_configs and rank == 0 and world == 1 and wl.name == "hunyuan":
+        configs = []
+        qp = kp = vp = op = None
+        torch.cuda.empty_cache()
+        for cw in (synth.WORKLOADS["cogvideox"], wl.with_bands(*synth.HUNYUAN_SWEEP[0.05], name="hunyuan-5%"),
+                   wl.with_bands(*synth.HUNYUAN_SWEEP[0.5], name="hunyuan-50%"), synth.WORKLOADS["mixed"]):
+            configs.append(measure_config(cw, dev, stream, peak))
+            torch.cuda.empty_cache()
+    # the seconds-long power-capped figure, shown beside the burst one
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not mixed:
@@ -647,8 +794,10 @@ def run_ours(args, wl, rank, world, local):
 
     line = {
         "metric": METRIC, "value": value, "unit": "ms/call", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl, world),
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False,
+        "scaling": "strong" if shard_heads else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(job_wl, world, "heads" if shard_heads else "replicas"),
         "effective_tflops": attn_tflops, "effective_tflops_call": flops / (step_ms * 1e-3) / 1e12,
         "frac_bf16_peak": attn_tflops / peak,
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
@@ -659,8 +808,11 @@ def run_ours(args, wl, rank, world, local):
                    if fused else "separate: permute -> attention -> unpermute"),
         "layout_plan": {"separate_tiles_per_head": plan_sep, "fused_tiles_per_head": plan_fused,
                         "choice": "fused" if plan_choice else "separate", "requested": args.layout},
-        "permute_gbs": perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
-        "unpermute_gbs": unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal and not fused else None,
+        "permute_gbs": (perm_bytes / (kern_ms["permute"] * 1e-3) / 1e9 if n_temporal and not fused else
+                        layout_kernels["permute_gbs"] if layout_kernels else None),
+        "unpermute_gbs": (unperm_bytes / (kern_ms["unpermute"] * 1e-3) / 1e9 if n_temporal and not fused else
+                          layout_kernels["unpermute_gbs"] if layout_kernels else None),
+        "layout_kernels": layout_kernels,
         "temporal_heads": n_temporal,
         "density": pairs / (wl.B * wl.H * float(wl.L) * wl.L),
         "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
@@ -670,7 +822,9 @@ def run_ours(args, wl, rank, world, local):
                          NCU_TRAFFIC.get(attn_source_key() + ("fused" if fused else "separate",))
                          if wl.name == "hunyuan" else None),
                      "algorithmic_work": f"{flops:.4e} flops/launch = 4*d*unmasked pairs"},
+        "roofline_profile": roofline_profile,
         "hbm_peak_gbs": hbm,
+        "configs": configs,
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": len(names) * args.steps + (0 if mixed else (PROFILE_LAUNCHES - 1) * args.steps),
@@ -692,12 +846,18 @@ def main():
     ap.add_argument("--density", type=float, default=None, help="HunyuanVideo sweep density (0.05..0.5)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard", choices=["heads", "replicas"], default="heads",
+                    help="N > 1: split the heads of one call over the ranks (strong scaling), or run one "
+                         "independent call per rank (weak scaling)")
     ap.add_argument("--layout", choices=["auto", "fused", "separate"], default="auto",
                     help="temporal heads' layout transformation fused into attention, or as separate kernels; "
                          "auto = the whole call's own choice")
     ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per chunk of the host-buffer call")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config lines (CogVideoX, the 5 %% / 50 %% sweep ends, mixed) and the "
+                         "stand-alone permute / unpermute timing that follow the timed region")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per attention launch from an ncu capture of this kernel")
     args = ap.parse_args()

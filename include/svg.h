@@ -89,6 +89,8 @@ typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
 #define SVG_DEV_TIMEOUT 0x1u  /* a pipeline wait exceeded its bound; outputs invalid */
 #define SVG_DEV_RANGE 0x2u    /* profiling: in-band weights underflowed (see svg_profile_heads);
                                  semantic attention: a cluster id out of range */
+#define SVG_DEV_BOUNDS 0x4u   /* debug build only: a kernel index outside its buffer (the access was
+                                 skipped; see svg_debug_checks) */
 
 typedef struct svg_shape {
   int32_t B, H, N, F, d;
@@ -105,6 +107,19 @@ SVG_API const char* svg_status_string(int32_t status);
 
 /* Message for the last non-OK status returned on the calling host thread. */
 SVG_API const char* svg_last_error(void);
+
+/*
+ * svg_debug_checks -- 1 if this library was built with range checks
+ * (libsvg_debug.so, compiled with SVG_DEBUG_BOUNDS=1), 0 otherwise.  In the
+ * checked build every global-memory index the tensor-core kernels compute
+ * (output rows, sampled rows, workspace slots, cluster ids and offsets, TMA
+ * tile coordinates) is compared with its buffer first; an index outside it
+ * sets SVG_DEV_BOUNDS in the status word and the store is skipped, so a
+ * wrong index is reported instead of faulting or trapping.  Shared-memory and
+ * tensor-memory offsets are fixed per kernel and checked at compile time.
+ * The checked build is slower and meant for tests.
+ */
+SVG_API int32_t svg_debug_checks(void);
 
 /*
  * svg_attn_tile -- query/key tile sizes (rows) of the attention kernel for a

@@ -6,6 +6,11 @@ Each csrc/*.cu is compiled with nvcc for sm_100a (arch-specific features:
 tcgen05, TMA) into _build/, then linked into
 sparse_attention_video_profile_b200/libsvg.so with the CUDA runtime linked
 statically.  Rebuilds only when a source or header is newer than the library.
+
+    python -m sparse_attention_video_profile_b200.build --debug
+
+builds the range-checked library libsvg_debug.so (-DSVG_DEBUG_BOUNDS=1, see
+svg_debug_checks in include/svg.h) beside it, for tests.
 """
 from __future__ import annotations
 
@@ -23,6 +28,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsvg.so")
+LIB_DEBUG = os.path.join(PKG, "libsvg_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -45,22 +51,25 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    build_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    flags = NVCC_FLAGS + (["-DSVG_DEBUG_BOUNDS=1"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     nv = nvcc()
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-        cmd = [nv, *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+        cmd = [nv, *ARCH, *flags, "-c", src, "-o", obj]
         if ptxas_verbose:
             cmd += ["-Xptxas", "-v"]
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -75,13 +84,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
             if log.strip():
                 print(log)
     objs = [o for o, _ in results]
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nv, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main(argv=None):
@@ -89,8 +98,9 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas", action="store_true", help="print -Xptxas -v register/smem usage")
+    ap.add_argument("--debug", action="store_true", help="build the range-checked libsvg_debug.so")
     a = ap.parse_args(argv)
-    print(build(force=a.force or a.ptxas, verbose=a.verbose, ptxas_verbose=a.ptxas))
+    print(build(force=a.force or a.ptxas, verbose=a.verbose, ptxas_verbose=a.ptxas, debug=a.debug))
 
 
 if __name__ == "__main__":

@@ -146,9 +146,23 @@ struct Cfg {
   // layout with a setmaxnreg register split measured about 4 % slower.)
   static constexpr int THREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
+  // d = 64 leaves TMEM room for P outside S: P_i gets its own 64 columns,
+  // so S_i is free as soon as the softmax has read it and the next S_i is
+  // computed while the softmax works (separate-P pipeline).  At d = 128 the
+  // two O accumulators fill the rest, and P is written over S.
+  static constexpr bool SEP_P = (D == 64);
   static constexpr uint32_t col_s(int i) { return 128u * i; }
-  static constexpr uint32_t col_o(int i) { return 256u + D * i; }
+  static constexpr uint32_t col_p(int i) { return SEP_P ? 256u + 64u * i : 128u * i; }
+  static constexpr uint32_t col_o(int i) { return SEP_P ? 384u + 64u * i : 256u + D * i; }
 };
+// Tensor-memory and shared-memory layouts fit their allocations.
+static_assert(Cfg<64>::col_s(1) + 128 <= Cfg<64>::TMEM_COLS && Cfg<64>::col_p(1) + 64 <= Cfg<64>::TMEM_COLS &&
+                  Cfg<64>::col_o(1) + 64 <= Cfg<64>::TMEM_COLS && Cfg<64>::col_s(1) + 128 <= Cfg<64>::col_p(0) &&
+                  Cfg<64>::col_p(1) + 64 <= Cfg<64>::col_o(0),
+              "d = 64 TMEM layout");
+static_assert(Cfg<128>::col_s(1) + 128 <= Cfg<128>::col_o(0) && Cfg<128>::col_o(1) + 128 <= Cfg<128>::TMEM_COLS,
+              "d = 128 TMEM layout");
+static_assert(Cfg<64>::SMEM_BYTES <= 232448 && Cfg<128>::SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // Pairs (of 8) per softmax row chunk whose exponentials use the FMA-pipe
 // polynomial instead of the MUFU ex2 unit.  A d = 64 tile has half the MMA
@@ -240,7 +254,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   uint64_t* bar_s = bars + 1 + 2 * C::NS;  // [2] S_i ready
   uint64_t* bar_p = bar_s + 2;             // [2][kPChunks] chunk of P_i written (128 arrivals)
   uint64_t* bar_o = bar_p + 2 * kPChunks;  // [2] P_i V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_o + 2);
+  uint64_t* bar_sfree = bar_o + 2;         // [2] separate-P pipeline: S_i read by the softmax (128 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_sfree + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* s2u = reinterpret_cast<uint32_t*>(tmem_slot + 2);  // [32] SVG2: union of kept key clusters
 
@@ -257,6 +272,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       mbar_init(&bar_s[i], 1);
       for (int j = 0; j < kPChunks; ++j) mbar_init(&bar_p[i * kPChunks + j], 128);
       mbar_init(&bar_o[i], 1);
+      mbar_init(&bar_sfree[i], 128);
     }
     fence_barrier_init();
   }
@@ -339,6 +355,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       tma_prefetch_desc(&p.tm_fq[p.glog[gq]]);
       mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
       const int shq = 7 - p.glog[gq];
+      in_range(pq0, p.F, p.status);
+      in_range(p.gfirst[gq] + (1 << p.glog[gq]) - 1, p.N, p.status);
 #pragma unroll
       for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -354,6 +372,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           break;
         }
         const CUtensorMap* tm = (n & 1) ? &p.tm_fv[p.glog[g]] : &p.tm_fk[p.glog[g]];
+        in_range(t << sh, p.F, p.status);  // key tiles start inside the head (checked build: reported)
+        in_range(p.gfirst[g] + (1 << p.glog[g]) - 1, p.N, p.status);
         mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
@@ -385,6 +405,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           break;
         }
         const CUtensorMap* tm = (n & 1) ? &p.tm_v : &p.tm_k;
+        in_range(kr.t, L, p.status);
         mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
@@ -400,6 +421,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       tma_prefetch_desc(tq);
       tma_prefetch_desc(tk);
       tma_prefetch_desc(tv);
+      in_range(q0, L, p.status);
       mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
 #pragma unroll
       for (int i = 0; i < 2; ++i)
@@ -415,6 +437,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         }
         const CUtensorMap* tm = (n & 1) ? tv : tk;
         const int row = (kt0 + (n >> 1)) * C::BK;
+        in_range(row, L, p.status);
         mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
@@ -452,7 +475,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
 #pragma unroll
         for (int u = 0; u < KK; ++u) {
           const int kk = j * KK + u;
-          umma_ts_warp(tmem + C::col_o(i), tmem + C::col_s(i) + kk * 8,
+          umma_ts_warp(tmem + C::col_o(i), tmem + C::col_p(i) + kk * 8,
                        b + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
@@ -463,7 +486,39 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         issue_qk(1, 0);
         umma_commit_warp(&bar_empty[0]);
       }
-      for (int k = 0; ok && k < nk; ++k) {
+      for (int k = 0; ok && C::SEP_P && k < nk; ++k) {
+        // separate-P pipeline: S_i <- K_{k+1} as soon as the softmax has read
+        // S_i (it writes P_i to its own columns), then O_i += P_i V_k once P_i
+        // is written.  The next scores are ready before the softmax needs them.
+        const int nV = 2 * k + 1, nK = 2 * k + 2;
+        const int slotV = nV % C::NS, slotK = nK % C::NS;
+        if (k + 1 < nk) {
+          ok = warp_wait(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+          for (int i = 0; ok && i < 2; ++i) {
+            ok = warp_wait(&bar_sfree[i], k & 1, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(i, slotK);
+          }
+          if (!ok) break;
+          umma_commit_warp(&bar_empty[slotK]);
+        }
+        ok = warp_wait(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
+        for (int i = 0; ok && i < 2; ++i) {
+#pragma unroll
+          for (int j = 0; j < kPChunks; ++j) {
+            ok = warp_wait(&bar_p[i * kPChunks + j], k & 1, p.wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv_chunk(i, slotV, k > 0, j);
+          }
+          if (!ok) break;
+          umma_commit_warp(&bar_o[i]);  // O_i holds P_i V_k and P_i may be overwritten
+        }
+        if (!ok) break;
+        umma_commit_warp(&bar_empty[slotV]);
+      }
+      for (int k = 0; ok && !C::SEP_P && k < nk; ++k) {
         const int nV = 2 * k + 1, nK = 2 * k + 2;
         const int slotV = nV % C::NS, slotK = nK % C::NS;
         const bool has_next = k + 1 < nk;
@@ -519,15 +574,18 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     int s2_kc = 0;
     uint32_t s2_km[4] = {0u, 0u, 0u, 0u};  // keep mask of the next tile, built ahead of its scores
     if (S2) {
-      const int cq = row_ok ? p.s2_cid[static_cast<size_t>(bh) * L + r] : 0;
+      int cq = row_ok ? p.s2_cid[static_cast<size_t>(bh) * L + r] : 0;
+      if (!in_range(cq, p.s2_Cq, p.status)) cq = 0;
       s2_row = p.s2_sel + (static_cast<size_t>(bh) * p.s2_Cq + cq) * p.s2_W;
       if (!idle) s2r = s2_run(s2u, s2_koff, p.s2_Ck, 0);
       if (S2 && row_ok) x_q = p.s2_perm[static_cast<size_t>(bh) * L + r];
+      if (S2 && row_ok && !in_range(x_q, L, p.status)) x_q = 0;
       if (nk > 0) s2_tile_mask(s2r, s2_koff, s2_row, p.s2_Ck, s2_kc, s2_km);
     }
     int kg = 0, ksh = 7 - p.glog[0], kt = kp_lo >> ksh, kt_end = kp_hi >> ksh;  // fused key-tile iterator
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::col_s(i);
+    const uint32_t tP = tmem + lane_bits + C::col_p(i);
     const uint32_t tO = tmem + lane_bits + C::col_o(i);
     const float sl2 = p.sl2;
     float m_used = -INFINITY, l = 0.f;
@@ -544,6 +602,10 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence32(sr[c]);
+      if (C::SEP_P) {  // S_i has been read: the next scores may overwrite it
+        tc_fence_before();
+        mbar_arrive(&bar_sfree[i]);
+      }
       float s[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -598,15 +660,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         resc = true;
       }
       l *= alpha;
-      if (k > 0 && __any_sync(0xffffffffu, resc)) {
-        // O_i holds P_i(k-1) V (its product completed before S_i(k) did);
-        // rescale it before any P_i(k) V product is issued.
-        if (!warp_wait(&bar_o[i], (k - 1) & 1, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // 16 columns at a time: the 128 scores stay live in registers here
+      // O_i rescale (separate-P pipeline: just before P_i is overwritten, below)
+      auto rescale_o = [&]() {
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           uint32_t ov[16];
@@ -617,6 +672,18 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
           tmem_st16(tO + c * 16, ov);
         }
+      };
+      const bool any_resc = k > 0 && __any_sync(0xffffffffu, resc);
+      if (!C::SEP_P && any_resc) {
+        // O_i holds P_i(k-1) V (its product completed before S_i(k) did);
+        // rescale it before any P_i(k) V product is issued.
+        if (!warp_wait(&bar_o[i], (k - 1) & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // 16 columns at a time: the 128 scores stay live in registers here
+        rescale_o();
       }
       const float nb = (m_used == -INFINITY) ? 0.f : -m_used * sl2;
       const float2 sl2x2 = make_float2(sl2, sl2), nb2 = make_float2(nb, nb);
@@ -643,13 +710,25 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           else add_bf16x2_f32(acc0, pp);
           pk[cc] = pp;
         }
+        if (C::SEP_P && j == 0 && k > 0) {
+          // P_i(k-1) V done: P_i may be overwritten and O_i holds it (the
+          // products of tile k-2 finished before S_i(k) was computed, those
+          // of tile k wait for this P, so the parity identifies the phase)
+          if (!warp_wait(&bar_o[i], (k - 1) & 1, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (any_resc) rescale_o();
+        }
         __syncwarp();
 #pragma unroll
-        for (int h = 0; h < PPC / 16; ++h) tmem_st16(tS + j * PPC + h * 16, pk + h * 16);
+        for (int h = 0; h < PPC / 16; ++h) tmem_st16(tP + j * PPC + h * 16, pk + h * 16);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar_p[i * kPChunks + j]);
       }
+      if (!ok) break;
       l += (acc0.x + acc1.x) + (acc0.y + acc1.y);
       if (S2 && k + 1 < nk) {
         // the next tile's keep mask, while the tensor cores compute its scores
@@ -661,7 +740,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       // no query rows here
     } else if (nk == 0) {
       // skipped head: its output rows are zero
-      if (row_ok) {
+      if (row_ok && in_range(x_q, L, p.status) && in_range(bh, p.BH, p.status)) {
         uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * L + x_q) * D);
 #pragma unroll
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
@@ -671,7 +750,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       // output row: token-major heads write to op, or, fused, straight to
       // the frame-major position of their row in o
-      const int orow = row_ok ? x_q : 0;
+      const bool store_ok = row_ok && in_range(x_q, L, p.status) && in_range(bh, p.BH, p.status);
+      const int orow = store_ok ? x_q : 0;
       __nv_bfloat16* out = (lab && !p.fused && !S2 ? p.op : p.o) + (static_cast<size_t>(bh) * L + orow) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -684,7 +764,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
-        if (row_ok) {
+        if (store_ok) {
           uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);

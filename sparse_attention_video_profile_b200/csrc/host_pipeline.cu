@@ -70,14 +70,22 @@ struct SlotLayout {
   int ntensors;
 };
 
+// Keys per profiling chunk of the whole call (all B*H heads): every chunk of
+// heads splits its keys the same way, so its MSEs round exactly as the device
+// call's.
+int full_call_chunk(const svg_shape* s, int S) {
+  ProfileLayout full;
+  if (!profile_layout(s->B, s->H, s->N * s->F, s->d, s->dtype, S, &full)) return 0;
+  return full.chunk;
+}
+
 SlotLayout slot_layout(const svg_shape* s, int S, int hc, bool fused) {
   SlotLayout l{};
   const size_t es = s->dtype == SVG_FP32 ? 4 : 2;
   l.tensor = align256(static_cast<size_t>(hc) * s->N * s->F * s->d * es);
-  svg_shape cs = *s;
-  cs.B = 1;
-  cs.H = hc;
-  l.prof = align256(svg_profile_workspace_size(&cs, S));
+  ProfileLayout pl;
+  if (!profile_layout(1, hc, s->N * s->F, s->d, s->dtype, S, &pl, 0, full_call_chunk(s, S))) pl.total = 0;
+  l.prof = align256(pl.total);
   l.mse = align256(static_cast<size_t>(hc) * 2 * sizeof(float));
   l.label = align256(static_cast<size_t>(hc));
   l.rows = align256(static_cast<size_t>(S) * sizeof(int32_t));
@@ -167,7 +175,8 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
     svg_shape cs = *shape;
     cs.B = 1;
     cs.H = nh;
-    if ((st = profile_heads_impl(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, status_dev, sc)) != SVG_OK)
+    if ((st = profile_heads_impl(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, status_dev, sc,
+                                 full_call_chunk(shape, S))) != SVG_OK)
       return st;
     if (fused) {
       if ((st = svg_block_sparse_attn_fused(&cs, q, k, v, o, lab, a1, a2, status_dev, stream)) != SVG_OK) return st;

@@ -8,6 +8,11 @@
 
 #include "svg.h"
 
+// Range checks of the debug build (libsvg_debug.so, -DSVG_DEBUG_BOUNDS=1).
+#ifndef SVG_DEBUG_BOUNDS
+#define SVG_DEBUG_BOUNDS 0
+#endif
+
 namespace svg {
 
 // Upper bound on any single pipeline wait inside a kernel.  Waits in a
@@ -122,8 +127,12 @@ struct ProfileLayout {
 inline size_t profile_status_offset(const ProfileLayout& lay) { return lay.o_bytes + lay.ml_bytes + lay.part_bytes; }
 
 // Workspace layout of the profiling kernels.  max_chunks > 0 caps the number
-// of key chunks (fewer chunks need less workspace); fp32 always uses one.
-bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks = 0);
+// of key chunks (fewer chunks need less workspace); chunk_len > 0 (bf16)
+// fixes the keys per chunk instead of choosing them for the head count, so a
+// call on a subset of heads splits the keys, and rounds, exactly as a call on
+// all of them; fp32 always uses one chunk.
+bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks = 0,
+                    int chunk_len = 0);
 
 // Online profiling.  Device-side failures (a wait that ran out, in-band
 // weights that underflowed) are recorded in the status word inside `ws`
@@ -167,8 +176,9 @@ svg_status internal_status_word(int** out, cudaStream_t stream);
 
 // svg_profile_heads with the failure bits also OR-ed into status_out (may be
 // NULL); the whole calls use it to carry a profiling failure to the caller.
+// chunk_len > 0 fixes the profiling key split (see profile_layout).
 svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
                               int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
-                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream);
+                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream, int chunk_len = 0);
 
 }  // namespace svg

@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
         break;
       }
       const int row = (t_begin + i) * 128 + warp * 32 + lane;
-      if (row < p.L) p.assign[static_cast<size_t>(bh) * p.L + row] = bi;
+      // checked build: the chosen centroid is one of the C real ones
+      if (row < p.L && in_range(bi, p.C, p.status)) p.assign[static_cast<size_t>(bh) * p.L + row] = bi;
     }
   }
   tc_fence_before();

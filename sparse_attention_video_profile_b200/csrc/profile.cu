@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (threadIdx.x == 0) {
     const double n = static_cast<double>(S) * D;
     const float ms = static_cast<float>(red[0][0] / n), mt = static_cast<float>(red[1][0] / n);
-    const int bits = status != nullptr ? (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE)) : 0;
+    const int bits = status != nullptr ? (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE | SVG_DEV_BOUNDS)) : 0;
     const bool failed = bits != 0;
     if (failed && status_out != nullptr && bh == 0) atomicOr(status_out, bits);
     mse[bh * 2 + 0] = failed ? __int_as_float(0x7fc00000) : ms;
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     const double n = static_cast<double>(S) * D;
     const float sp[4] = {sparsity.x, sparsity.y, sparsity.z, sparsity.w};  // skip, diagonal, multi-diag, stripe
     const int modes[4] = {SVG_MODE_SKIP, SVG_MODE_DIAGONAL, SVG_MODE_MULTIDIAG, SVG_MODE_STRIPE};
-    const bool failed = status != nullptr && (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE));
+    const bool failed = status != nullptr && (*status & (SVG_DEV_TIMEOUT | SVG_DEV_RANGE | SVG_DEV_BOUNDS));
     int best = -1;
     float best_l = 0.f;
     for (int q = 0; q < 4; ++q) {
@@ -291,19 +291,23 @@ int row_block(int /*d*/, int dtype) { return dtype == SVG_FP32 ? 4 : 128; }
 
 }  // namespace
 
-bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks) {
-  if (B < 1 || H < 1 || L < 1 || S < 1 || S > 128 || max_chunks < 0) return false;
+bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks, int chunk_len) {
+  if (B < 1 || H < 1 || L < 1 || S < 1 || S > 128 || max_chunks < 0 || chunk_len < 0) return false;
   const int rb = row_block(d, dtype);
   ProfileLayout lay{};
   lay.S_pad = (S + rb - 1) / rb * rb;
   if (dtype == SVG_FP32) {
     lay.n_chunks = 1;
     lay.chunk = L;
+  } else if (chunk_len > 0) {
+    long long chunk = (static_cast<long long>(chunk_len) + kKT - 1) / kKT * kKT;
+    if (chunk > L) chunk = (L + kKT - 1) / kKT * kKT;
+    lay.chunk = static_cast<int>(chunk);
+    lay.n_chunks = static_cast<int>((L + chunk - 1) / chunk);
   } else {
-    // A pair of CTAs per (chunk, head) (one per restricted variant), one CTA
-    // per SM.  Pick the chunk count that minimises waves x (key tiles per
-    // chunk + a fixed per-CTA cost of about two tiles for setup, Q gather and
-    // the partials' store).
+    // One CTA per (chunk, head), one CTA per SM.  Pick the chunk count that
+    // minimises waves x (key tiles per chunk + a fixed per-CTA cost of about
+    // two tiles for setup, Q gather and the partials' store).
     const long long heads = static_cast<long long>(B) * H;
     const long long tiles = (L + kKT - 1) / kKT;
     long long limit = tiles;

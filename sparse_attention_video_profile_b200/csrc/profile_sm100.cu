@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
         break;
       }
       const CUtensorMap* tm = (n & 1) ? &p.tm_v : &p.tm_k;
+      in_range((kt0 + (n >> 1)) * 128, p.L, p.status);
       mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
       for (int h = 0; h < C::HALVES; ++h)
@@ -289,6 +290,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     // scale their weights by the same reference.
     const int q = warp & 3, h = warp >> 2;
     const int r = q * 32 + lane;  // row of the tile = sampled-row index (padded)
+    in_range(p.rows[min(r, p.S - 1)], p.L, p.status);  // checked build: a sampled row outside [0, L) is reported
     const int x = min(max(p.rows[min(r, p.S - 1)], 0), p.L - 1);
     if (h == 0) {
       // gather Q row x into the 128-byte-swizzled K-major tile layout
@@ -500,7 +502,11 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
 #pragma unroll
       for (int v = 0; v < 3; ++v) {
         const size_t base = ((static_cast<size_t>(bh) * p.nch + chunk) * 3 + v) * 128 + r;
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + base * D + h * (D / 2));
+        // checked build: a slot outside the workspace is reported and its stores
+        // skipped (the tensor-memory loads below are warp-collective and stay)
+        const bool store_ok =
+            in_range(static_cast<long long>(base), static_cast<long long>(p.BH) * p.nch * 3 * 128, p.status);
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (store_ok ? base : 0) * D + h * (D / 2));
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t ov[32];
@@ -510,10 +516,11 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
           reg_fence32(ov);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            dst[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
-                                         __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+            if (store_ok)
+              dst[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                           __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
         }
-        if (h == 0) {
+        if (h == 0 && store_ok) {
           const float lv = (v == 0) ? l_d : (v == 1 ? l_s : l_t);
           const int nin = (v == 0) ? 1 : (v == 1 ? inband_s : inband_t);
           // max in log2 units; a variant with no kept key in this chunk has none

@@ -7,7 +7,32 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "svg.h"
+
+// Range checks of the debug build (libsvg_debug.so, -DSVG_DEBUG_BOUNDS=1).
+#ifndef SVG_DEBUG_BOUNDS
+#define SVG_DEBUG_BOUNDS 0
+#endif
+
 namespace svg {
+
+// True if 0 <= i < n.  In the debug build an index outside [0, n) sets
+// SVG_DEV_BOUNDS in *status and returns false, so the caller skips the
+// access (or, for a TMA load the pipeline must issue, only reports it); in
+// the normal build it is always true and compiles to nothing.
+__device__ __forceinline__ bool in_range(long long i, long long n, int* status) {
+#if SVG_DEBUG_BOUNDS
+  if (i < 0 || i >= n) {
+    atomicOr(status, static_cast<int>(SVG_DEV_BOUNDS));
+    return false;
+  }
+#else
+  (void)i;
+  (void)n;
+  (void)status;
+#endif
+  return true;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -123,6 +123,8 @@ extern "C" {
 
 int32_t svg_abi_version(void) { return SVG_ABI_VERSION; }
 
+int32_t svg_debug_checks(void) { return SVG_DEBUG_BOUNDS ? 1 : 0; }
+
 const char* svg_status_string(int32_t st) {
   switch (st) {
     case SVG_OK: return "SVG_OK";
@@ -218,7 +220,7 @@ namespace svg {
 
 svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
                               int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
-                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream) {
+                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream, int chunk_len) {
   svg_status st = check_shape(shape);
   if (st != SVG_OK) return st;
   if ((st = check_tensors({q, k, v})) != SVG_OK) return st;
@@ -229,7 +231,7 @@ svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void*
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   ProfileLayout lay;
-  profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay);
+  profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay, 0, chunk_len);
   if (workspace_bytes < lay.total)
     return fail(SVG_ERR_WORKSPACE, "profile workspace %zu bytes < %zu required", workspace_bytes, lay.total);
   return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, eff_scale(shape), q, k, v,

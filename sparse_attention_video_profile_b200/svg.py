@@ -20,7 +20,9 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsvg.so")
+# SVG_LIB names another build of the same library (the range-checked
+# libsvg_debug.so in the tests); the default is the in-tree libsvg.so.
+LIB_PATH = os.environ.get("SVG_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsvg.so")
 
 SVG_OK = 0
 SVG_BF16 = 0
@@ -29,6 +31,7 @@ SPATIAL = 0
 TEMPORAL = 1
 SVG_DEV_TIMEOUT = 0x1
 SVG_DEV_RANGE = 0x2
+SVG_DEV_BOUNDS = 0x4
 
 # Every symbol include/svg.h declares.
 EXPORTED = (
@@ -40,7 +43,7 @@ EXPORTED = (
     "svg_sparse_3d_attn_host", "svg_mode_search_workspace_size", "svg_mode_search", "svg_block_sparse_attn_fused",
     "svg_mixed_attn_fused", "svg_sparse_3d_attn_plan", "svg_semantic_attn_workspace_size", "svg_semantic_attn",
     "svg_kmeans_workspace_size", "svg_kmeans", "svg_semantic_3d_attn_workspace_size", "svg_semantic_3d_attn",
-    "svg_head_shard", "svg_sparse_3d_attn_shard_workspace_size", "svg_sparse_3d_attn_shard",
+    "svg_head_shard", "svg_sparse_3d_attn_shard_workspace_size", "svg_sparse_3d_attn_shard", "svg_debug_checks",
 )
 
 MODE_FULL, MODE_SKIP, MODE_DIAGONAL, MODE_MULTIDIAG, MODE_STRIPE = 0, 1, 2, 3, 4
@@ -70,6 +73,7 @@ def _load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     sig = {
         "svg_abi_version": (_I, []),
+        "svg_debug_checks": (_I, []),
         "svg_status_string": (ctypes.c_char_p, [_I]),
         "svg_last_error": (ctypes.c_char_p, []),
         "svg_attn_tile": (_I, [_I, _I, _P, _P]),

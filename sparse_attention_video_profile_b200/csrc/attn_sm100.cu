@@ -139,8 +139,19 @@ struct Cfg {
   static constexpr int HALF_BYTES = 128 * 128;  // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = BK * D * 2;
   static constexpr int NS = (D == 128) ? 5 : 8;  // K/V ring slots (fills shared memory)
+  // d = 64: the row sums come from the tensor cores.  The P V product runs
+  // with N = d + 16, its B operand V extended by a 16-column block of ones,
+  // so O_i's last 16 columns accumulate sum_y P_i[x, y], the very bf16 weights
+  // the product sees, in fp32.  TMEM: 2 x 128 S + 2 x 80 O columns; P is
+  // written over S.
+#ifndef SVG_ROWSUM_MMA
+#define SVG_ROWSUM_MMA 1
+#endif
+  static constexpr bool ROWSUM_MMA = (D == 64) && SVG_ROWSUM_MMA;
+  static constexpr int ON = D + (ROWSUM_MMA ? 16 : 0);  // O columns (+ the row-sum block)
   static constexpr int SMEM_Q = 2 * TILE_BYTES;
-  static constexpr int SMEM_BAR = SMEM_Q + NS * TILE_BYTES;
+  static constexpr int SMEM_ONES = SMEM_Q + NS * TILE_BYTES;  // 128 rows x 64 bf16 ones (row-sum operand)
+  static constexpr int SMEM_BAR = SMEM_ONES + (ROWSUM_MMA ? HALF_BYTES : 0);
   static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;  // barriers + alignment slack
   // 10 warps: softmax 0-3 and 4-7, TMA producer 8, MMA issuer 9.  (A 12-warp
   // layout with a setmaxnreg register split measured about 4 % slower.)
@@ -150,15 +161,18 @@ struct Cfg {
   // so S_i is free as soon as the softmax has read it and the next S_i is
   // computed while the softmax works (separate-P pipeline).  At d = 128 the
   // two O accumulators fill the rest, and P is written over S.
-  static constexpr bool SEP_P = (D == 64);
+  static constexpr bool SEP_P = (D == 64) && !ROWSUM_MMA;
   static constexpr uint32_t col_s(int i) { return 128u * i; }
   static constexpr uint32_t col_p(int i) { return SEP_P ? 256u + 64u * i : 128u * i; }
-  static constexpr uint32_t col_o(int i) { return SEP_P ? 384u + 64u * i : 256u + D * i; }
+  // O_i starts on a 32-column boundary (the epilogue loads 32 columns at a time)
+  static constexpr uint32_t col_o(int i) { return SEP_P ? 384u + 64u * i : 256u + ((ON + 31) / 32 * 32) * i; }
 };
 // Tensor-memory and shared-memory layouts fit their allocations.
 static_assert(Cfg<64>::col_s(1) + 128 <= Cfg<64>::TMEM_COLS && Cfg<64>::col_p(1) + 64 <= Cfg<64>::TMEM_COLS &&
-                  Cfg<64>::col_o(1) + 64 <= Cfg<64>::TMEM_COLS && Cfg<64>::col_s(1) + 128 <= Cfg<64>::col_p(0) &&
-                  Cfg<64>::col_p(1) + 64 <= Cfg<64>::col_o(0),
+                  Cfg<64>::col_o(1) + Cfg<64>::ON <= Cfg<64>::TMEM_COLS &&
+                  (!Cfg<64>::SEP_P || (Cfg<64>::col_s(1) + 128 <= Cfg<64>::col_p(0) &&
+                                       Cfg<64>::col_p(1) + 64 <= Cfg<64>::col_o(0))) &&
+                  Cfg<64>::col_s(1) + 128 <= Cfg<64>::col_o(0),
               "d = 64 TMEM layout");
 static_assert(Cfg<128>::col_s(1) + 128 <= Cfg<128>::col_o(0) && Cfg<128>::col_o(1) + 128 <= Cfg<128>::TMEM_COLS,
               "d = 128 TMEM layout");
@@ -279,6 +293,14 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
   if (warp == 9) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  if (C::ROWSUM_MMA) {
+    // the ones block of the row-sum product (bf16 1.0 = 0x3F80), made visible
+    // to the tensor cores' (async-proxy) reads
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::SMEM_ONES);
+    for (int e = threadIdx.x; e < C::HALF_BYTES / 16; e += C::THREADS)
+      ones[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (S2 && threadIdx.x < p.s2_W) {
     // union of the key clusters kept by the query clusters of this CTA's rows
@@ -451,7 +473,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       // operands stay warp-uniform, which keeps the per-MMA issue cost low
       // while the softmax warps on the same sub-partition keep it busy.
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::ON, 0, 1);
       const uint32_t ring_base = smem_u32(sRing);
       // Descriptors are built once; offsets go into the start-address field
       // (address >> 4 in the low bits; every operand lies below 256 KB).
@@ -469,8 +491,13 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         umma_commit_warp(&bar_s[i]);
       };
       // The P V products of one chunk of P_i (keys [j, j+1) * BK / kPChunks).
+      const uint32_t ones_addr = smem_u32(smem + C::SMEM_ONES);
       auto issue_pv_chunk = [&](int i, int slot, bool acc, int j) {
-        const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
+        // row-sum form: the ones block is V's second 64-column block, one
+        // leading-dimension offset past the slot (a per-slot offset)
+        const uint32_t vslot = ring_base + slot * C::TILE_BYTES;
+        const uint64_t b = C::ROWSUM_MMA ? smem_desc_sw128(vslot, ones_addr - vslot, 1024)
+                                         : dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
         constexpr int KK = C::BK / 16 / kPChunks;
 #pragma unroll
         for (int u = 0; u < KK; ++u) {
@@ -663,7 +690,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       // O_i rescale (separate-P pipeline: just before P_i is overwritten, below)
       auto rescale_o = [&]() {
 #pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; c < C::ON / 16; ++c) {  // with the row-sum columns, if any
           uint32_t ov[16];
           tmem_ld16(tO + c * 16, ov);
           tmem_wait_ld();
@@ -705,9 +732,12 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
           }
           const uint32_t pp = pack_bf16x2(pr.x, pr.y);
           // The row sum uses the same bf16-rounded weights the P V product
-          // sees, so each output row is an exact convex combination of V rows.
-          if (c & 1) add_bf16x2_f32(acc1, pp);
-          else add_bf16x2_f32(acc0, pp);
+          // sees, so each output row is an exact convex combination of V rows
+          // (with ROWSUM_MMA the tensor cores add them up in O's last columns).
+          if (!C::ROWSUM_MMA) {
+            if (c & 1) add_bf16x2_f32(acc1, pp);
+            else add_bf16x2_f32(acc0, pp);
+          }
           pk[cc] = pp;
         }
         if (C::SEP_P && j == 0 && k > 0) {
@@ -747,6 +777,14 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       }
     } else if (ok && warp_wait(&bar_o[i], (nk - 1) & 1, p.wait_ns)) {
       tc_fence_after();
+      if (C::ROWSUM_MMA) {  // the row sum is column D of O_i
+        uint32_t lv[16];
+        __syncwarp();
+        tmem_ld16(tO + D, lv);
+        tmem_wait_ld();
+        reg_fence16(lv);
+        l = __uint_as_float(lv[0]);
+      }
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       // output row: token-major heads write to op, or, fused, straight to
       // the frame-major position of their row in o

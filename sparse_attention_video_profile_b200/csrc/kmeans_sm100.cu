@@ -12,6 +12,9 @@
 //           memory for the whole CTA, row tiles stream through a 2-slot TMA
 //           ring, and the score accumulator alternates between two 256-column
 //           TMEM slots so the epilogue of one overlaps the MMAs of the next.
+//           The argmin runs on eight warps, two threads per row, each
+//           scanning half of every slot's columns; the halves compare their
+//           results once per row tile through shared memory.
 //   update  each centroid to the mean of its rows: the counting sort by
 //           cluster (svg2_sort), then eight warps per cluster summing its
 //           rows in fp32 in a fixed order (deterministic); an empty cluster
@@ -27,7 +30,7 @@ svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L,
 
 namespace {
 
-constexpr int kKmThreads = 192;  // warps 0-3 epilogue (one row each lane), 4 TMA, 5 MMA
+constexpr int kKmThreads = 320;  // warps 0-7 epilogue (two threads per row), 8 TMA, 9 MMA
 constexpr int kKmSlotCols = 256;
 
 struct KmParams {
@@ -61,13 +64,16 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
   uint8_t* sC = smem;                                                       // centroids, C_pad rows per 64-col half
   uint8_t* sX = smem + static_cast<size_t>(p.C_pad) * 128 * K::HALVES;      // 2 row tiles
   float* sNorm = reinterpret_cast<float*>(sX + 2 * K::TILE_BYTES);           // [C_pad]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sNorm + p.C_pad);
+  float* xbest = sNorm + p.C_pad;                                           // [2 parity][128 rows] second half's minimum
+  int* xbi = reinterpret_cast<int*>(xbest + 256);                           // [2][128] and its column
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xbi + 256);
   uint64_t* bar_c = bars;              // centroids loaded
   uint64_t* bar_xfull = bars + 1;      // [2]
   uint64_t* bar_xempty = bars + 3;     // [2]
   uint64_t* bar_s = bars + 5;          // [2] scores of a TMEM slot ready
-  uint64_t* bar_free = bars + 7;       // [2] epilogue done with a TMEM slot (128 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* bar_free = bars + 7;       // [2] epilogue done with a TMEM slot (256 arrivals)
+  uint64_t* bar_x = bars + 9;          // [4] the two halves of 32 rows compared (64 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int t_begin = blockIdx.x * p.tiles_per_cta;
@@ -80,14 +86,15 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
       mbar_init(&bar_xfull[i], 1);
       mbar_init(&bar_xempty[i], 1);
       mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_free[i], 128);
+      mbar_init(&bar_free[i], 256);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&bar_x[q], 64);
     fence_barrier_init();
   }
   // padding centroids score +inf, so they never win the argmin
   for (int c = threadIdx.x; c < p.C_pad; c += kKmThreads)
     sNorm[c] = c < p.C ? p.norm[static_cast<size_t>(bh) * p.C + c] : INFINITY;
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 2 * p.slot_cols);
     tmem_relinquish();
   }
@@ -96,7 +103,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (nt > 0 && warp == 4 && lane == 0) {
+  if (nt > 0 && warp == 8 && lane == 0) {
     // ---------------------------------------------- TMA producer
     tma_prefetch_desc(&p.tm_c);
     tma_prefetch_desc(&p.tm_x);
@@ -117,7 +124,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
       for (int h = 0; h < K::HALVES; ++h)
         tma_load_3d(sX + s * K::TILE_BYTES + h * K::HALF_BYTES, &p.tm_x, &bar_xfull[s], h * 64, (t_begin + i) * 128, bh);
     }
-  } else if (nt > 0 && warp == 5) {
+  } else if (nt > 0 && warp == 9) {
     // ---------------------------------------------- MMA issuer (whole warp, elected lane issues)
     const uint64_t dc = smem_desc_sw128(smem_u32(sC), 16, 1024);
     const uint64_t dx = smem_desc_sw128(smem_u32(sX), 16, 1024);
@@ -149,9 +156,13 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
       umma_commit_warp(&bar_xempty[xs]);  // the row tile is free once its MMAs are done
     }
     if (!ok && lane == 0) atomicOr(p.status, SVG_DEV_TIMEOUT);
-  } else if (nt > 0 && warp < 4) {
+  } else if (nt > 0 && warp < 8) {
     // ---------------------------------------------- epilogue: argmin per row
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    // warps q and q + 4 share rows 32 q .. 32 q + 31: half hh scans columns
+    // [hh w/2, (hh + 1) w/2) of every slot of width w
+    const int q = warp & 3, hh = warp >> 2;
+    const int r = q * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(q * 32) << 16;
     for (int i = 0; i < nt; ++i) {
       float best = INFINITY;
       int bi = 0;
@@ -164,13 +175,14 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
         }
         tc_fence_after();
         const int width = min(kKmSlotCols, p.C_pad - j * kKmSlotCols);
+        const int c_begin = hh * (width / 2), c_end = c_begin + width / 2;  // multiples of 64
         const uint32_t ts = tmem + lane_bits + s * p.slot_cols;
         // 32 columns at a time, the next load in flight while this one is reduced
         uint32_t v[2][32];
-        tmem_ld32(ts, v[0]);
+        tmem_ld32(ts + c_begin, v[0]);
         tmem_wait_ld();
         reg_fence32(v[0]);
-        for (int c0 = 0; c0 < width; c0 += 64) {
+        for (int c0 = c_begin; c0 < c_end; c0 += 64) {
           tmem_ld32(ts + c0 + 32, v[1]);  // width is a multiple of 128
           const float* nrm = sNorm + j * kKmSlotCols + c0;
 #pragma unroll
@@ -183,7 +195,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
           }
           tmem_wait_ld();
           reg_fence32(v[1]);
-          if (c0 + 64 < width) tmem_ld32(ts + c0 + 64, v[0]);
+          if (c0 + 64 < c_end) tmem_ld32(ts + c0 + 64, v[0]);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float score = fmaf(-2.f, __uint_as_float(v[1][e]), nrm[32 + e]);
@@ -192,7 +204,7 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
               bi = j * kKmSlotCols + c0 + 32 + e;
             }
           }
-          if (c0 + 64 < width) {
+          if (c0 + 64 < c_end) {
             tmem_wait_ld();
             reg_fence32(v[0]);
           }
@@ -200,18 +212,36 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
         tc_fence_before();
         mbar_arrive(&bar_free[s]);
       }
+      if (ok) {
+        // the second half hands its minimum to the first; ties go to the
+        // lower column, wherever it was found
+        if (hh == 1) {
+          xbest[(i & 1) * 128 + r] = best;
+          xbi[(i & 1) * 128 + r] = bi;
+        }
+        mbar_arrive(&bar_x[q]);
+        ok = km_warp_wait(&bar_x[q], i & 1, p.wait_ns);
+      }
       if (!ok) {
         if (lane == 0) atomicOr(p.status, SVG_DEV_TIMEOUT);
         break;
       }
-      const int row = (t_begin + i) * 128 + warp * 32 + lane;
-      // checked build: the chosen centroid is one of the C real ones
-      if (row < p.L && in_range(bi, p.C, p.status)) p.assign[static_cast<size_t>(bh) * p.L + row] = bi;
+      if (hh == 0) {
+        const float b1 = xbest[(i & 1) * 128 + r];
+        const int i1 = xbi[(i & 1) * 128 + r];
+        if (b1 < best || (b1 == best && i1 < bi)) {
+          best = b1;
+          bi = i1;
+        }
+        const int row = (t_begin + i) * 128 + r;
+        // checked build: the chosen centroid is one of the C real ones
+        if (row < p.L && in_range(bi, p.C, p.status)) p.assign[static_cast<size_t>(bh) * p.L + row] = bi;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 2 * p.slot_cols);
@@ -344,7 +374,7 @@ svg_status launch_assign(const void* x, const __nv_bfloat16* mu_b, const float* 
   p.status = status;
   p.wait_ns = 1000000000ull;
   const size_t smem = 1024 + static_cast<size_t>(p.C_pad) * 128 * K::HALVES + 2 * K::TILE_BYTES +
-                      static_cast<size_t>(p.C_pad) * 4 + 128;
+                      static_cast<size_t>(p.C_pad) * 4 + 2048 + 128;
   if (smem > 227 * 1024) return fail(SVG_ERR_UNSUPPORTED, "k-means with C = %d does not fit shared memory", C);
   cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

@@ -38,7 +38,19 @@ METRIC = "ms per sparse 3D-attention call; effective TFLOPS vs bf16 peak; speedu
 # the sha256 prefix of the kernel sources it was taken on and by the layout
 # (fused or separate).  Any other revision or layout reports traffic as null
 # until it is captured again.
-NCU_TRAFFIC = {("645b18066bbc1e1a", "d2f4abb45748fc0c", "fused"): 2.8525e9}
+NCU_TRAFFIC = {("645b18066bbc1e1a", "d2f4abb45748fc0c", "fused"): 2.8525e9,
+               ("20c87c577a0d9af9", "5edc1f6588b2c178", "fused"): 2.8583e9}
+
+
+# The same for the profiling stage-1 kernel (full HunyuanVideo launch), keyed by
+# the sha256 prefix of its source.
+PROF_NCU_TRAFFIC = {"5732be8477404d60": 1.488e9}
+
+
+def prof_source_key():
+    import hashlib
+    path = os.path.join(ROOT, "sparse_attention_video_profile_b200", "csrc", "profile_sm100.cu")
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
 
 def attn_source_key():
@@ -772,7 +784,8 @@ def run_ours(args, wl, rank, world, local):
         roofline_profile = {"bound": "hbm", "kernel": "svg_profile_heads: profile_sm100_kernel + "
                             "profile_combine_rows_kernel + profile_finalize_kernel (whole call timed)",
                             "achieved": prof_gbs, "peak": hbm, "peak_kind": f"{peak_kind} hbm_gbs",
-                            "unit": "GB/s", "frac": prof_gbs / hbm, "traffic": None,
+                            "unit": "GB/s", "frac": prof_gbs / hbm,
+                            "traffic": PROF_NCU_TRAFFIC.get(prof_source_key()) if wl.name == "hunyuan" else None,
                             "algorithmic_work": f"{prof_bytes:.4e} bytes/launch = K and V of every head once"}
     configs = None
     if not args.no_configs and rank == 0 and world == 1 and wl.name == "hunyuan":

@@ -455,17 +455,21 @@ def time_calls(fn, reps, stream, warm=2):
     return a.elapsed_time(b) / reps
 
 
-def measure_config(wl, dev, stream, peak, seed=0, steps=5, warm=2):
+def measure_config(wl, dev, stream, peak, seed=0, steps=5, warm=2, layout="bhld"):
     """One workload timed outside the headline's timed region: the whole call
     step by step (profile -> attention with the layout the call picks, or
-    permute -> attention -> unpermute), CUDA events around each stage.
-    Returns ms per call, attention-kernel ms, effective TFLOPS and the
-    fraction of the bf16 peak."""
+    permute -> attention -> unpermute), CUDA events around each stage, on
+    [B, H, L, d] tensors or (layout "blhd") [B, L, H, d] ones.  Returns ms per
+    call, attention-kernel ms, effective TFLOPS and the fraction of the bf16
+    peak."""
     from sparse_attention_video_profile_b200 import svg
     q, k, v = synth.make_qkv(wl, seed=seed, device=dev)
+    if layout == "blhd":
+        q, k, v = (t.transpose(1, 2).contiguous() for t in (q, k, v))
     rows = torch.from_numpy(synth.sample_rows(wl.L, wl.S, seed)).to(dev)
     N, F = wl.N, wl.F
-    shape = svg.make_shape(q, N, F)
+    shape = svg.make_shape(q, N, F, layout=layout)
+    lk = {"layout": layout}  # every call of this config
     o = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     mixed = wl.name.startswith("mixed")
@@ -486,24 +490,24 @@ def measure_config(wl, dev, stream, peak, seed=0, steps=5, warm=2):
     def step(ev):
         ev[0].record(stream)
         if not mixed:
-            svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws)
+            svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws, **lk)
         lab = md_label if mixed else label
         if not fused:
-            svg.svg_permute_qkv(q, k, v, N, F, lab, out=(qp, kp, vp))
+            svg.svg_permute_qkv(q, k, v, N, F, lab, out=(qp, kp, vp), **lk)
         ev[1].record(stream)
         if mixed and fused:
             svg.svg_mixed_attn_fused(q, k, v, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
-                                     status=status)
+                                     status=status, **lk)
         elif mixed:
             svg.svg_mixed_attn(q, k, v, qp, kp, vp, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
-                               op=op, status=status)
+                               op=op, status=status, **lk)
         elif fused:
-            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status)
+            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status, **lk)
         else:
-            svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status)
+            svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status, **lk)
         ev[2].record(stream)
         if not fused:
-            svg.svg_unpermute(op, N, F, lab, out=o)
+            svg.svg_unpermute(op, N, F, lab, out=o, **lk)
         ev[3].record(stream)
 
     def events():
@@ -525,7 +529,8 @@ def measure_config(wl, dev, stream, peak, seed=0, steps=5, warm=2):
     else:
         pairs = metrics.effective_pairs(N, F, wl.a1, wl.a2, label.cpu().numpy())
     tflops = metrics.attention_flops(pairs, wl.d) / (attn_ms * 1e-3) / 1e12
-    return {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={N} F={F} L={wl.L} d={wl.d} a1={wl.a1} a2={wl.a2}",
+    tag = "" if layout == "bhld" else " [B, L, H, d]"
+    return {"workload": f"{wl.name}{tag}: B={wl.B} H={wl.H} N={N} F={F} L={wl.L} d={wl.d} a1={wl.a1} a2={wl.a2}",
             "ms": call_ms, "attn_ms": attn_ms, "effective_tflops": tflops, "frac_bf16_peak": tflops / peak,
             "density": pairs / (wl.B * wl.H * float(wl.L) * wl.L),
             "layout": "fused" if fused else "separate", "steps": steps}
@@ -796,6 +801,9 @@ def run_ours(args, wl, rank, world, local):
                    wl.with_bands(*synth.HUNYUAN_SWEEP[0.5], name="hunyuan-50%"), synth.WORKLOADS["mixed"]):
             configs.append(measure_config(cw, dev, stream, peak))
             torch.cuda.empty_cache()
+        # the headline workload again on [B, L, H, d] tensors
+        configs.append(measure_config(wl, dev, stream, peak, layout="blhd"))
+        torch.cuda.empty_cache()
     # the seconds-long power-capped figure, shown beside the burst one
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
 

@@ -29,10 +29,16 @@
  *   Shapes.   B batch, H heads, N frames, F tokens per frame, L = N*F tokens,
  *             d head dim.  Token (i, j) (frame i, in-frame position j) sits at
  *             row x = i*F + j of the frame-major layout.
- *   Layout.   Every Q/K/V/O tensor is contiguous [B, H, L, d], row-major, d
- *             fastest, in the element type of shape->dtype (bf16 or fp32).
- *             Token-major ("permuted") tensors have the same shape with
- *             token (i, j) at row x' = j*N + i.
+ *   Layout.   Every Q/K/V/O tensor argument of a call is contiguous, d
+ *             fastest, in the element type of shape->dtype (bf16 or fp32),
+ *             and ordered as shape->layout says: [B, H, L, d]
+ *             (SVG_LAYOUT_BHLD, the default) or [B, L, H, d]
+ *             (SVG_LAYOUT_BLHD, the heads of one token side by side, as a
+ *             fused QKV projection writes them).  The arithmetic does not
+ *             depend on the layout: both give bit-identical results.
+ *             Token-major ("permuted") tensors have the same shape and
+ *             layout with token (i, j) at row x' = j*N + i.  Workspaces are
+ *             opaque.  svg_sparse_3d_attn_host takes [B, H, L, d] only.
  *   Labels.   int8 per (b, h), [B, H]: SVG_SPATIAL (0) or SVG_TEMPORAL (1),
  *             standing for the pages' -1 and +1.
  *   Memory.   The caller allocates and owns every buffer.  Pointers named
@@ -92,14 +98,19 @@ typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
 #define SVG_DEV_BOUNDS 0x4u   /* debug build only: a kernel index outside its buffer (the access was
                                  skipped; see svg_debug_checks) */
 
+/* Order of the Q/K/V/O tensors of a call (svg_shape.layout). */
+#define SVG_LAYOUT_BHLD 0 /* [B, H, L, d]: each head's L rows are contiguous */
+#define SVG_LAYOUT_BLHD 1 /* [B, L, H, d]: row x of head h is H*d elements after row x - 1 */
+
 typedef struct svg_shape {
   int32_t B, H, N, F, d;
-  int32_t dtype; /* svg_dtype */
-  float scale;   /* softmax scale on q.k; 0 selects 1/sqrt(d) */
+  int32_t dtype;  /* svg_dtype */
+  float scale;    /* softmax scale on q.k; 0 selects 1/sqrt(d) */
+  int32_t layout; /* SVG_LAYOUT_*; a zero-initialised shape is [B, H, L, d] */
 } svg_shape;
 
-/* ABI version of this header (bumped on any signature change). */
-#define SVG_ABI_VERSION 1
+/* ABI version of this header (bumped on any signature or struct change). */
+#define SVG_ABI_VERSION 2
 SVG_API int32_t svg_abi_version(void);
 
 /* Static text for a status code; never NULL. */
@@ -366,6 +377,8 @@ SVG_API size_t svg_sparse_3d_attn_host_workspace_size(const svg_shape* shape, in
  *
  * q_host, k_host, v_host, o_host: [B,H,L,d] in host memory, page-locked for the
  * copies to overlap (pageable memory works, but the copies then serialise);
+ * shape->layout must be SVG_LAYOUT_BHLD (a chunk of heads is then one
+ * contiguous copy), else SVG_ERR_UNSUPPORTED;
  * rows_host [S], mse_host [B,H,2], label_host [B,H] in host memory.  Heads
  * are independent, so the call is cut into chunks of heads_per_chunk heads.
  * The host-to-device copies of one chunk, the kernels of another and the
@@ -399,13 +412,14 @@ SVG_API svg_status svg_head_shard(int32_t n_heads, int32_t rank, int32_t world, 
 /*
  * svg_sparse_3d_attn_shard_workspace_size / svg_sparse_3d_attn_shard --
  * svg_sparse_3d_attn on this rank's block of heads only.  q, k, v, o, mse and
- * label are the FULL [B, H, ...] tensors on this rank's device (the same
- * addresses' layout as for svg_sparse_3d_attn); only the block's heads are
- * read and written, so a caller that wants the whole output gathers the
- * blocks from the other ranks afterwards (one all-gather over NVLink), and a
- * caller that keeps heads sharded never does.  The workspace is sized for
- * the block.  With no heads on this rank the call does nothing and returns
- * SVG_OK.
+ * label are the FULL tensors on this rank's device, in shape->layout as for
+ * svg_sparse_3d_attn; heads are numbered over (b, h), so in [B, L, H, d] a
+ * block can end in one batch entry and go on in the next.  Only the block's
+ * heads are read and written, so a caller that wants the whole output
+ * gathers the blocks from the other ranks afterwards (one all-gather over
+ * NVLink), and a caller that keeps heads sharded never does.  The workspace
+ * is sized for the block.  With no heads on this rank the call does nothing
+ * and returns SVG_OK.
  */
 SVG_API size_t svg_sparse_3d_attn_shard_workspace_size(const svg_shape* shape, int32_t rank, int32_t world,
                                                        int32_t a2, int32_t S);

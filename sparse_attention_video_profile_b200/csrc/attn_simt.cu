@@ -18,8 +18,8 @@ template <int D>
 __global__ void __launch_bounds__(kSimtWarps * 32)
     attn_simt_kernel(const float* __restrict__ q0, const float* __restrict__ k0, const float* __restrict__ v0,
                      float* __restrict__ o0, const float* __restrict__ q1, const float* __restrict__ k1,
-                     const float* __restrict__ v1, float* __restrict__ o1, const int8_t* __restrict__ label,
-                     int BH, int L, int G0, int a0, int G1, int a1, float sl2) {
+                     const float* __restrict__ v1, float* __restrict__ o1, const HeadStrides s0, const HeadStrides s1,
+                     const int8_t* __restrict__ label, int BH, int L, int G0, int a0, int G1, int a1, float sl2) {
   constexpr int PER = D / 32;
   __shared__ float sq[kSimtWarps][D];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
   const int x = static_cast<int>(gid - static_cast<long long>(bh) * L);
   const int lab = (label != nullptr && label[bh] == SVG_TEMPORAL) ? 1 : 0;  // any other label runs spatial
   const int G = lab ? G1 : G0, a = lab ? a1 : a0;
-  const size_t hoff = static_cast<size_t>(bh) * L * D;
+  const HeadStrides& hs = lab ? s1 : s0;  // (q0, k0, v0, o0) and (q1, k1, v1, o1) layouts
+  const long long hoff = hs.head(bh), sl = hs.sl;
   const float* q = (lab ? q1 : q0) + hoff;
   const float* k = (lab ? k1 : k0) + hoff;
   const float* v = (lab ? v1 : v0) + hoff;
@@ -39,7 +40,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
   const int lo = static_cast<int>(max(0LL, (g - a + 1) * G));
   const int hi = static_cast<int>(min(static_cast<long long>(L), (g + a) * G));
 
-  for (int c = lane; c < D; c += 32) sq[warp][c] = q[static_cast<size_t>(x) * D + c] * sl2;
+  for (int c = lane; c < D; c += 32) sq[warp][c] = q[x * sl + c] * sl2;
   __syncwarp();
 
   float m = -INFINITY, l = 0.f, acc[PER];
@@ -50,7 +51,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
     const int y = y0 + lane;
     float s = -INFINITY;
     if (y < hi) {
-      const float* kr = k + static_cast<size_t>(y) * D;
+      const float* kr = k + y * sl;
       float dot = 0.f;
 #pragma unroll 8
       for (int c = 0; c < D; ++c) dot = fmaf(sq[warp][c], kr[c], dot);
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
     const int nvalid = min(32, hi - y0);
     for (int jj = 0; jj < nvalid; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const float* vr = v + static_cast<size_t>(y0 + jj) * D;
+      const float* vr = v + (y0 + jj) * sl;
 #pragma unroll
       for (int t = 0; t < PER; ++t) acc[t] = fmaf(pj, vr[lane + 32 * t], acc[t]);
     }
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-  for (int t = 0; t < PER; ++t) o[static_cast<size_t>(x) * D + lane + 32 * t] = acc[t] * inv;
+  for (int t = 0; t < PER; ++t) o[x * sl + lane + 32 * t] = acc[t] * inv;
 }
 
 template <int D>
@@ -91,8 +92,8 @@ svg_status launch_simt_d(const BandAttnArgs& a, cudaStream_t stream) {
   attn_simt_kernel<D><<<static_cast<unsigned>(blocks), kSimtWarps * 32, 0, stream>>>(
       static_cast<const float*>(a.q), static_cast<const float*>(a.k), static_cast<const float*>(a.v),
       static_cast<float*>(a.o), static_cast<const float*>(a.qp), static_cast<const float*>(a.kp),
-      static_cast<const float*>(a.vp), static_cast<float*>(a.op), a.label, a.B * a.H, a.L, a.G0, a.a0, a.G1,
-      a.a1, sl2);
+      static_cast<const float*>(a.vp), static_cast<float*>(a.op), a.hs, a.label ? a.hsp : a.hs, a.label, a.B * a.H,
+      a.L, a.G0, a.a0, a.G1, a.a1, sl2);
   return cuda_check(cudaGetLastError(), "fp32 attention launch");
 }
 

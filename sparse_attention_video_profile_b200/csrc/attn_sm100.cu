@@ -39,22 +39,20 @@
 
 namespace svg {
 
-svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D);
-svg_status make_group_map_bf16(CUtensorMap* map, const void* base, int BH, int N, int F, int D, int size);
-
 namespace {
 
 constexpr int kMaxFrameGroups = 24;
 
 struct AttnParams {
-  CUtensorMap tm_q, tm_k, tm_v;     // frame-major [BH, L, D] bf16
-  CUtensorMap tm_qp, tm_kp, tm_vp;  // token-major [BH, L, D] bf16
+  CUtensorMap tm_q, tm_k, tm_v;     // frame-major, laid out as st_in
+  CUtensorMap tm_qp, tm_kp, tm_vp;  // token-major, laid out as st_p
   // Fused layout transformation: 4D views (d, frame, position, head) of the
   // frame-major q/k/v whose box is s frames x 128/s positions (s = 2^e, map
   // index e): one box is a 128-row tile already in token-major order.
   CUtensorMap tm_fq[8], tm_fk[8], tm_fv[8];
-  __nv_bfloat16* o;
-  __nv_bfloat16* op;
+  __nv_bfloat16* o;   // laid out as st_o
+  __nv_bfloat16* op;  // laid out as st_p
+  HeadStrides st_in, st_p, st_o;
   const int8_t* label;  // spatial (0) / temporal (1) per head, or nullptr
   const int8_t* modes;  // mixed-pattern mode per head (SVG_MODE_*), or nullptr
   int BH, L, n_ctiles;
@@ -367,6 +365,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     nk = (hi_cta > lo_cta) ? (hi_cta + C::BK - 1) / C::BK - kt0 : 0;  // 0: skipped head
   }
   const bool run = (*abort_flag == 0);
+  const int th_in = p.st_in.tma_h(bh), tb_in = p.st_in.tma_b(bh);  // TMA (head, batch) of q, k, v
 
   if (warp >= 8) {
     if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads && fz) {
@@ -383,8 +382,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
-          tma_load_4d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, &p.tm_fq[p.glog[gq]], bar_q, h * 64,
-                      p.gfirst[gq], pq0 + (i << shq), bh);
+          tma_load_5d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, &p.tm_fq[p.glog[gq]], bar_q, h * 64,
+                      p.gfirst[gq], pq0 + (i << shq), th_in, tb_in);
       int g = 0, sh = 7 - p.glog[0], t = kp_lo >> sh, t_end = kp_hi >> sh;
       for (int n = 0; n < 2 * nk; ++n) {
         const int slot = n % C::NS;
@@ -399,8 +398,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
-          tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, p.gfirst[g],
-                      t << sh, bh);
+          tma_load_5d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, p.gfirst[g],
+                      t << sh, th_in, tb_in);
         if ((n & 1) && ++t > t_end && ++g < p.ng) {  // next key tile after its V
           sh = 7 - p.glog[g];
           t = kp_lo >> sh;
@@ -417,7 +416,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
-          tma_load_3d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, &p.tm_q, bar_q, h * 64, q0 + i * C::BQ, bh);
+          tma_load_4d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, &p.tm_q, bar_q, h * 64, q0 + i * C::BQ, th_in,
+                      tb_in);
       S2Run kr = s2_run(s2u, s2_koff, p.s2_Ck, 0);
       for (int n = 0; n < 2 * nk; ++n) {
         const int slot = n % C::NS;
@@ -431,7 +431,8 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
-          tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, kr.t, bh);
+          tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, kr.t, th_in,
+                      tb_in);
         if (n & 1) s2_next(kr, s2u, s2_koff, p.s2_Ck);
       }
     } else if (run && nk > 0 && warp == 8 && lane == 0 && !p.withhold_loads) {
@@ -440,6 +441,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       const CUtensorMap* tq = lab ? &p.tm_qp : &p.tm_q;
       const CUtensorMap* tk = lab ? &p.tm_kp : &p.tm_k;
       const CUtensorMap* tv = lab ? &p.tm_vp : &p.tm_v;
+      const int th = lab ? p.st_p.tma_h(bh) : th_in, tb = lab ? p.st_p.tma_b(bh) : tb_in;
       tma_prefetch_desc(tq);
       tma_prefetch_desc(tk);
       tma_prefetch_desc(tv);
@@ -449,7 +451,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
-          tma_load_3d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, tq, bar_q, h * 64, q0 + i * C::BQ, bh);
+          tma_load_4d(sQ + i * C::TILE_BYTES + h * C::HALF_BYTES, tq, bar_q, h * 64, q0 + i * C::BQ, th, tb);
       for (int n = 0; n < 2 * nk; ++n) {
         const int slot = n % C::NS;
         const uint32_t ph = (n / C::NS) & 1;
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
         mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < C::HALVES; ++h)
-          tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, row, bh);
+          tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64, row, th, tb);
       }
     }
     } else if (run && nk > 0 && warp == 9) {
@@ -771,7 +773,9 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
     } else if (nk == 0) {
       // skipped head: its output rows are zero
       if (row_ok && in_range(x_q, L, p.status) && in_range(bh, p.BH, p.status)) {
-        uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * L + x_q) * D);
+        const bool to_op = lab && !p.fused && !S2;
+        const HeadStrides& so = to_op ? p.st_p : p.st_o;
+        uint4* dst = reinterpret_cast<uint4*>((to_op ? p.op : p.o) + so.head(bh) + x_q * so.sl);
 #pragma unroll
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -790,7 +794,9 @@ __global__ void __launch_bounds__(320, 1) attn_sm100_kernel(const __grid_constan
       // the frame-major position of their row in o
       const bool store_ok = row_ok && in_range(x_q, L, p.status) && in_range(bh, p.BH, p.status);
       const int orow = store_ok ? x_q : 0;
-      __nv_bfloat16* out = (lab && !p.fused && !S2 ? p.op : p.o) + (static_cast<size_t>(bh) * L + orow) * D;
+      const bool to_op = lab && !p.fused && !S2;
+      const HeadStrides& so = to_op ? p.st_p : p.st_o;
+      __nv_bfloat16* out = (to_op ? p.op : p.o) + so.head(store_ok ? bh : 0) + orow * so.sl;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -832,13 +838,18 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
   memset(&p, 0, sizeof(p));
   const int BH = a.B * a.H;
   svg_status st;
-  if ((st = make_tile_map_bf16(&p.tm_q, a.q, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_tile_map_bf16(&p.tm_k, a.k, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_tile_map_bf16(&p.tm_v, a.v, BH, a.L, D)) != SVG_OK) return st;
   const bool perm = (a.label != nullptr || a.modes != nullptr) && !a.fused;
-  if ((st = make_tile_map_bf16(&p.tm_qp, perm ? a.qp : a.q, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_tile_map_bf16(&p.tm_kp, perm ? a.kp : a.k, BH, a.L, D)) != SVG_OK) return st;
-  if ((st = make_tile_map_bf16(&p.tm_vp, perm ? a.vp : a.v, BH, a.L, D)) != SVG_OK) return st;
+  // q, k, v: the caller's, or in the SVG2 mode the cluster-permuted copies;
+  // qp..op: the token-major copies, standing in for q..o when unused
+  p.st_in = a.s2 ? a.hsp : a.hs;
+  p.st_p = perm ? a.hsp : p.st_in;
+  p.st_o = a.hs;
+  if ((st = make_tile_map_bf16(&p.tm_q, a.q, p.st_in, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_k, a.k, p.st_in, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_v, a.v, p.st_in, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_qp, perm ? a.qp : a.q, p.st_p, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_kp, perm ? a.kp : a.k, p.st_p, a.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_vp, perm ? a.vp : a.v, p.st_p, a.L, D)) != SVG_OK) return st;
   p.fused = a.fused;
   p.F = a.N > 0 ? a.L / a.N : 0;
   p.s2 = a.s2;
@@ -875,9 +886,9 @@ svg_status launch_d(const BandAttnArgs& a, cudaStream_t stream) {
       const int lg = p.glog[g];
       if (made[lg]) continue;
       made[lg] = true;
-      if ((st = make_group_map_bf16(&p.tm_fq[lg], a.q, BH, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
-      if ((st = make_group_map_bf16(&p.tm_fk[lg], a.k, BH, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
-      if ((st = make_group_map_bf16(&p.tm_fv[lg], a.v, BH, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
+      if ((st = make_group_map_bf16(&p.tm_fq[lg], a.q, p.st_in, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
+      if ((st = make_group_map_bf16(&p.tm_fk[lg], a.k, p.st_in, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
+      if ((st = make_group_map_bf16(&p.tm_fv[lg], a.v, p.st_in, a.N, p.F, D, 1 << lg)) != SVG_OK) return st;
     }
   }
   p.o = static_cast<__nv_bfloat16*>(a.o);
@@ -937,36 +948,40 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH, L, D] bf16, box = 64 elements x 128 rows x 1 head, 128-byte swizzle.
-svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D) {
+// 4D view (d, row, head, batch entry): box = 64 elements x 128 rows, 128-byte
+// swizzle.  In [B, L, H, d] the row stride exceeds the head stride, so the
+// strides need not increase with the dimension.
+svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, const HeadStrides& s, int L, int D) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(s.H),
+                              static_cast<cuuint64_t>(s.nb)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(s.sl) * 2, static_cast<cuuint64_t>(s.sh) * 2,
+                                 static_cast<cuuint64_t>(s.sb) * 2};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return SVG_OK;
 }
 
-// 4D view (d, frame, position, head) of a frame-major [BH, N*F, D] bf16
-// tensor with a box of `size` frames x 128/size positions: the box's 128 rows
-// come out position-major, i.e. in the token-major order of those frames.
-// Dimension 1 (frames) has the larger stride, so the strides are not in
-// increasing order; the box walks frames fastest.
-svg_status make_group_map_bf16(CUtensorMap* map, const void* base, int BH, int N, int F, int D, int size) {
+// 5D view (d, frame, position, head, batch entry) of a frame-major tensor
+// with a box of `size` frames x 128/size positions: the box's 128 rows come
+// out position-major, i.e. in the token-major order of those frames.  The
+// frame dimension has the larger stride, so the box walks frames fastest.
+svg_status make_group_map_bf16(CUtensorMap* map, const void* base, const HeadStrides& s, int N, int F, int D,
+                               int size) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return fail(SVG_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(F),
-                              static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(F) * D * 2, static_cast<cuuint64_t>(D) * 2,
-                                 static_cast<cuuint64_t>(N) * F * D * 2};
-  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(size), static_cast<cuuint32_t>(128 / size), 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(F),
+                              static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.nb)};
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(F) * s.sl * 2, static_cast<cuuint64_t>(s.sl) * 2,
+                                 static_cast<cuuint64_t>(s.sh) * 2, static_cast<cuuint64_t>(s.sb) * 2};
+  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(size), static_cast<cuuint32_t>(128 / size), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)

@@ -115,6 +115,8 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
                                            int32_t heads_per_chunk, void* workspace, size_t workspace_bytes,
                                            int32_t* status_dev, void* stream) {
   if (shape == nullptr) return fail(SVG_ERR_INVALID_ARG, "shape is NULL");
+  if (shape->layout != SVG_LAYOUT_BHLD)
+    return fail(SVG_ERR_UNSUPPORTED, "the host-buffer call copies whole heads: [B, H, L, d] tensors only");
   if (!q_host || !k_host || !v_host || !o_host || !rows_host || !mse_host || !label_host || !workspace)
     return fail(SVG_ERR_INVALID_ARG, "NULL host buffer or workspace");
   if (heads_per_chunk < 1) return fail(SVG_ERR_INVALID_ARG, "heads_per_chunk must be >= 1");
@@ -175,7 +177,7 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
     svg_shape cs = *shape;
     cs.B = 1;
     cs.H = nh;
-    if ((st = profile_heads_impl(&cs, q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, status_dev, sc,
+    if ((st = profile_heads_impl(&cs, shape_strides(&cs), q, k, v, a1, a2, rows, S, mse, lab, prof, lay.prof, status_dev, sc,
                                  full_call_chunk(shape, S))) != SVG_OK)
       return st;
     if (fused) {

@@ -24,15 +24,49 @@ svg_status fail(svg_status st, const char* fmt, ...);
 // Maps a CUDA error to SVG_ERR_CUDA with a message; SVG_OK if e == cudaSuccess.
 svg_status cuda_check(cudaError_t e, const char* what);
 
+// ------------------------------------------------------------- tensor layout
+
+// Where the rows of a q/k/v/o tensor live.  Head bh of a call (bh = b*H + h
+// over the call's own heads) is head g = bh + bh0 of the tensor, whose nb
+// batch entries hold H heads each; element c of row x of that head sits at
+// element (g / H)*sb + (g % H)*sh + x*sl + c.  [B, H, L, d]: sb = H*L*d,
+// sh = L*d, sl = d.  [B, L, H, d]: sb = L*H*d, sh = d, sl = H*d.
+struct HeadStrides {
+  int H, nb, bh0;
+  long long sb, sh, sl;
+  __host__ __device__ long long head(int bh) const {
+    const int g = bh + bh0;
+    return static_cast<long long>(g / H) * sb + static_cast<long long>(g % H) * sh;
+  }
+  // TMA coordinates (head, batch entry) of call head bh
+  __host__ __device__ int tma_h(int bh) const { return (bh + bh0) % H; }
+  __host__ __device__ int tma_b(int bh) const { return (bh + bh0) / H; }
+};
+// Contiguous [B, H, L, d] (workspace copies are always laid out this way).
+HeadStrides dense_strides(int B, int H, int L, int d);
+// The caller's tensors of a call on `s` (s->layout).
+HeadStrides shape_strides(const svg_shape* s);
+
+// TMA views (bf16, 128-byte swizzle) of a tensor laid out as s, indexed by
+// (column, row, tma_h, tma_b):
+// tiles (d, L, H, nb) with 64 x 128 x 1 x 1 boxes (attn_sm100.cu);
+svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, const HeadStrides& s, int L, int D);
+// frame groups (d, frame, position, H, nb) of a frame-major tensor with
+// `size` frames x 128/size positions per box, indexed (column, first frame,
+// first position, tma_h, tma_b).
+svg_status make_group_map_bf16(CUtensorMap* map, const void* base, const HeadStrides& s, int N, int F, int D,
+                               int size);
+
 // ------------------------------------------------------------- permute
 
 // Moves rows between frame-major (x = i*F + j) and token-major (x' = j*N + i)
 // order for up to three tensors.  to_token_major: src frame-major -> dst
 // token-major; otherwise the inverse.  label == nullptr: every head.
 // Only heads whose label equals `sel` move (SVG_TEMPORAL unless given).
-svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F,
-                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream,
-                          int sel = SVG_TEMPORAL);
+// Rows of d elements of elem_bytes each; src and dst laid out as ss and ds.
+svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F, int d,
+                          int elem_bytes, const HeadStrides& ss, const HeadStrides& ds, const int8_t* label,
+                          bool to_token_major, cudaStream_t stream, int sel = SVG_TEMPORAL);
 
 // ------------------------------------------------------------- attention
 
@@ -40,6 +74,9 @@ struct BandAttnArgs {
   int B, H, L, d;
   int dtype;  // svg_dtype
   float scale;
+  // Layouts: hs of q, k, v, o; hsp of qp, kp, vp, op (and, in the SVG2 mode,
+  // of the cluster-permuted q, k, v).
+  HeadStrides hs, hsp;
   // frame-major tensors (spatial heads, or all heads when label == nullptr)
   const void *q, *k, *v;
   void* o;
@@ -79,15 +116,16 @@ struct Svg2Sizes {
 Svg2Sizes svg2_sizes(int BH, int L, int Cq, int Ck, int d);
 svg_status svg2_sort(const int32_t* assign, int BH, int L, int C, int nblk, int32_t* hist, int32_t* perm,
                      int32_t* cid, int32_t* off, int* status, cudaStream_t stream);
-svg_status svg2_gather(const void* src, const int32_t* perm, void* dst, int BH, int L, int d, cudaStream_t stream);
+svg_status svg2_gather(const void* src, const HeadStrides& ss, const int32_t* perm, void* dst, int BH, int L, int d,
+                       cudaStream_t stream);
 svg_status svg2_centroids(const void* xp, const int32_t* off, int BH, int L, int C, int d, float* mu,
                           cudaStream_t stream);
 svg_status svg2_topp(const float* mu_q, const float* mu_k, const int32_t* off_k, int BH, int Cq, int Ck, int d,
                      float scale, float p, uint32_t* sel, cudaStream_t stream);
 // k-means (kmeans_sm100.cu): workspace bytes and the Lloyd iterations.
 size_t kmeans_workspace_bytes(int BH, int L, int C, int d);
-svg_status launch_kmeans(const void* x, int BH, int L, int C, int d, int iters, int32_t* assign, float* mu,
-                         void* workspace, int* status, cudaStream_t stream);
+svg_status launch_kmeans(const void* x, const HeadStrides& xs, int BH, int L, int C, int d, int iters, int32_t* assign,
+                         float* mu, void* workspace, int* status, cudaStream_t stream);
 
 svg_status launch_attn_sm100(const BandAttnArgs& a, cudaStream_t stream);
 // Frame groups of the fused layout transformation: powers of two, largest
@@ -139,7 +177,7 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
 // (zeroed first, so calls with separate workspaces do not interfere) and,
 // when status_out is not NULL, also OR-ed into *status_out.
 svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
-                          const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
+                          const void* k, const void* v, const HeadStrides& hs, int a1, int a2, const int32_t* rows, int S,
                           float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
                           int* status_out, cudaStream_t stream);
 
@@ -153,20 +191,20 @@ constexpr int kProfNone = 4;          // no key
 // bf16 stage 1 of profiling on the tensor cores (profile_sm100.cu): dense and
 // two restricted variants (kind[v], par[v]) of the sampled rows' attention.
 svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const void* q, const void* k,
-                                const void* v, const int (&kind)[2], const int (&par)[2], const int32_t* rows, int S,
+                                const void* v, const HeadStrides& hs, const int (&kind)[2], const int (&par)[2], const int32_t* rows, int S,
                                 float* ws_o, float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream);
 
 // One profiling pass: stage 1 with the given variants, then the per-row sums
 // part[bh][s][3] = {sum (O_1 - O_d)^2, sum (O_2 - O_d)^2, sum O_d^2} over d.
 svg_status launch_profile_pass(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
-                               const void* k, const void* v, const int (&kind)[2], const int (&par)[2],
+                               const void* k, const void* v, const HeadStrides& hs, const int (&kind)[2], const int (&par)[2],
                                const int32_t* rows, int S, void* ws, const ProfileLayout& lay, double* part,
                                int* status, cudaStream_t stream);
 
 // Sparse-vDiT mode search: two passes (diagonal, multi-diagonal) and (stripe,
 // none) plus the selection kernel.  part2 holds the second pass's sums.
 svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, const void* q, const void* k,
-                              const void* v, const int32_t* rows, int S, int window, int md_half, int stripe,
+                              const void* v, const HeadStrides& hs, const int32_t* rows, int S, int window, int md_half, int stripe,
                               float lambda, float epsilon, float* loss, int8_t* mode, void* ws,
                               const ProfileLayout& lay, double* part2, cudaStream_t stream);
 
@@ -176,8 +214,10 @@ svg_status internal_status_word(int** out, cudaStream_t stream);
 
 // svg_profile_heads with the failure bits also OR-ed into status_out (may be
 // NULL); the whole calls use it to carry a profiling failure to the caller.
-// chunk_len > 0 fixes the profiling key split (see profile_layout).
-svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
+// q, k, v are laid out as hs.  chunk_len > 0 fixes the profiling key split
+// (see profile_layout).
+svg_status profile_heads_impl(const svg_shape* shape, const HeadStrides& hs, const void* q, const void* k,
+                              const void* v, int32_t a1,
                               int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
                               size_t workspace_bytes, int32_t* status_out, cudaStream_t stream, int chunk_len = 0);
 

@@ -26,16 +26,15 @@
 
 namespace svg {
 
-svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D);
-
 namespace {
 
 constexpr int kKmThreads = 320;  // warps 0-7 epilogue (two threads per row), 8 TMA, 9 MMA
 constexpr int kKmSlotCols = 256;
 
 struct KmParams {
-  CUtensorMap tm_x;  // rows of x: [BH, L, D], box 64 x 128
+  CUtensorMap tm_x;  // rows of x, laid out as xs, box 64 x 128
   CUtensorMap tm_c;  // bf16 centroids: [BH, C, D], box 64 x 128
+  HeadStrides xs;
   const float* norm;  // [BH][C] ||bf16 centroid||^2
   int32_t* assign;    // [BH][L]
   int L, C, C_pad, nch, tiles, tiles_per_cta;
@@ -111,8 +110,9 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
     for (int r = 0; r < p.C_pad; r += 128)
 #pragma unroll
       for (int h = 0; h < K::HALVES; ++h)
-        tma_load_3d(sC + static_cast<size_t>(h) * p.C_pad * 128 + static_cast<size_t>(r) * 128, &p.tm_c, bar_c, h * 64,
-                    r, bh);
+        tma_load_4d(sC + static_cast<size_t>(h) * p.C_pad * 128 + static_cast<size_t>(r) * 128, &p.tm_c, bar_c, h * 64,
+                    r, bh, 0);
+    const int th = p.xs.tma_h(bh), tb = p.xs.tma_b(bh);
     for (int i = 0; i < nt; ++i) {
       const int s = i & 1;
       if (!mbar_wait(&bar_xempty[s], ((i >> 1) & 1) ^ 1, p.wait_ns)) {
@@ -122,7 +122,8 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
       mbar_arrive_expect_tx(&bar_xfull[s], K::TILE_BYTES);
 #pragma unroll
       for (int h = 0; h < K::HALVES; ++h)
-        tma_load_3d(sX + s * K::TILE_BYTES + h * K::HALF_BYTES, &p.tm_x, &bar_xfull[s], h * 64, (t_begin + i) * 128, bh);
+        tma_load_4d(sX + s * K::TILE_BYTES + h * K::HALF_BYTES, &p.tm_x, &bar_xfull[s], h * 64, (t_begin + i) * 128, th,
+                    tb);
     }
   } else if (nt > 0 && warp == 9) {
     // ---------------------------------------------- MMA issuer (whole warp, elected lane issues)
@@ -250,13 +251,13 @@ __global__ void __launch_bounds__(kKmThreads, 1) kmeans_assign_kernel(const __gr
 
 // Centroids of the rows floor(c L / C) (fp32, bf16 copy, norm of the copy).
 template <int D>
-__global__ void __launch_bounds__(32) kmeans_init_kernel(const __nv_bfloat16* __restrict__ x, int L, int C,
-                                                         float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_b,
-                                                         float* __restrict__ norm) {
+__global__ void __launch_bounds__(32) kmeans_init_kernel(const __nv_bfloat16* __restrict__ x, const HeadStrides xs,
+                                                         int L, int C, float* __restrict__ mu,
+                                                         __nv_bfloat16* __restrict__ mu_b, float* __restrict__ norm) {
   constexpr int PER = D / 32;
   const int c = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x;
   const long long r = static_cast<long long>(c) * L / C;
-  const __nv_bfloat16* xr = x + (static_cast<size_t>(bh) * L + r) * D;
+  const __nv_bfloat16* xr = x + xs.head(bh) + r * xs.sl;
   const size_t o = (static_cast<size_t>(bh) * C + c) * D;
   float n2 = 0.f;
 #pragma unroll
@@ -280,6 +281,7 @@ constexpr int kUpdWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kUpdWarps * 32) kmeans_update_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const HeadStrides xs,
                                                             const int32_t* __restrict__ perm,
                                                             const int32_t* __restrict__ off, int L, int C,
                                                             float* __restrict__ mu, __nv_bfloat16* __restrict__ mu_b,
@@ -293,12 +295,13 @@ __global__ void __launch_bounds__(kUpdWarps * 32) kmeans_update_kernel(const __n
   float s[PER], t[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) s[e] = t[e] = 0.f;
-  const __nv_bfloat16* xh = x + static_cast<size_t>(bh) * L * D;
+  const __nv_bfloat16* xh = x + xs.head(bh);
+  const long long sl = xs.sl;
   const int32_t* pm = perm + static_cast<size_t>(bh) * L;
   int r = r0 + warp;
   for (; r + kUpdWarps < r1; r += 2 * kUpdWarps) {  // two independent rows per step
-    const __nv_bfloat16* xa = xh + static_cast<size_t>(pm[r]) * D;
-    const __nv_bfloat16* xb = xh + static_cast<size_t>(pm[r + kUpdWarps]) * D;
+    const __nv_bfloat16* xa = xh + pm[r] * sl;
+    const __nv_bfloat16* xb = xh + pm[r + kUpdWarps] * sl;
     __nv_bfloat16 va[PER], vb[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32) kmeans_update_kernel(const __n
     }
   }
   if (r < r1) {
-    const __nv_bfloat16* xa = xh + static_cast<size_t>(pm[r]) * D;
+    const __nv_bfloat16* xa = xh + pm[r] * sl;
 #pragma unroll
     for (int e = 0; e < PER; ++e) s[e] += __bfloat162float(xa[e * 32 + lane]);
   }
@@ -350,14 +353,15 @@ __global__ void __launch_bounds__(kUpdWarps * 32) kmeans_update_kernel(const __n
 }
 
 template <int D>
-svg_status launch_assign(const void* x, const __nv_bfloat16* mu_b, const float* norm, int BH, int L, int C,
-                         int32_t* assign, int* status, cudaStream_t stream) {
+svg_status launch_assign(const void* x, const HeadStrides& xs, const __nv_bfloat16* mu_b, const float* norm, int BH,
+                         int L, int C, int32_t* assign, int* status, cudaStream_t stream) {
   using K = KmCfg<D>;
   KmParams p;
   memset(&p, 0, sizeof(p));
   svg_status st;
-  if ((st = make_tile_map_bf16(&p.tm_x, x, BH, L, D)) != SVG_OK) return st;
-  if ((st = make_tile_map_bf16(&p.tm_c, mu_b, BH, C, D)) != SVG_OK) return st;
+  p.xs = xs;
+  if ((st = make_tile_map_bf16(&p.tm_x, x, xs, L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_c, mu_b, dense_strides(1, BH, C, D), C, D)) != SVG_OK) return st;
   p.norm = norm;
   p.assign = assign;
   p.L = L;
@@ -395,8 +399,8 @@ size_t kmeans_workspace_bytes(int BH, int L, int C, int d) {
          + al(static_cast<size_t>(BH) * (C + 1) * 4);   // offsets
 }
 
-svg_status launch_kmeans(const void* x, int BH, int L, int C, int d, int iters, int32_t* assign, float* mu,
-                         void* workspace, int* status, cudaStream_t stream) {
+svg_status launch_kmeans(const void* x, const HeadStrides& xs, int BH, int L, int C, int d, int iters, int32_t* assign,
+                         float* mu, void* workspace, int* status, cudaStream_t stream) {
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
   const int nblk = (L + 2047) / 2048;
   uint8_t* w = static_cast<uint8_t*>(workspace);
@@ -413,19 +417,19 @@ svg_status launch_kmeans(const void* x, int BH, int L, int C, int d, int iters, 
   int32_t* off = reinterpret_cast<int32_t*>(w);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (d == 128)
-    kmeans_init_kernel<128><<<dim3(C, BH), 32, 0, stream>>>(xb, L, C, mu, mu_b, norm);
+    kmeans_init_kernel<128><<<dim3(C, BH), 32, 0, stream>>>(xb, xs, L, C, mu, mu_b, norm);
   else
-    kmeans_init_kernel<64><<<dim3(C, BH), 32, 0, stream>>>(xb, L, C, mu, mu_b, norm);
+    kmeans_init_kernel<64><<<dim3(C, BH), 32, 0, stream>>>(xb, xs, L, C, mu, mu_b, norm);
   svg_status st = cuda_check(cudaGetLastError(), "k-means init launch");
   for (int it = 0; st == SVG_OK && it < iters; ++it) {
-    st = d == 128 ? launch_assign<128>(x, mu_b, norm, BH, L, C, assign, status, stream)
-                  : launch_assign<64>(x, mu_b, norm, BH, L, C, assign, status, stream);
+    st = d == 128 ? launch_assign<128>(x, xs, mu_b, norm, BH, L, C, assign, status, stream)
+                  : launch_assign<64>(x, xs, mu_b, norm, BH, L, C, assign, status, stream);
     if (st != SVG_OK) break;
     if ((st = svg2_sort(assign, BH, L, C, nblk, hist, perm, cid, off, status, stream)) != SVG_OK) break;
     if (d == 128)
-      kmeans_update_kernel<128><<<dim3(C, BH), kUpdWarps * 32, 0, stream>>>(xb, perm, off, L, C, mu, mu_b, norm);
+      kmeans_update_kernel<128><<<dim3(C, BH), kUpdWarps * 32, 0, stream>>>(xb, xs, perm, off, L, C, mu, mu_b, norm);
     else
-      kmeans_update_kernel<64><<<dim3(C, BH), kUpdWarps * 32, 0, stream>>>(xb, perm, off, L, C, mu, mu_b, norm);
+      kmeans_update_kernel<64><<<dim3(C, BH), kUpdWarps * 32, 0, stream>>>(xb, xs, perm, off, L, C, mu, mu_b, norm);
     st = cuda_check(cudaGetLastError(), "k-means update launch");
   }
   return st;

@@ -8,8 +8,9 @@
 // x' = j*N + i.  Every row is d contiguous elements (128 or 256 bytes in
 // bf16), so the transformation is a row gather: each 16-byte chunk is read
 // once and written once, and both sides touch whole rows, i.e. whole 32-byte
-// sectors.  The kernel walks the DESTINATION contiguously (coalesced
-// streaming stores) and gathers source rows; a block handles one slab of one
+// sectors.  The kernel walks the DESTINATION head row by row (coalesced
+// streaming stores; the rows are adjacent in [B, H, L, d] and H*d apart in
+// [B, L, H, d]) and gathers source rows; a block handles one slab of one
 // head of one tensor and exits at once for heads the label says stay put.
 #include "internal.h"
 
@@ -19,6 +20,7 @@ namespace {
 struct PermuteParams {
   const uint4* src[3];
   uint4* dst[3];
+  HeadStrides ss, ds;  // in 16-byte chunks
   const int8_t* label;
   int sel;                    // heads whose label equals sel move
   long long chunks_per_head;  // L * row_chunks
@@ -34,10 +36,10 @@ __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const __grid
   const int t = blockIdx.y / p.BH;       // tensor
   const int bh = blockIdx.y - t * p.BH;  // head
   if (p.label != nullptr && p.label[bh] != p.sel) return;
-  const long long head_off = static_cast<long long>(bh) * p.chunks_per_head;
-  const uint4* __restrict__ src = p.src[t] + head_off;
-  uint4* __restrict__ dst = p.dst[t] + head_off;
+  const uint4* __restrict__ src = p.src[t] + p.ss.head(bh);
+  uint4* __restrict__ dst = p.dst[t] + p.ds.head(bh);
   const int rc = p.row_chunks;
+  const long long srs = p.ss.sl, drs = p.ds.sl;  // row strides
   const long long step = static_cast<long long>(gridDim.x) * kPermThreads * kPermUnroll;
   for (long long base = static_cast<long long>(blockIdx.x) * kPermThreads * kPermUnroll + threadIdx.x;
        base < p.chunks_per_head; base += step) {
@@ -46,10 +48,11 @@ __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const __grid
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u) {
       const long long e = base + static_cast<long long>(u) * kPermThreads;
-      didx[u] = e;
+      didx[u] = -1;
       if (e < p.chunks_per_head) {
         const int row = static_cast<int>(e / rc);
         const int c = static_cast<int>(e - static_cast<long long>(row) * rc);
+        didx[u] = row * drs + c;
         int srow;
         if (p.to_token_major) {  // dst row x' = j*N + i  <-  src row i*F + j
           const int j = row / p.N, i = row - j * p.N;
@@ -58,21 +61,33 @@ __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(const __grid
           const int i = row / p.F, j = row - i * p.F;
           srow = j * p.N + i;
         }
-        val[u] = __ldg(src + static_cast<long long>(srow) * rc + c);
+        val[u] = __ldg(src + srow * srs + c);
       }
     }
 #pragma unroll
     for (int u = 0; u < kPermUnroll; ++u)
-      if (didx[u] < p.chunks_per_head) __stcs(dst + didx[u], val[u]);
+      if (didx[u] >= 0) __stcs(dst + didx[u], val[u]);
   }
 }
 
 }  // namespace
 
-svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F,
-                          int row_bytes, const int8_t* label, bool to_token_major, cudaStream_t stream, int sel) {
+svg_status launch_permute(int ntensors, const void* const* src, void* const* dst, int BH, int N, int F, int d,
+                          int elem_bytes, const HeadStrides& ss, const HeadStrides& ds, const int8_t* label,
+                          bool to_token_major, cudaStream_t stream, int sel) {
+  const int row_bytes = d * elem_bytes;
   if (row_bytes % 16 != 0) return fail(SVG_ERR_UNSUPPORTED, "row of %d bytes is not a multiple of 16", row_bytes);
+  // element strides -> 16-byte chunks (every stride is a multiple of d)
+  const int per = 16 / elem_bytes;
+  auto chunks = [per](HeadStrides s) {
+    s.sb /= per;
+    s.sh /= per;
+    s.sl /= per;
+    return s;
+  };
   PermuteParams p{};
+  p.ss = chunks(ss);
+  p.ds = chunks(ds);
   for (int t = 0; t < ntensors; ++t) {
     p.src[t] = static_cast<const uint4*>(src[t]);
     p.dst[t] = static_cast<uint4*>(dst[t]);

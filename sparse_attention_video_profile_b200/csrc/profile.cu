@@ -30,9 +30,10 @@ namespace {
 constexpr int kKT = 128;  // keys per tile of the bf16 stage 1
 
 struct ProfParams {
-  const void* q;
+  const void* q;  // q, k, v laid out as hs
   const void* k;
   const void* v;
+  HeadStrides hs;
   const int32_t* rows;
   float* ws_o;   // [BH][nch][3][S_pad][D]
   float* ws_ml;  // [BH][nch][3][S_pad][2]  (max in log2 units, sum)
@@ -50,13 +51,13 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
   const int s = blockIdx.x * 4 + warp;
   const int bh = blockIdx.y;
   if (s >= p.S_pad) return;
-  const size_t hoff = static_cast<size_t>(bh) * p.L * D;
+  const long long hoff = p.hs.head(bh), sl = p.hs.sl;
   const float* q = static_cast<const float*>(p.q) + hoff;
   const float* k = static_cast<const float*>(p.k) + hoff;
   const float* v = static_cast<const float*>(p.v) + hoff;
   const int x = min(max(p.rows[min(s, p.S - 1)], 0), p.L - 1);
   const int ir = x / p.F, jr = x % p.F;
-  for (int c = lane; c < D; c += 32) sq[warp][c] = q[static_cast<size_t>(x) * D + c] * p.sl2;
+  for (int c = lane; c < D; c += 32) sq[warp][c] = q[x * sl + c] * p.sl2;
   __syncwarp();
   float m[3], l[3], acc[3][PER];
 #pragma unroll
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
     float sc = -INFINITY;
     int iy = -1, jy = -1;
     if (y < p.L) {
-      const float* kr = k + static_cast<size_t>(y) * D;
+      const float* kr = k + y * sl;
       float dot = 0.f;
 #pragma unroll 8
       for (int c = 0; c < D; ++c) dot = fmaf(sq[warp][c], kr[c], dot);
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
     }
     const int nvalid = min(32, p.L - y0);
     for (int jj = 0; jj < nvalid; ++jj) {
-      const float* vr = v + static_cast<size_t>(y0 + jj) * D;
+      const float* vr = v + (y0 + jj) * sl;
       float vals[PER];
 #pragma unroll
       for (int t = 0; t < PER; ++t) vals[t] = vr[lane + 32 * t];
@@ -337,13 +338,14 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
 }
 
 svg_status launch_profile_pass(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
-                               const void* k, const void* v, const int (&kind)[2], const int (&par)[2],
+                               const void* k, const void* v, const HeadStrides& hs, const int (&kind)[2], const int (&par)[2],
                                const int32_t* rows, int S, void* ws, const ProfileLayout& lay, double* part,
                                int* status, cudaStream_t stream) {
   ProfParams p{};
   p.q = q;
   p.k = k;
   p.v = v;
+  p.hs = hs;
   p.rows = rows;
   p.ws_o = static_cast<float*>(ws);
   p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.o_bytes);
@@ -361,7 +363,7 @@ svg_status launch_profile_pass(int B, int H, int N, int F, int d, int dtype, flo
   if (p.BH > 65535) return fail(SVG_ERR_UNSUPPORTED, "B*H = %d exceeds the grid limit", p.BH);
   svg_status st;
   if (dtype == SVG_BF16) {
-    st = launch_profile_sm100(p.BH, N, F, d, scale, q, k, v, kind, par, rows, S, p.ws_o, p.ws_ml, lay.n_chunks,
+    st = launch_profile_sm100(p.BH, N, F, d, scale, q, k, v, hs, kind, par, rows, S, p.ws_o, p.ws_ml, lay.n_chunks,
                               lay.chunk, status, stream);
   } else {
     if (kind[0] != kProfFrameBand || kind[1] != kProfPositionBand)
@@ -386,7 +388,7 @@ static svg_status call_status_word(void* ws, const ProfileLayout& lay, int** out
 }
 
 svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float scale, const void* q,
-                          const void* k, const void* v, int a1, int a2, const int32_t* rows, int S,
+                          const void* k, const void* v, const HeadStrides& hs, int a1, int a2, const int32_t* rows, int S,
                           float* mse, int8_t* label, void* ws, const ProfileLayout& lay,
                           int* status_out, cudaStream_t stream) {
   int* status = nullptr;
@@ -394,7 +396,7 @@ svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float sc
   if (st != SVG_OK) return st;
   double* part = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
   const int kind[2] = {kProfFrameBand, kProfPositionBand}, par[2] = {a1, a2};
-  if ((st = launch_profile_pass(B, H, N, F, d, dtype, scale, q, k, v, kind, par, rows, S, ws, lay, part, status,
+  if ((st = launch_profile_pass(B, H, N, F, d, dtype, scale, q, k, v, hs, kind, par, rows, S, ws, lay, part, status,
                                 stream)) != SVG_OK)
     return st;
   profile_finalize_kernel<<<B * H, kCombineThreads, 0, stream>>>(part, S, lay.S_pad, d, mse, label, status,
@@ -403,7 +405,7 @@ svg_status launch_profile(int B, int H, int N, int F, int d, int dtype, float sc
 }
 
 svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, const void* q, const void* k,
-                              const void* v, const int32_t* rows, int S, int window, int md_half, int stripe,
+                              const void* v, const HeadStrides& hs, const int32_t* rows, int S, int window, int md_half, int stripe,
                               float lambda, float epsilon, float* loss, int8_t* mode, void* ws,
                               const ProfileLayout& lay, double* part2, cudaStream_t stream) {
   int* status = nullptr;
@@ -412,10 +414,10 @@ svg_status launch_mode_search(int B, int H, int N, int F, int d, float scale, co
   double* part1 = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + lay.o_bytes + lay.ml_bytes);
   const int kind1[2] = {kProfWindow, kProfPositionBand}, par1[2] = {window, md_half + 1};
   const int kind2[2] = {kProfPrefix, kProfNone}, par2[2] = {stripe, 0};
-  if ((st = launch_profile_pass(B, H, N, F, d, SVG_BF16, scale, q, k, v, kind1, par1, rows, S, ws, lay, part1,
+  if ((st = launch_profile_pass(B, H, N, F, d, SVG_BF16, scale, q, k, v, hs, kind1, par1, rows, S, ws, lay, part1,
                                 status, stream)) != SVG_OK)
     return st;
-  if ((st = launch_profile_pass(B, H, N, F, d, SVG_BF16, scale, q, k, v, kind2, par2, rows, S, ws, lay, part2,
+  if ((st = launch_profile_pass(B, H, N, F, d, SVG_BF16, scale, q, k, v, hs, kind2, par2, rows, S, ws, lay, part2,
                                 status, stream)) != SVG_OK)
     return st;
   // sparsity of each mode: 1 - kept pairs / L^2 (closed forms of the masks)

@@ -59,6 +59,8 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
     return fail(SVG_ERR_INVALID_ARG, "B, H, N, F, d must be >= 1");
   if (static_cast<long long>(shape->N) * shape->F > (1LL << 30)) return fail(SVG_ERR_INVALID_ARG, "L too large");
   if (shape->dtype != SVG_BF16 && shape->dtype != SVG_FP32) return fail(SVG_ERR_INVALID_ARG, "unknown dtype");
+  if (shape->layout != SVG_LAYOUT_BHLD && shape->layout != SVG_LAYOUT_BLHD)
+    return fail(SVG_ERR_INVALID_ARG, "unknown layout");
   if (!(shape->scale >= 0.f) || isinf(shape->scale)) return fail(SVG_ERR_INVALID_ARG, "bad scale");
   if ((shape->dtype == SVG_BF16 && shape->d != 64 && shape->d != 128) ||
       (shape->dtype == SVG_FP32 && shape->d != 32 && shape->d != 64 && shape->d != 128))
@@ -95,6 +97,7 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
   const int a1c = a1 < shape->N ? a1 : shape->N;
   const int a2c = a2 < shape->F ? a2 : shape->F;
   // the same kernels as svg_profile_heads, on the static scratch
-  return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, scale, q, k, v, a1c, a2c,
+  return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, scale, q, k, v,
+                        shape_strides(shape), a1c, a2c,
                         rows, S, mse, label, scratch, lay, nullptr, static_cast<cudaStream_t>(stream));
 }

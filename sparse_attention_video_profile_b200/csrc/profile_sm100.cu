@@ -31,8 +31,9 @@
 namespace svg {
 
 struct ProfSm100Params {
-  CUtensorMap tm_k, tm_v;  // frame-major [BH, L, D] bf16
-  const __nv_bfloat16* q;
+  CUtensorMap tm_k, tm_v;  // frame-major, laid out as hs
+  const __nv_bfloat16* q;  // laid out as hs
+  HeadStrides hs;
   const int32_t* rows;
   float* ws_o;   // [BH][nch][3][128][D]
   float* ws_ml;  // [BH][nch][3][128][2]  (max in log2 units, sum)
@@ -216,6 +217,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     // ------------------------------------------------ TMA producer (K, V)
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
+    const int th = p.hs.tma_h(bh), tb = p.hs.tma_b(bh);
     for (int n = 0; n < 2 * nk; ++n) {
       const int slot = n % C::NS;
       if (!mbar_wait(&bar_empty[slot], ((n / C::NS) & 1) ^ 1, p.wait_ns)) {
@@ -228,8 +230,8 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
       for (int h = 0; h < C::HALVES; ++h)
-        tma_load_3d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64,
-                    (kt0 + (n >> 1)) * 128, bh);
+        tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64,
+                    (kt0 + (n >> 1)) * 128, th, tb);
     }
   } else if (run && warp == 9) {
     // ------------------------------------------------ MMA issuer
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     const int x = min(max(p.rows[min(r, p.S - 1)], 0), p.L - 1);
     if (h == 0) {
       // gather Q row x into the 128-byte-swizzled K-major tile layout
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.L + x) * D);
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + p.hs.head(bh) + x * p.hs.sl);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
         const uint4 val = __ldg(src + c);
@@ -545,15 +547,12 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
 
 }  // namespace
 
-// [BH, L, D] bf16 tensor map with 64 x 128 x 1 boxes (defined in attn_sm100.cu).
-svg_status make_tile_map_bf16(CUtensorMap* map, const void* base, int BH, int L, int D);
-
 template <int D>
 svg_status launch_profile_sm100_d(ProfSm100Params& p, const void* k, const void* v, cudaStream_t stream) {
   using C = PCfg<D>;
   svg_status st;
-  if ((st = make_tile_map_bf16(&p.tm_k, k, p.BH, p.L, D)) != SVG_OK) return st;
-  if ((st = make_tile_map_bf16(&p.tm_v, v, p.BH, p.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_k, k, p.hs, p.L, D)) != SVG_OK) return st;
+  if ((st = make_tile_map_bf16(&p.tm_v, v, p.hs, p.L, D)) != SVG_OK) return st;
   cudaError_t e = cudaFuncSetAttribute(profile_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_check(e, "cudaFuncSetAttribute(profile smem)");
@@ -562,11 +561,12 @@ svg_status launch_profile_sm100_d(ProfSm100Params& p, const void* k, const void*
 }
 
 svg_status launch_profile_sm100(int BH, int N, int F, int d, float scale, const void* q, const void* k,
-                                const void* v, const int (&kind)[2], const int (&par)[2], const int32_t* rows, int S,
+                                const void* v, const HeadStrides& hs, const int (&kind)[2], const int (&par)[2], const int32_t* rows, int S,
                                 float* ws_o, float* ws_ml, int nch, int chunk, int* status, cudaStream_t stream) {
   ProfSm100Params p;
   memset(&p, 0, sizeof(p));
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.hs = hs;
   p.rows = rows;
   p.ws_o = ws_o;
   p.ws_ml = ws_ml;

@@ -112,16 +112,17 @@ __global__ void __launch_bounds__(32) svg2_scatter_kernel(const int32_t* __restr
   }
 }
 
-// Row gather: dst[bh][r] = src[bh][perm[bh][r]], rows of `rc` 16-byte chunks.
-__global__ void __launch_bounds__(256) svg2_gather_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm,
-                                                          uint4* __restrict__ dst, int L, int rc, long long total) {
+// Row gather: dst[bh][r] = src[bh][perm[bh][r]], rows of `rc` 16-byte chunks;
+// dst is [BH, L, rc], src laid out as ss (strides in chunks).
+__global__ void __launch_bounds__(256) svg2_gather_kernel(const uint4* __restrict__ src, const HeadStrides ss,
+                                                          const int32_t* __restrict__ perm, uint4* __restrict__ dst,
+                                                          int L, int rc, long long total) {
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long row = e / rc;  // bh * L + r
     const int c = static_cast<int>(e - row * rc);
-    const long long bh = row / L;
-    const long long srow = bh * L + perm[row];
-    __stcs(dst + e, __ldg(src + srow * rc + c));
+    const int bh = static_cast<int>(row / L);
+    __stcs(dst + e, __ldg(src + ss.head(bh) + perm[row] * ss.sl + c));
   }
 }
 
@@ -273,13 +274,18 @@ svg_status svg2_sort(const int32_t* assign, int BH, int L, int C, int nblk, int3
   return cuda_check(cudaGetLastError(), "cluster sort launch");
 }
 
-svg_status svg2_gather(const void* src, const int32_t* perm, void* dst, int BH, int L, int d, cudaStream_t stream) {
+svg_status svg2_gather(const void* src, const HeadStrides& ss, const int32_t* perm, void* dst, int BH, int L, int d,
+                       cudaStream_t stream) {
   const int rc = d * 2 / 16;
+  HeadStrides sc = ss;  // element strides -> 16-byte chunks (multiples of d)
+  sc.sb /= 8;
+  sc.sh /= 8;
+  sc.sl /= 8;
   const long long total = static_cast<long long>(BH) * L * rc;
   const long long blocks = (total + 255) / 256;
   const unsigned grid = static_cast<unsigned>(blocks < 148LL * 64 ? blocks : 148LL * 64);
-  svg2_gather_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(src), perm, static_cast<uint4*>(dst), L, rc,
-                                               total);
+  svg2_gather_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(src), sc, perm, static_cast<uint4*>(dst), L,
+                                               rc, total);
   return cuda_check(cudaGetLastError(), "cluster gather launch");
 }
 

@@ -41,6 +41,8 @@ svg_status check_shape(const svg_shape* s) {
   if (static_cast<long long>(s->N) * s->F > (1LL << 30))
     return fail(SVG_ERR_INVALID_ARG, "L = N*F = %lld is too large", static_cast<long long>(s->N) * s->F);
   if (s->dtype != SVG_BF16 && s->dtype != SVG_FP32) return fail(SVG_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+  if (s->layout != SVG_LAYOUT_BHLD && s->layout != SVG_LAYOUT_BLHD)
+    return fail(SVG_ERR_INVALID_ARG, "unknown layout %d", s->layout);
   if (!(s->scale >= 0.f) || isinf(s->scale)) return fail(SVG_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (s->dtype == SVG_BF16 && s->d != 64 && s->d != 128)
     return fail(SVG_ERR_UNSUPPORTED, "bf16 supports d in {64, 128}, got %d", s->d);
@@ -67,6 +69,30 @@ int clamp_band(int a, int G, int L) {
 }
 
 }  // namespace
+
+HeadStrides dense_strides(int B, int H, int L, int d) {
+  HeadStrides s;
+  s.H = H;
+  s.nb = B;
+  s.bh0 = 0;
+  s.sl = d;
+  s.sh = static_cast<long long>(L) * d;
+  s.sb = static_cast<long long>(H) * L * d;
+  return s;
+}
+
+HeadStrides shape_strides(const svg_shape* sh) {
+  const int L = sh->N * sh->F;
+  if (sh->layout != SVG_LAYOUT_BLHD) return dense_strides(sh->B, sh->H, L, sh->d);
+  HeadStrides s;
+  s.H = sh->H;
+  s.nb = sh->B;
+  s.bh0 = 0;
+  s.sl = static_cast<long long>(sh->H) * sh->d;
+  s.sh = sh->d;
+  s.sb = static_cast<long long>(L) * sh->H * sh->d;
+  return s;
+}
 
 // The whole bf16 call folds the layout transformation into attention when
 // that costs at most 3 % more attention work than the token-major copies.
@@ -99,8 +125,12 @@ svg_status internal_status_word(int** out, cudaStream_t stream) {
 
 namespace {
 
-svg_status run_attention(const svg_shape* s, BandAttnArgs& a, int32_t* status_dev, cudaStream_t stream,
-                         uint64_t wait_ns = kDefaultWaitNs) {
+// hs: layout of q, k, v, o; hsp: of the token-major (or, SVG2, cluster-
+// permuted) copies.
+svg_status run_attention(const svg_shape* s, const HeadStrides& hs, const HeadStrides& hsp, BandAttnArgs& a,
+                         int32_t* status_dev, cudaStream_t stream, uint64_t wait_ns = kDefaultWaitNs) {
+  a.hs = hs;
+  a.hsp = hsp;
   a.B = s->B;
   a.H = s->H;
   a.L = s->N * s->F;
@@ -210,17 +240,20 @@ size_t svg_workspace_size(const svg_shape* shape, int32_t n_temporal_heads_max) 
 svg_status svg_profile_heads(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
                              size_t workspace_bytes, void* stream) {
-  return profile_heads_impl(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, nullptr,
-                            static_cast<cudaStream_t>(stream));
+  svg_status st = check_shape(shape);
+  if (st != SVG_OK) return st;
+  return profile_heads_impl(shape, shape_strides(shape), q, k, v, a1, a2, rows, S, mse, label, workspace,
+                            workspace_bytes, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
 
 namespace svg {
 
-svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void* k, const void* v, int32_t a1,
-                              int32_t a2, const int32_t* rows, int32_t S, float* mse, int8_t* label, void* workspace,
-                              size_t workspace_bytes, int32_t* status_out, cudaStream_t stream, int chunk_len) {
+svg_status profile_heads_impl(const svg_shape* shape, const HeadStrides& hs, const void* q, const void* k,
+                              const void* v, int32_t a1, int32_t a2, const int32_t* rows, int32_t S, float* mse,
+                              int8_t* label, void* workspace, size_t workspace_bytes, int32_t* status_out,
+                              cudaStream_t stream, int chunk_len) {
   svg_status st = check_shape(shape);
   if (st != SVG_OK) return st;
   if ((st = check_tensors({q, k, v})) != SVG_OK) return st;
@@ -234,10 +267,63 @@ svg_status profile_heads_impl(const svg_shape* shape, const void* q, const void*
   profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay, 0, chunk_len);
   if (workspace_bytes < lay.total)
     return fail(SVG_ERR_WORKSPACE, "profile workspace %zu bytes < %zu required", workspace_bytes, lay.total);
-  return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, eff_scale(shape), q, k, v,
+  return launch_profile(shape->B, shape->H, shape->N, shape->F, shape->d, shape->dtype, eff_scale(shape), q, k, v, hs,
                         clamp_band(a1, 1, shape->N), clamp_band(a2, 1, shape->F), rows, S, mse, label, workspace, lay,
                         status_out, stream);
 }
+
+namespace {
+
+// The layout transformation of up to three tensors, src laid out as ss and
+// dst as ds; only heads whose label equals sel move (every head when label is
+// NULL).
+svg_status permute_impl(const svg_shape* s, int n, const void* const* src, void* const* dst, const HeadStrides& ss,
+                        const HeadStrides& ds, const int8_t* label, bool to_token_major, cudaStream_t stream,
+                        int sel = SVG_TEMPORAL) {
+  return launch_permute(n, src, dst, s->B * s->H, s->N, s->F, s->d, static_cast<int>(elem_size(s->dtype)), ss, ds,
+                        label, to_token_major, stream, sel);
+}
+
+// Block-sparse attention of labelled heads: spatial heads on (q, k, v) -> o
+// laid out as hs, temporal heads on the token-major copies (qp, kp, vp) -> op
+// laid out as hsp, or with fused != 0 temporal heads straight from (q, k, v)
+// into o.
+svg_status block_sparse_impl(const svg_shape* shape, const HeadStrides& hs, const HeadStrides& hsp, const void* q,
+                             const void* k, const void* v, const void* qp, const void* kp, const void* vp, void* o,
+                             void* op, const int8_t* label, int32_t a1, int32_t a2, int fused, int32_t* status_dev,
+                             cudaStream_t stream) {
+  const int L = shape->N * shape->F;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  if (!fused) {
+    a.qp = qp;
+    a.kp = kp;
+    a.vp = vp;
+    a.op = op;
+  }
+  a.label = label;
+  a.G0 = shape->F;
+  a.a0 = clamp_band(a1, shape->F, L);
+  a.G1 = shape->N;
+  a.a1 = clamp_band(a2, shape->N, L);
+  if (fused) {
+    a.N = shape->N;
+    a.fused = 1;
+  }
+  return run_attention(shape, hs, hsp, a, status_dev, stream);
+}
+
+// The whole call on `shape`'s heads, q, k, v, o laid out as hs (the
+// token-major copies in the workspace are contiguous [B, H, L, d]).
+svg_status sparse_3d_attn_impl(const svg_shape* shape, const HeadStrides& hs, const void* q, const void* k,
+                               const void* v, void* o, int32_t a1, int32_t a2, const int32_t* rows, int32_t S,
+                               float* mse, int8_t* label, void* workspace, size_t workspace_bytes,
+                               int32_t* status_dev, cudaStream_t stream);
+
+}  // namespace
 
 }  // namespace svg
 
@@ -250,9 +336,8 @@ svg_status svg_permute(const svg_shape* shape, const void* x, void* xp, const in
   if (x == xp) return fail(SVG_ERR_INVALID_ARG, "permute cannot run in place");
   const void* src[1] = {x};
   void* dst[1] = {xp};
-  return launch_permute(1, src, dst, shape->B * shape->H, shape->N, shape->F,
-                        static_cast<int>(shape->d * elem_size(shape->dtype)), label, true,
-                        static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return permute_impl(shape, 1, src, dst, hs, hs, label, true, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_permute_qkv(const svg_shape* shape, const void* q, const void* k, const void* v, void* qp, void* kp,
@@ -263,9 +348,8 @@ svg_status svg_permute_qkv(const svg_shape* shape, const void* q, const void* k,
   if (q == qp || k == kp || v == vp) return fail(SVG_ERR_INVALID_ARG, "permute cannot run in place");
   const void* src[3] = {q, k, v};
   void* dst[3] = {qp, kp, vp};
-  return launch_permute(3, src, dst, shape->B * shape->H, shape->N, shape->F,
-                        static_cast<int>(shape->d * elem_size(shape->dtype)), label, true,
-                        static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return permute_impl(shape, 3, src, dst, hs, hs, label, true, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_unpermute(const svg_shape* shape, const void* xp, void* x, const int8_t* label, void* stream) {
@@ -275,9 +359,8 @@ svg_status svg_unpermute(const svg_shape* shape, const void* xp, void* x, const 
   if (x == xp) return fail(SVG_ERR_INVALID_ARG, "unpermute cannot run in place");
   const void* src[1] = {xp};
   void* dst[1] = {x};
-  return launch_permute(1, src, dst, shape->B * shape->H, shape->N, shape->F,
-                        static_cast<int>(shape->d * elem_size(shape->dtype)), label, false,
-                        static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return permute_impl(shape, 1, src, dst, hs, hs, label, false, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_block_sparse_attn(const svg_shape* shape, const void* q, const void* k, const void* v, const void* qp,
@@ -288,22 +371,9 @@ svg_status svg_block_sparse_attn(const svg_shape* shape, const void* q, const vo
   if ((st = check_tensors({q, k, v, o, qp, kp, vp, op})) != SVG_OK) return st;
   if (label == nullptr) return fail(SVG_ERR_INVALID_ARG, "label is NULL");
   if (a1 < 1 || a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a1 and a2 must be >= 1");
-  const int L = shape->N * shape->F;
-  BandAttnArgs a{};
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.o = o;
-  a.qp = qp;
-  a.kp = kp;
-  a.vp = vp;
-  a.op = op;
-  a.label = label;
-  a.G0 = shape->F;
-  a.a0 = clamp_band(a1, shape->F, L);
-  a.G1 = shape->N;
-  a.a1 = clamp_band(a2, shape->N, L);
-  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return block_sparse_impl(shape, hs, hs, q, k, v, qp, kp, vp, o, op, label, a1, a2, 0, status_dev,
+                           static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_block_sparse_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
@@ -314,20 +384,9 @@ svg_status svg_block_sparse_attn_fused(const svg_shape* shape, const void* q, co
   if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
   if (label == nullptr) return fail(SVG_ERR_INVALID_ARG, "label is NULL");
   if (a1 < 1 || a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a1 and a2 must be >= 1");
-  const int L = shape->N * shape->F;
-  BandAttnArgs a{};
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.o = o;
-  a.label = label;
-  a.G0 = shape->F;
-  a.a0 = clamp_band(a1, shape->F, L);
-  a.G1 = shape->N;
-  a.a1 = clamp_band(a2, shape->N, L);
-  a.N = shape->N;
-  a.fused = 1;
-  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return block_sparse_impl(shape, hs, hs, q, k, v, nullptr, nullptr, nullptr, o, nullptr, label, a1, a2, 1, status_dev,
+                           static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_banded_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o, int32_t G,
@@ -348,7 +407,8 @@ svg_status svg_banded_attn(const svg_shape* shape, const void* q, const void* k,
   a.a0 = clamp_band(a_band, G, L);
   a.G1 = a.G0;
   a.a1 = a.a0;
-  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return run_attention(shape, hs, hs, a, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_dense_attn(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
@@ -387,33 +447,61 @@ svg_status svg_sparse_3d_attn(const svg_shape* shape, const void* q, const void*
                               size_t workspace_bytes, int32_t* status_dev, void* stream) {
   svg_status st = check_shape(shape);
   if (st != SVG_OK) return st;
+  return sparse_3d_attn_impl(shape, shape_strides(shape), q, k, v, o, a1, a2, rows, S, mse, label, workspace,
+                             workspace_bytes, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace svg {
+namespace {
+
+svg_status sparse_3d_attn_impl(const svg_shape* shape, const HeadStrides& hs, const void* q, const void* k,
+                               const void* v, void* o, int32_t a1, int32_t a2, const int32_t* rows, int32_t S,
+                               float* mse, int8_t* label, void* workspace, size_t workspace_bytes,
+                               int32_t* status_dev, cudaStream_t stream) {
+  svg_status st;
   if ((st = check_tensors({q, k, v, o})) != SVG_OK) return st;
   if (!workspace) return fail(SVG_ERR_INVALID_ARG, "workspace is NULL");
+  if (a1 < 1 || a2 < 1) return fail(SVG_ERR_INVALID_ARG, "a1 and a2 must be >= 1");
   const size_t need = svg_sparse_3d_attn_workspace_size(shape, a2, S);
   if (need == 0) return fail(SVG_ERR_INVALID_ARG, "S must be in [1, 128] and a2 >= 1");
   if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if (whole_call_fused(shape, a2)) {
-    if ((st = profile_heads_impl(shape, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes, status_dev,
-                                 static_cast<cudaStream_t>(stream))) != SVG_OK)
+    if ((st = profile_heads_impl(shape, hs, q, k, v, a1, a2, rows, S, mse, label, workspace, workspace_bytes,
+                                 status_dev, stream)) != SVG_OK)
       return st;
-    return svg_block_sparse_attn_fused(shape, q, k, v, o, label, a1, a2, status_dev, stream);
+    return block_sparse_impl(shape, hs, hs, q, k, v, nullptr, nullptr, nullptr, o, nullptr, label, a1, a2, 1,
+                             status_dev, stream);
   }
-  const size_t t = static_cast<size_t>(shape->B) * shape->H * shape->N * shape->F * shape->d * elem_size(shape->dtype);
+  const int L = shape->N * shape->F;
+  const size_t t = static_cast<size_t>(shape->B) * shape->H * L * shape->d * elem_size(shape->dtype);
   const size_t t_al = (t + 255) / 256 * 256;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   void *qp = w, *kp = w + t_al, *vp = w + 2 * t_al, *op = w + 3 * t_al;
   void* prof_ws = w + 4 * t_al;
   const size_t prof_bytes = workspace_bytes - 4 * t_al;
-  if ((st = profile_heads_impl(shape, q, k, v, a1, a2, rows, S, mse, label, prof_ws, prof_bytes, status_dev,
-                               static_cast<cudaStream_t>(stream))) != SVG_OK)
+  const HeadStrides ws = dense_strides(shape->B, shape->H, L, shape->d);  // the token-major copies
+  if ((st = profile_heads_impl(shape, hs, q, k, v, a1, a2, rows, S, mse, label, prof_ws, prof_bytes, status_dev,
+                               stream)) != SVG_OK)
     return st;
-  if ((st = svg_permute_qkv(shape, q, k, v, qp, kp, vp, label, stream)) != SVG_OK) return st;
-  if ((st = svg_block_sparse_attn(shape, q, k, v, qp, kp, vp, o, op, label, a1, a2, status_dev, stream)) != SVG_OK)
+  const void* src3[3] = {q, k, v};
+  void* dst3[3] = {qp, kp, vp};
+  if ((st = permute_impl(shape, 3, src3, dst3, hs, ws, label, true, stream)) != SVG_OK) return st;
+  if ((st = block_sparse_impl(shape, hs, ws, q, k, v, qp, kp, vp, o, op, label, a1, a2, 0, status_dev, stream)) !=
+      SVG_OK)
     return st;
-  return svg_unpermute(shape, op, o, label, stream);
+  const void* src1[1] = {op};
+  void* dst1[1] = {o};
+  return permute_impl(shape, 1, src1, dst1, ws, hs, label, false, stream);
 }
+
+}  // namespace
+}  // namespace svg
+
+extern "C" {
 
 svg_status svg_head_shard(int32_t n_heads, int32_t rank, int32_t world, int32_t* first, int32_t* count) {
   if (first == nullptr || count == nullptr) return fail(SVG_ERR_INVALID_ARG, "NULL output");
@@ -450,17 +538,16 @@ svg_status svg_sparse_3d_attn_shard(const svg_shape* shape, int32_t rank, int32_
   if (!mse || !label) return fail(SVG_ERR_INVALID_ARG, "NULL mse/label");
   if (count == 0) return SVG_OK;  // more ranks than heads: this rank has none
   // heads are flattened over (b, h): this rank's heads are one contiguous
-  // block of every [B, H, ...] array, so the shard is the whole call on that
-  // block
+  // block of the [B, H] arrays (mse, label), and heads first .. first +
+  // count - 1 of q, k, v, o in either layout, so the shard is the whole call
+  // on that block
   svg_shape local = *shape;
   local.B = 1;
   local.H = count;
-  const size_t head_bytes = static_cast<size_t>(shape->N) * shape->F * shape->d * elem_size(shape->dtype);
-  const size_t off = static_cast<size_t>(first) * head_bytes;
-  auto at = [off](const void* p) { return static_cast<const uint8_t*>(p) + off; };
-  return svg_sparse_3d_attn(&local, at(q), at(k), at(v), static_cast<uint8_t*>(o) + off, a1, a2, rows, S,
-                            mse + 2 * static_cast<size_t>(first), label + first, workspace, workspace_bytes,
-                            status_dev, stream);
+  HeadStrides hs = shape_strides(shape);
+  hs.bh0 = first;
+  return sparse_3d_attn_impl(&local, hs, q, k, v, o, a1, a2, rows, S, mse + 2 * static_cast<size_t>(first),
+                             label + first, workspace, workspace_bytes, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_mixed_attn(const svg_shape* shape, const void* q, const void* k, const void* v, const void* qp,
@@ -491,7 +578,8 @@ svg_status svg_mixed_attn(const svg_shape* shape, const void* q, const void* k, 
   a.N = shape->N;
   a.md_a = clamp_band(md_half + 1, shape->N, L);
   a.stripe = stripe < L ? stripe : L;
-  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return run_attention(shape, hs, hs, a, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_mixed_attn_fused(const svg_shape* shape, const void* q, const void* k, const void* v, void* o,
@@ -519,7 +607,8 @@ svg_status svg_mixed_attn_fused(const svg_shape* shape, const void* q, const voi
   a.md_a = clamp_band(md_half + 1, shape->N, L);
   a.stripe = stripe < L ? stripe : L;
   a.fused = 1;
-  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream));
+  const HeadStrides hs = shape_strides(shape);
+  return run_attention(shape, hs, hs, a, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 size_t svg_mixed_3d_attn_workspace_size(const svg_shape* shape) {
@@ -539,22 +628,39 @@ svg_status svg_mixed_3d_attn(const svg_shape* shape, const void* q, const void* 
   if (workspace_bytes < need) return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(SVG_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (window < 0 || md_half < 0 || stripe < 1) return fail(SVG_ERR_INVALID_ARG, "window, md_half >= 0 and stripe >= 1");
+  if (shape->dtype != SVG_BF16) return fail(SVG_ERR_UNSUPPORTED, "mixed-pattern attention runs in bf16 only");
   const size_t t_al = need / 4;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   void *qp = w, *kp = w + t_al, *vp = w + 2 * t_al, *op = w + 3 * t_al;
-  const int BH = shape->B * shape->H;
-  const int rb = static_cast<int>(shape->d * elem_size(shape->dtype));
+  const int L = shape->N * shape->F;
+  const HeadStrides hs = shape_strides(shape), ws = dense_strides(shape->B, shape->H, L, shape->d);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const void* src3[3] = {q, k, v};
   void* dst3[3] = {qp, kp, vp};
-  if ((st = launch_permute(3, src3, dst3, BH, shape->N, shape->F, rb, mode, true, s, SVG_MODE_MULTIDIAG)) != SVG_OK)
-    return st;
-  if ((st = svg_mixed_attn(shape, q, k, v, qp, kp, vp, o, op, mode, window, md_half, stripe, status_dev, stream)) !=
-      SVG_OK)
-    return st;
+  if ((st = permute_impl(shape, 3, src3, dst3, hs, ws, mode, true, s, SVG_MODE_MULTIDIAG)) != SVG_OK) return st;
+  BandAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.qp = qp;
+  a.kp = kp;
+  a.vp = vp;
+  a.op = op;
+  a.modes = mode;
+  a.G0 = L;
+  a.a0 = 1;
+  a.G1 = L;
+  a.a1 = 1;
+  a.win = window < L ? window : L;
+  a.N = shape->N;
+  a.md_a = clamp_band(md_half + 1, shape->N, L);
+  a.stripe = stripe < L ? stripe : L;
+  if ((st = run_attention(shape, hs, ws, a, status_dev, s)) != SVG_OK) return st;
   const void* src1[1] = {op};
   void* dst1[1] = {o};
-  return launch_permute(1, src1, dst1, BH, shape->N, shape->F, rb, mode, false, s, SVG_MODE_MULTIDIAG);
+  return permute_impl(shape, 1, src1, dst1, ws, hs, mode, false, s, SVG_MODE_MULTIDIAG);
 }
 
 size_t svg_semantic_attn_workspace_size(const svg_shape* shape, int32_t Cq, int32_t Ck) {
@@ -604,9 +710,10 @@ svg_status svg_semantic_attn(const svg_shape* shape, const void* q, const void* 
   if ((st = status_word(status_dev, &dev_status, s)) != SVG_OK) return st;
   if ((st = svg2_sort(assign_q, BH, L, Cq, z.nblk, hist, perm_q, cid_q, off_q, dev_status, s)) != SVG_OK) return st;
   if ((st = svg2_sort(assign_k, BH, L, Ck, z.nblk, hist, perm_k, cid_k, off_k, dev_status, s)) != SVG_OK) return st;
-  if ((st = svg2_gather(q, perm_q, qp, BH, L, d, s)) != SVG_OK) return st;
-  if ((st = svg2_gather(k, perm_k, kp, BH, L, d, s)) != SVG_OK) return st;
-  if ((st = svg2_gather(v, perm_k, vp, BH, L, d, s)) != SVG_OK) return st;
+  const HeadStrides hs = shape_strides(shape), ws = dense_strides(shape->B, shape->H, L, d);
+  if ((st = svg2_gather(q, hs, perm_q, qp, BH, L, d, s)) != SVG_OK) return st;
+  if ((st = svg2_gather(k, hs, perm_k, kp, BH, L, d, s)) != SVG_OK) return st;
+  if ((st = svg2_gather(v, hs, perm_k, vp, BH, L, d, s)) != SVG_OK) return st;
   if ((st = svg2_centroids(qp, off_q, BH, L, Cq, d, mu_q, s)) != SVG_OK) return st;
   if ((st = svg2_centroids(kp, off_k, BH, L, Ck, d, mu_k, s)) != SVG_OK) return st;
   if ((st = svg2_topp(mu_q, mu_k, off_k, BH, Cq, Ck, d, eff_scale(shape), p, selected, s)) != SVG_OK) return st;
@@ -626,7 +733,7 @@ svg_status svg_semantic_attn(const svg_shape* shape, const void* q, const void* 
   a.s2_perm = perm_q;
   a.s2_koff = off_k;
   a.s2_sel = selected;
-  return run_attention(shape, a, dev_status, s);
+  return run_attention(shape, hs, ws, a, dev_status, s);
 }
 
 size_t svg_kmeans_workspace_size(const svg_shape* shape, int32_t C) {
@@ -652,7 +759,8 @@ svg_status svg_kmeans(const svg_shape* shape, const void* x, int32_t C, int32_t 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* dev_status = nullptr;
   if ((st = status_word(status_dev, &dev_status, s)) != SVG_OK) return st;
-  return launch_kmeans(x, shape->B * shape->H, L, C, shape->d, iters, assign, centroids, workspace, dev_status, s);
+  return launch_kmeans(x, shape_strides(shape), shape->B * shape->H, L, C, shape->d, iters, assign, centroids, workspace,
+                       dev_status, s);
 }
 
 size_t svg_semantic_3d_attn_workspace_size(const svg_shape* shape, int32_t Cq, int32_t Ck) {
@@ -714,7 +822,8 @@ svg_status svg_mode_search(const svg_shape* shape, const void* q, const void* k,
   if (workspace_bytes < lay.total + lay.part_bytes)
     return fail(SVG_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, lay.total + lay.part_bytes);
   double* part2 = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + lay.total);
-  return launch_mode_search(shape->B, shape->H, shape->N, shape->F, shape->d, eff_scale(shape), q, k, v, rows, S,
+  return launch_mode_search(shape->B, shape->H, shape->N, shape->F, shape->d, eff_scale(shape), q, k, v,
+                            shape_strides(shape), rows, S,
                             window < L ? window : L, md_half < shape->F ? md_half : shape->F, stripe < L ? stripe : L,
                             lambda, epsilon, loss, mode, workspace, lay, part2, static_cast<cudaStream_t>(stream));
 }
@@ -740,7 +849,8 @@ svg_status svg_selftest_wait_bound(const svg_shape* shape, const void* q, const 
   a.G1 = L;
   a.a1 = 1;
   a.withhold_loads = 1;
-  return run_attention(shape, a, status_dev, static_cast<cudaStream_t>(stream), wait_ns);
+  const HeadStrides hs = shape_strides(shape);
+  return run_attention(shape, hs, hs, a, status_dev, static_cast<cudaStream_t>(stream), wait_ns);
 }
 
 }  // extern "C"

@@ -6,10 +6,10 @@ are allocated with torch when the caller does not pass them) and the current
 CUDA stream.  Importing this module raises ImportError if libsvg.so has not
 been built -- there is no fallback path.
 
-Function names match the C entry points.  Tensors are contiguous
-[B, H, L, d] CUDA tensors (bf16 or fp32) with L = N * F in frame-major order
-(token (i, j) at row i*F + j); labels are int8 [B, H] with 0 = spatial and
-1 = temporal.
+Function names match the C entry points.  Tensors are contiguous CUDA
+tensors (bf16 or fp32), [B, H, L, d] by default or [B, L, H, d] with
+layout="blhd", with L = N * F in frame-major order (token (i, j) at row
+i*F + j); labels are int8 [B, H] with 0 = spatial and 1 = temporal.
 """
 from __future__ import annotations
 
@@ -32,6 +32,9 @@ TEMPORAL = 1
 SVG_DEV_TIMEOUT = 0x1
 SVG_DEV_RANGE = 0x2
 SVG_DEV_BOUNDS = 0x4
+SVG_LAYOUT_BHLD = 0
+SVG_LAYOUT_BLHD = 1
+LAYOUTS = {"bhld": SVG_LAYOUT_BHLD, "blhd": SVG_LAYOUT_BLHD}
 
 # Every symbol include/svg.h declares.
 EXPORTED = (
@@ -59,7 +62,8 @@ class SvgError(RuntimeError):
 
 class svg_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("F", ctypes.c_int32),
-                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("layout", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -137,13 +141,20 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
 
 
-def make_shape(x: torch.Tensor, N: int, F: int, scale: float = 0.0) -> svg_shape:
+def make_shape(x: torch.Tensor, N: int, F: int, scale: float = 0.0, layout: str = "bhld") -> svg_shape:
+    """The svg_shape of a q/k/v tensor: [B, H, L, d] (layout "bhld") or
+    [B, L, H, d] ("blhd")."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}, got {layout!r}")
     if x.dim() != 4:
-        raise ValueError("expected a [B, H, L, d] tensor")
-    B, H, L, d = x.shape
+        raise ValueError(f"expected a [B, H, L, d] or [B, L, H, d] tensor, got {x.dim()} dims")
+    if layout == "bhld":
+        B, H, L, d = x.shape
+    else:
+        B, L, H, d = x.shape
     if L != N * F:
         raise ValueError(f"L = {L} but N*F = {N * F}")
-    return svg_shape(B, H, N, F, d, _dtype_code(x), float(scale))
+    return svg_shape(B, H, N, F, d, _dtype_code(x), float(scale), LAYOUTS[layout])
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -213,10 +224,10 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 # ------------------------------------------------------------------ device calls
 
 def svg_profile_heads(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, mse=None, label=None,
-                      workspace=None, scale: float = 0.0, stream=None):
+                      workspace=None, scale: float = 0.0, layout: str = "bhld", stream=None):
     """Online profiling.  Returns (mse [B,H,2] f32, label [B,H] int8) on q's device."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if rows.dtype != torch.int32 or rows.device != q.device:
         raise ValueError("rows must be an int32 tensor on q's device")
     S = rows.numel()
@@ -233,13 +244,13 @@ def svg_profile_heads(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Ten
 
 
 def svg_profile_heads_noalloc(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, mse=None,
-                              label=None, scale: float = 0.0, stream=None):
+                              label=None, scale: float = 0.0, layout: str = "bhld", stream=None):
     """Online profiling without a workspace, for callers that cannot allocate
     device memory.  The library's fixed scratch array stands in for the
     workspace (see include/svg.h).  mse and label should be passed in by
     such callers; they are allocated here only for convenience."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if rows.dtype != torch.int32 or rows.device != q.device:
         raise ValueError("rows must be an int32 tensor on q's device")
     if mse is None:
@@ -251,25 +262,26 @@ def svg_profile_heads_noalloc(q, k, v, N: int, F: int, a1: int, a2: int, rows: t
     return mse, label
 
 
-def svg_permute(x, N: int, F: int, label=None, *, out=None, stream=None):
-    shape = make_shape(x, N, F)
+def svg_permute(x, N: int, F: int, label=None, *, out=None, layout: str = "bhld", stream=None):
+    shape = make_shape(x, N, F, 0.0, layout)
     if out is None:
         out = torch.empty_like(x)
     _check(lib.svg_permute(ctypes.byref(shape), _ptr(x), _ptr(out), _ptr(label), _stream(stream)))
     return out
 
 
-def svg_permute_qkv(q, k, v, N: int, F: int, label=None, *, out: Optional[Sequence] = None, stream=None):
+def svg_permute_qkv(q, k, v, N: int, F: int, label=None, *, out: Optional[Sequence] = None, layout: str = "bhld",
+                    stream=None):
     _same(q, k, v)
-    shape = make_shape(q, N, F)
+    shape = make_shape(q, N, F, 0.0, layout)
     qp, kp, vp = out if out is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     _check(lib.svg_permute_qkv(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(qp), _ptr(kp), _ptr(vp),
                                _ptr(label), _stream(stream)))
     return qp, kp, vp
 
 
-def svg_unpermute(xp, N: int, F: int, label=None, *, out=None, stream=None):
-    shape = make_shape(xp, N, F)
+def svg_unpermute(xp, N: int, F: int, label=None, *, out=None, layout: str = "bhld", stream=None):
+    shape = make_shape(xp, N, F, 0.0, layout)
     if out is None:
         out = torch.empty_like(xp)
     _check(lib.svg_unpermute(ctypes.byref(shape), _ptr(xp), _ptr(out), _ptr(label), _stream(stream)))
@@ -277,10 +289,10 @@ def svg_unpermute(xp, N: int, F: int, label=None, *, out=None, stream=None):
 
 
 def svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N: int, F: int, a1: int, a2: int, *, o=None, op=None,
-                          status=None, scale: float = 0.0, stream=None):
+                          status=None, scale: float = 0.0, layout: str = "bhld", stream=None):
     """Returns (o, op): spatial heads' output in o, temporal heads' in op."""
     _same(q, k, v, qp, kp, vp)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     if op is None:
@@ -291,11 +303,11 @@ def svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N: int, F: int, a1: int, a
 
 
 def svg_block_sparse_attn_fused(q, k, v, label, N: int, F: int, a1: int, a2: int, *, o=None, status=None,
-                                scale: float = 0.0, stream=None):
+                                scale: float = 0.0, layout: str = "bhld", stream=None):
     """Block-sparse attention with the layout transformation fused in: every
     head's output lands frame-major in o (no permuted copies).  bf16."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_block_sparse_attn_fused(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(label), a1,
@@ -304,9 +316,9 @@ def svg_block_sparse_attn_fused(q, k, v, label, N: int, F: int, a1: int, a2: int
 
 
 def svg_banded_attn(q, k, v, N: int, F: int, G: int, a: int, *, o=None, status=None, scale: float = 0.0,
-                    stream=None):
+                    layout: str = "bhld", stream=None):
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_banded_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), G, a, _ptr(status),
@@ -314,9 +326,10 @@ def svg_banded_attn(q, k, v, N: int, F: int, G: int, a: int, *, o=None, status=N
     return o
 
 
-def svg_dense_attn(q, k, v, N: int, F: int, *, o=None, status=None, scale: float = 0.0, stream=None):
+def svg_dense_attn(q, k, v, N: int, F: int, *, o=None, status=None, scale: float = 0.0, layout: str = "bhld",
+                   stream=None):
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_dense_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(status),
@@ -325,10 +338,11 @@ def svg_dense_attn(q, k, v, N: int, F: int, *, o=None, status=None, scale: float
 
 
 def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, o=None, mse=None,
-                       label=None, workspace=None, status=None, scale: float = 0.0, stream=None):
+                       label=None, workspace=None, status=None, scale: float = 0.0, layout: str = "bhld",
+                       stream=None):
     """One whole sparse 3D-attention call.  Returns (o, mse, label)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     S = rows.numel()
     if o is None:
         o = torch.empty_like(q)
@@ -371,15 +385,30 @@ def gather_heads(x: torch.Tensor, n_heads: int, rank: int, world: int, group=Non
     return x
 
 
+def gather_output(o: torch.Tensor, n_heads: int, rank: int, world: int, layout: str = "bhld",
+                  group=None) -> torch.Tensor:
+    """gather_heads for an attention output in either layout.  In
+    [B, L, H, d] a block of heads is not contiguous, so the blocks travel as
+    a [B, H, L, d] copy that is written back afterwards."""
+    if layout == "bhld":
+        return gather_heads(o, n_heads, rank, world, group)
+    if layout != "blhd":
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}, got {layout!r}")
+    oh = o.transpose(1, 2).contiguous()
+    gather_heads(oh, n_heads, rank, world, group)
+    o.copy_(oh.transpose(1, 2))
+    return o
+
+
 def svg_sparse_3d_attn_shard(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, rank: int, world: int, *,
                              o=None, mse=None, label=None, workspace=None, status=None, scale: float = 0.0,
-                             stream=None, gather: bool = False, group=None):
+                             layout: str = "bhld", stream=None, gather: bool = False, group=None):
     """This rank's block of heads of one whole call (q, k, v are the full
     tensors).  Returns (o, mse, label) full-size; only this rank's heads are
     written unless gather=True, which then fills the rest from the other
     ranks (torch.distributed must be initialised)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     S = rows.numel()
     if o is None:
         o = torch.empty_like(q)
@@ -395,16 +424,17 @@ def svg_sparse_3d_attn_shard(q, k, v, N: int, F: int, a1: int, a2: int, rows: to
                                         _ptr(status), _stream(stream)))
     if gather and world > 1:
         n = shape.B * shape.H
-        for t in (o, mse, label):
+        for t in (mse, label):
             gather_heads(t, n, rank, world, group)
+        gather_output(o, n, rank, world, layout, group)
     return o, mse, label
 
 
 def svg_mixed_attn_fused(q, k, v, mode, N: int, F: int, window: int, md_half: int, stripe: int, *, o=None,
-                         status=None, scale: float = 0.0, stream=None):
+                         status=None, scale: float = 0.0, layout: str = "bhld", stream=None):
     """Mixed-pattern attention with the multi-diagonal heads' layout fused in."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_mixed_attn_fused(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(mode), window,
@@ -413,10 +443,10 @@ def svg_mixed_attn_fused(q, k, v, mode, N: int, F: int, window: int, md_half: in
 
 
 def svg_mixed_attn(q, k, v, qp, kp, vp, mode, N: int, F: int, window: int, md_half: int, stripe: int, *,
-                   o=None, op=None, status=None, scale: float = 0.0, stream=None):
+                   o=None, op=None, status=None, scale: float = 0.0, layout: str = "bhld", stream=None):
     """Every head under its own mode (SVG_MODE_*), one launch.  Returns (o, op)."""
     _same(q, k, v, qp, kp, vp)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     if op is None:
@@ -428,10 +458,10 @@ def svg_mixed_attn(q, k, v, qp, kp, vp, mode, N: int, F: int, window: int, md_ha
 
 
 def svg_mixed_3d_attn(q, k, v, mode, N: int, F: int, window: int, md_half: int, stripe: int, *, o=None,
-                      workspace=None, status=None, scale: float = 0.0, stream=None):
+                      workspace=None, status=None, scale: float = 0.0, layout: str = "bhld", stream=None):
     """One mixed-pattern call (permutation of multi-diagonal heads included)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     if workspace is None:
@@ -471,11 +501,12 @@ def svg_sparse_3d_attn_host(q, k, v, N: int, F: int, a1: int, a2: int, rows, *, 
 
 
 def svg_mode_search(q, k, v, N: int, F: int, rows, window: int, md_half: int, stripe: int, *, lam: float = 0.5,
-                    epsilon: float = 1.0, loss=None, mode=None, workspace=None, scale: float = 0.0, stream=None):
+                    epsilon: float = 1.0, loss=None, mode=None, workspace=None, scale: float = 0.0,
+                    layout: str = "bhld", stream=None):
     """Sparse-vDiT mode selection per head.  Returns (loss [B,H,4]: skip,
     diagonal, multi-diagonal, stripe; mode [B,H] int8 SVG_MODE_*)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if loss is None:
         loss = torch.empty(shape.B, shape.H, 4, dtype=torch.float32, device=q.device)
     if mode is None:
@@ -490,11 +521,12 @@ def svg_mode_search(q, k, v, N: int, F: int, rows, window: int, md_half: int, st
 
 
 def svg_semantic_attn(q, k, v, N: int, F: int, assign_q, assign_k, Cq: int, Ck: int, p: float, *, o=None,
-                      selected=None, workspace=None, status=None, scale: float = 0.0, stream=None):
+                      selected=None, workspace=None, status=None, scale: float = 0.0, layout: str = "bhld",
+                      stream=None):
     """SVG2-style attention given the token clusters (int32 [B,H,L] each).
     Returns (o, selected [B,H,Cq,ceil(Ck/32)] uint32 bitmask as int32)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     if o is None:
         o = torch.empty_like(q)
     if selected is None:
@@ -508,9 +540,9 @@ def svg_semantic_attn(q, k, v, N: int, F: int, assign_q, assign_k, Cq: int, Ck: 
 
 
 def svg_kmeans(x, N: int, F: int, C: int, iters: int, *, assign=None, centroids=None, workspace=None, status=None,
-               stream=None):
+               layout: str = "bhld", stream=None):
     """k-means of every head's rows.  Returns (assign int32 [B,H,L], centroids float32 [B,H,C,d])."""
-    shape = make_shape(x, N, F, 0.0)
+    shape = make_shape(x, N, F, 0.0, layout)
     if assign is None:
         assign = torch.empty(shape.B, shape.H, N * F, dtype=torch.int32, device=x.device)
     if centroids is None:
@@ -523,11 +555,12 @@ def svg_kmeans(x, N: int, F: int, C: int, iters: int, *, assign=None, centroids=
 
 
 def svg_semantic_3d_attn(q, k, v, N: int, F: int, Cq: int, Ck: int, iters: int, p: float, *, o=None, assign_q=None,
-                         assign_k=None, selected=None, workspace=None, status=None, scale: float = 0.0, stream=None):
+                         assign_k=None, selected=None, workspace=None, status=None, scale: float = 0.0,
+                         layout: str = "bhld", stream=None):
     """The whole SVG2-style call (k-means of Q and K, top-p, attention).
     Returns (o, assign_q, assign_k, selected)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, layout)
     L = N * F
     if o is None:
         o = torch.empty_like(q)
@@ -555,10 +588,10 @@ def selected_bits(selected, Ck: int):
 
 
 def svg_selftest_wait_bound(q, k, v, N: int, F: int, status, *, wait_ns: int = 50_000_000, o=None,
-                            stream=None):
+                            layout: str = "bhld", stream=None):
     """Failure-detection self-test: the attention kernel with its loads
     withheld must time out, set SVG_DEV_TIMEOUT in `status` and exit."""
-    shape = make_shape(q, N, F)
+    shape = make_shape(q, N, F, 0.0, layout)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_selftest_wait_bound(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), int(wait_ns),
@@ -571,14 +604,15 @@ class SparseAttention3D:
     workspace between calls (svg_sparse_3d_attn: profiling, then attention
     with the layout transformation fused in or as separate passes)."""
 
-    def __init__(self, N: int, F: int, a1: int, a2: int, scale: float = 0.0):
-        self.N, self.F, self.a1, self.a2, self.scale = N, F, a1, a2, scale
+    def __init__(self, N: int, F: int, a1: int, a2: int, scale: float = 0.0, layout: str = "bhld"):
+        self.N, self.F, self.a1, self.a2, self.scale, self.layout = N, F, a1, a2, scale, layout
         self._ws = None
 
     def __call__(self, q, k, v, rows, *, o=None, mse=None, label=None, status=None, stream=None):
-        shape = make_shape(q, self.N, self.F, self.scale)
+        shape = make_shape(q, self.N, self.F, self.scale, self.layout)
         need = svg_sparse_3d_attn_workspace_size(shape, self.a2, rows.numel())
         if self._ws is None or self._ws.numel() < need or self._ws.device != q.device:
             self._ws = alloc_workspace(need, q.device)
         return svg_sparse_3d_attn(q, k, v, self.N, self.F, self.a1, self.a2, rows, o=o, mse=mse, label=label,
-                                  workspace=self._ws, status=status, scale=self.scale, stream=stream)
+                                  workspace=self._ws, status=status, scale=self.scale, layout=self.layout,
+                                  stream=stream)

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert svg.svg_abi_version() == 1
+    assert svg.svg_abi_version() == 2
     assert svg.lib.svg_status_string(0) == b"SVG_OK"
     assert svg.lib.svg_status_string(5) == b"SVG_ERR_WORKSPACE"
     assert svg.lib.svg_status_string(99) == b"SVG_ERR_UNKNOWN"
@@ -99,6 +99,55 @@ def test_validation_rejects_bad_arguments():
     assert svg.lib.svg_profile_heads(ctypes.byref(s), p, p, p, 1, 1, p, 129, p, p, ws, 1 << 30, None) == 1
     assert svg.lib.svg_profile_heads(ctypes.byref(s), p, p, p, 1, 1, p, 32, p, p, ws, 16, None) == 5  # workspace
     assert svg.lib.svg_block_list(0, 1, 1, 1, 1, p, p, p, p) == 1
+
+
+def test_shape_struct_matches_header():
+    """svg_shape as the header declares it: seven 4-byte fields, then the
+    layout; a zero-initialised layout is [B, H, L, d]."""
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct svg_shape \{(.*?)\} svg_shape;", src, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"(\w+)\s*[,;]", body)
+    assert fields == ["B", "H", "N", "F", "d", "dtype", "scale", "layout"]
+    assert [f for f, _ in svg.svg_shape._fields_] == fields
+    assert ctypes.sizeof(svg.svg_shape) == 32 and svg.svg_shape.layout.offset == 28
+    assert svg.svg_shape(1, 2, 3, 4, 64, 0, 0.0).layout == svg.SVG_LAYOUT_BHLD
+    for name, val in (("SVG_LAYOUT_BHLD", 0), ("SVG_LAYOUT_BLHD", 1)):
+        assert re.search(rf"#define {name} {val}\b", src)
+        assert getattr(svg, name) == val
+
+
+def test_layout_validation_and_sizes():
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    bad = svg.svg_shape(1, 2, 4, 64, 64, svg.SVG_BF16, 0.0, 2)
+    assert svg.lib.svg_permute(ctypes.byref(bad), p, ctypes.c_void_p(2 << 20), None, None) == 1
+    assert b"unknown layout" in svg.lib.svg_last_error()
+    assert svg.lib.svg_profile_heads_noalloc(ctypes.byref(bad), p, p, p, 1, 1, p, 16, p, p, None) == 1
+    assert svg.svg_sparse_3d_attn_workspace_size(bad, 4, 16) == 0
+    # the host-buffer call copies whole heads: [B, H, L, d] only
+    s = svg.svg_shape(1, 2, 4, 64, 64, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BLHD)
+    st = svg.lib.svg_sparse_3d_attn_host(ctypes.byref(s), p, p, p, p, 1, 4, p, 16, p, p, 1, p, 1 << 30, None, None)
+    assert st == 2 and b"[B, H, L, d]" in svg.lib.svg_last_error()
+    # workspaces do not depend on the layout
+    for (B, H, N, F, d, a2) in ((2, 3, 5, 100, 64, 60), (1, 24, 33, 3600, 128, 281), (2, 3, 16, 64, 128, 4)):
+        s0 = svg.svg_shape(B, H, N, F, d, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BHLD)
+        s1 = svg.svg_shape(B, H, N, F, d, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BLHD)
+        assert svg.svg_sparse_3d_attn_workspace_size(s0, a2, 64) == svg.svg_sparse_3d_attn_workspace_size(s1, a2, 64)
+        assert svg.svg_sparse_3d_attn_plan(s0, a2) == svg.svg_sparse_3d_attn_plan(s1, a2)
+        assert svg.svg_profile_workspace_size(s0, 64) == svg.svg_profile_workspace_size(s1, 64)
+
+
+def test_make_shape_reads_either_layout():
+    import torch
+    x = torch.empty(2, 3, 5 * 7, 64, dtype=torch.bfloat16)  # [B, H, L, d]
+    s = svg.make_shape(x, 5, 7)
+    assert (s.B, s.H, s.N, s.F, s.d, s.layout) == (2, 3, 5, 7, 64, svg.SVG_LAYOUT_BHLD)
+    s = svg.make_shape(x.transpose(1, 2).contiguous(), 5, 7, layout="blhd")  # [B, L, H, d]
+    assert (s.B, s.H, s.N, s.F, s.d, s.layout) == (2, 3, 5, 7, 64, svg.SVG_LAYOUT_BLHD)
+    with pytest.raises(ValueError):
+        svg.make_shape(x, 5, 7, layout="blhd")  # 3 rows of 35 heads: L != N*F
+    with pytest.raises(ValueError):
+        svg.make_shape(x, 5, 7, layout="lbhd")
 
 
 def test_workspace_sizes():

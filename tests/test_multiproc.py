@@ -5,7 +5,9 @@
   calls all ranks made.
 * Head sharding: the library's partition (svg_head_shard) covers every head
   exactly once, and the binding's all-gather (gather_heads) assembles the
-  ranks' blocks into the single-rank result of the whole call.
+  ranks' blocks into the single-rank result of the whole call; gather_output
+  does the same for outputs in the [B, L, H, d] layout, whose head blocks are
+  not contiguous.
 """
 import os
 import socket
@@ -162,3 +164,43 @@ def test_head_sharded_call_assembles_the_single_rank_result(world):
         np.testing.assert_array_equal(label, ref_label)
         np.testing.assert_array_equal(mse, ref_mse)
         np.testing.assert_array_equal(o, ref_o)
+
+
+def _layout_gather_worker(rank, world, port, out):
+    """Each rank writes only its own block of heads of a [B, L, H, d] output
+    (value = a code of (b, h, x, c)) and gathers the rest."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from sparse_attention_video_profile_b200 import svg
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, H, L, d = 2, 3, 5, 4
+        code = torch.arange(B * H * L * d, dtype=torch.float32).view(B, H, L, d).transpose(1, 2).contiguous()
+        o = torch.full_like(code, -1.0)
+        first, count = svg.svg_head_shard(B * H, rank, world)
+        for g in range(first, first + count):
+            o[g // H, :, g % H] = code[g // H, :, g % H]
+        svg.gather_output(o, B * H, rank, world, "blhd")
+        out[rank] = bool(torch.equal(o, code))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gather_output_blhd(world):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_layout_gather_worker, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(300)
+            assert p.exitcode == 0
+        res = dict(out)
+    assert all(res[r] for r in range(world))

@@ -35,7 +35,9 @@
  *             (SVG_LAYOUT_BHLD, the default) or [B, L, H, d]
  *             (SVG_LAYOUT_BLHD, the heads of one token side by side, as a
  *             fused QKV projection writes them).  The arithmetic does not
- *             depend on the layout: both give bit-identical results.
+ *             depend on the layout: every kernel gives bit-identical
+ *             results on either (svg_sparse_3d_attn picks its plan per
+ *             layout, see there).
  *             Token-major ("permuted") tensors have the same shape and
  *             layout with token (i, j) at row x' = j*N + i.  Workspaces are
  *             opaque.  svg_sparse_3d_attn_host takes [B, H, L, d] only.
@@ -348,10 +350,14 @@ SVG_API svg_status svg_sparse_3d_attn_plan(const svg_shape* shape, int32_t a2, i
  * `stream` with no host synchronisation: profile -> block-sparse attention
  * with the layout transformation fused in (svg_block_sparse_attn_fused), or
  * profile -> permute temporal heads -> block-sparse attention -> unpermute.
- * The fused form is used for bf16 when its frame-group tiling costs at most
- * 3 % more attention work than the token-major copies (about what the two
- * permutation passes cost), counted on the host from N, F and a2; fp32
- * always permutes.  Outputs o (frame-major [B,H,L,d]) plus the profiling
+ * The fused form is used for bf16 [B, H, L, d] tensors when its frame-group
+ * tiling costs at most 3 % more attention work than the token-major copies
+ * (about what the two permutation passes cost), counted on the host from N,
+ * F and a2; fp32 and [B, L, H, d] tensors always permute (in [B, L, H, d]
+ * the fused boxes span the whole tensor and measured slower than the
+ * copies, which the workspace holds as [B, H, L, d]).  Results are
+ * bit-identical across layouts for the same plan; the two plans differ in
+ * the order keys are summed (rounding only).  Outputs o (frame-major [B,H,L,d]) plus the profiling
  * results mse [B,H,2] and label [B,H] (device).  If profiling fails on the
  * device (see svg_profile_heads), its SVG_DEV_* bits are OR-ed into
  * status_dev and every head, labelled -1, gets the spatial attention; both

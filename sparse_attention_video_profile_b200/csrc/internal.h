@@ -140,8 +140,9 @@ void token_major_tile_counts(int N, int F, int a, long long* separate, long long
 // True when the fused layout does at most 3 % more attention work than the
 // token-major copies (about what the permute + unpermute passes cost).
 bool fused_layout_preferred(int N, int F, int a);
-// The choice svg_sparse_3d_attn makes (and its host-buffer form): bf16 and
-// fused_layout_preferred with the clamped temporal band.
+// The choice svg_sparse_3d_attn makes (and its host-buffer form): bf16,
+// [B, H, L, d] tensors and fused_layout_preferred with the clamped temporal
+// band.
 bool whole_call_fused(const svg_shape* s, int a2);
 svg_status launch_attn_simt(const BandAttnArgs& a, cudaStream_t stream);
 // Tile shape of the tcgen05 kernel (rows of Q per tile, keys per tile).

@@ -96,8 +96,13 @@ HeadStrides shape_strides(const svg_shape* sh) {
 
 // The whole bf16 call folds the layout transformation into attention when
 // that costs at most 3 % more attention work than the token-major copies.
+// Not for [B, L, H, d] tensors: there one frame-group box, and one warp's
+// output rows, span every frame of the tensor (frame stride F*H*d elements,
+// 21.6 MB at HunyuanVideo, against F*d in [B, H, L, d]), and the fused
+// attention ran 4 % slower than on [B, H, L, d] while the separate passes
+// (token-major copies in [B, H, L, d]) ran as fast.
 bool whole_call_fused(const svg_shape* s, int a2) {
-  if (s->dtype != SVG_BF16 || a2 < 1) return false;
+  if (s->dtype != SVG_BF16 || a2 < 1 || s->layout == SVG_LAYOUT_BLHD) return false;
   return fused_layout_preferred(s->N, s->F, clamp_band(a2, s->N, s->N * s->F));
 }
 

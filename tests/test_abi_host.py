@@ -128,13 +128,19 @@ def test_layout_validation_and_sizes():
     s = svg.svg_shape(1, 2, 4, 64, 64, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BLHD)
     st = svg.lib.svg_sparse_3d_attn_host(ctypes.byref(s), p, p, p, p, 1, 4, p, 16, p, p, 1, p, 1 << 30, None, None)
     assert st == 2 and b"[B, H, L, d]" in svg.lib.svg_last_error()
-    # workspaces do not depend on the layout
+    # [B, L, H, d] whole calls always permute into [B, H, L, d] copies; the
+    # tile counts and the profiling workspace do not depend on the layout
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
     for (B, H, N, F, d, a2) in ((2, 3, 5, 100, 64, 60), (1, 24, 33, 3600, 128, 281), (2, 3, 16, 64, 128, 4)):
         s0 = svg.svg_shape(B, H, N, F, d, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BHLD)
         s1 = svg.svg_shape(B, H, N, F, d, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BLHD)
-        assert svg.svg_sparse_3d_attn_workspace_size(s0, a2, 64) == svg.svg_sparse_3d_attn_workspace_size(s1, a2, 64)
-        assert svg.svg_sparse_3d_attn_plan(s0, a2) == svg.svg_sparse_3d_attn_plan(s1, a2)
-        assert svg.svg_profile_workspace_size(s0, 64) == svg.svg_profile_workspace_size(s1, 64)
+        sep0, fz0, _ = svg.svg_sparse_3d_attn_plan(s0, a2)
+        sep1, fz1, fused1 = svg.svg_sparse_3d_attn_plan(s1, a2)
+        assert (sep0, fz0) == (sep1, fz1) and fused1 is False
+        prof = svg.svg_profile_workspace_size(s0, 64)
+        assert svg.svg_profile_workspace_size(s1, 64) == prof
+        assert svg.svg_sparse_3d_attn_workspace_size(s1, a2, 64) == prof + 4 * al(B * H * N * F * d * 2)
+    assert svg.svg_sparse_3d_attn_plan(svg.svg_shape(1, 24, 33, 3600, 128, svg.SVG_BF16, 0.0), 281)[2] is True
 
 
 def test_make_shape_reads_either_layout():

@@ -163,33 +163,45 @@ def test_dense_layouts_identical(dtype, d):
     assert_close(f64(bhld(o1)), oracle.dense_attention(f64(q), f64(k), f64(v)), q.dtype, "dense, [B, L, H, d]")
 
 
-def _whole_call_shapes():
-    """Small shapes on which the whole call takes each of its two layout
-    plans (fused into attention, or separate permute passes)."""
-    out = []
-    for (N, F, a2) in ((16, 64, 4), (5, 100, 60), (8, 128, 3), (3, 200, 150)):
-        shape = svg.svg_shape(2, 3, N, F, 64, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BLHD)
-        out.append((N, F, a2, svg.svg_sparse_3d_attn_plan(shape, a2)[2]))
-    return out
+def separate_call(q, k, v, N, F, a1, a2, rows, status):
+    """The whole call's separate plan on [B, H, L, d] tensors, step by step:
+    profile -> permute -> block-sparse attention -> unpermute (the plan the
+    [B, L, H, d] whole call always takes)."""
+    mse, label = svg.svg_profile_heads(q, k, v, N, F, a1, a2, rows)
+    qp, kp, vp = svg.svg_permute_qkv(q, k, v, N, F, label)
+    o, op = svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, a1, a2, status=status)
+    svg.svg_unpermute(op, N, F, label, out=o)
+    return o, mse, label
 
 
-def test_whole_call_shapes_cover_both_plans():
-    assert {fused for *_, fused in _whole_call_shapes()} == {True, False}
+def test_whole_call_plan_by_layout():
+    """[B, L, H, d] whole calls permute into copies; [B, H, L, d] ones fuse
+    where the fused tiling costs little (both plans occur in the shapes below)."""
+    plans = set()
+    for (N, F, a2) in WHOLE_CALL_SHAPES:
+        s0 = svg.svg_shape(2, 3, N, F, 64, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BHLD)
+        s1 = svg.svg_shape(2, 3, N, F, 64, svg.SVG_BF16, 0.0, svg.SVG_LAYOUT_BLHD)
+        plans.add(svg.svg_sparse_3d_attn_plan(s0, a2)[2])
+        assert svg.svg_sparse_3d_attn_plan(s1, a2)[2] is False
+    assert plans == {True, False}
 
 
-@pytest.mark.parametrize("N,F,a2,fused", _whole_call_shapes())
+WHOLE_CALL_SHAPES = ((16, 64, 4), (5, 100, 60), (8, 128, 3), (3, 200, 150))
+
+
+@pytest.mark.parametrize("N,F,a2", WHOLE_CALL_SHAPES)
 @pytest.mark.parametrize("d", [64, 128])
-def test_whole_call_layouts_identical(N, F, a2, fused, d):
+def test_whole_call_layouts_identical(N, F, a2, d):
     wl = workload(N, F, d, a1=2, a2=a2)
     (q, k, v), (qt, kt, vt), rows_np, rows = inputs(wl, 16)
     s0, s1 = new_status(), new_status()
-    o0, mse0, lab0 = svg.svg_sparse_3d_attn(q, k, v, N, F, wl.a1, wl.a2, rows, status=s0)
+    o0, mse0, lab0 = separate_call(q, k, v, N, F, wl.a1, wl.a2, rows, s0)
     o1, mse1, lab1 = svg.svg_sparse_3d_attn(qt, kt, vt, N, F, wl.a1, wl.a2, rows, status=s1, layout="blhd")
     sync_ok(s0, s1)
     assert torch.equal(mse0, mse1) and torch.equal(lab0, lab1)
     assert torch.equal(o0, bhld(o1))
     ref = oracle.sparse_attention(f64(q), f64(k), f64(v), lab1.cpu().numpy(), N, F, wl.a1, wl.a2)
-    assert_close(f64(bhld(o1)), ref, torch.bfloat16, f"whole call ({'fused' if fused else 'separate'})")
+    assert_close(f64(bhld(o1)), ref, torch.bfloat16, "whole call, [B, L, H, d]")
 
 
 def test_whole_call_fp32_layouts_identical():
@@ -270,15 +282,23 @@ def test_shard_layouts_identical(world):
 
 @pytest.mark.parametrize("name", ["cogvideox", "hunyuan"])
 def test_video_shape_layouts_identical(name):
-    """The full call at the video-model shape, every output element."""
+    """The full call at the video-model shape, every output element: the
+    [B, L, H, d] whole call against the same plan on [B, H, L, d] tensors,
+    and the fused attention in both layouts."""
     wl = synth.WORKLOADS[name]
     q, k, v = synth.make_qkv(wl, seed=3, device=DEV)
     rows = torch.from_numpy(synth.sample_rows(wl.L, wl.S, 3)).to(DEV)
-    s0, s1 = new_status(), new_status()
-    o0, mse0, lab0 = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, status=s0)
+    s0, s1, s2, s3 = new_status(), new_status(), new_status(), new_status()
+    o0, mse0, lab0 = separate_call(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, s0)
+    f0 = svg.svg_block_sparse_attn_fused(q, k, v, lab0, wl.N, wl.F, wl.a1, wl.a2, status=s2)
+    torch.cuda.synchronize()
+    o0, f0 = o0.cpu(), f0.cpu()
     qt, kt, vt = blhd(q), blhd(k), blhd(v)
     del q, k, v
+    torch.cuda.empty_cache()
     o1, mse1, lab1 = svg.svg_sparse_3d_attn(qt, kt, vt, wl.N, wl.F, wl.a1, wl.a2, rows, status=s1, layout="blhd")
-    sync_ok(s0, s1)
+    f1 = svg.svg_block_sparse_attn_fused(qt, kt, vt, lab1, wl.N, wl.F, wl.a1, wl.a2, status=s3, layout="blhd")
+    sync_ok(s0, s1, s2, s3)
     assert torch.equal(mse0, mse1) and torch.equal(lab0, lab1)
-    assert torch.equal(o0, bhld(o1))
+    assert torch.equal(o0, bhld(o1).cpu())
+    assert torch.equal(f0, bhld(f1).cpu())

@@ -34,17 +34,20 @@ from sparse_attention_video_profile_b200 import metrics, synth  # noqa: E402
 METRIC = "ms per sparse 3D-attention call; effective TFLOPS vs bf16 peak; speedup vs dense"
 
 # DRAM bytes (read + write) per full-size launch of the attention kernel, from
-# an ncu capture of a 4-head case of the same shape scaled by heads, keyed by
+# an ncu capture of a 4-head case of the same shape scaled by heads (the
+# "-blhd" entry: of the full launch itself), keyed by
 # the sha256 prefix of the kernel sources it was taken on and by the layout
-# (fused or separate).  Any other revision or layout reports traffic as null
-# until it is captured again.
+# (fused or separate, "-blhd" appended for [B, L, H, d] tensors).  Any other
+# revision or layout reports traffic as null until it is captured again.
 NCU_TRAFFIC = {("645b18066bbc1e1a", "d2f4abb45748fc0c", "fused"): 2.8525e9,
-               ("20c87c577a0d9af9", "5edc1f6588b2c178", "fused"): 2.8583e9}
+               ("20c87c577a0d9af9", "5edc1f6588b2c178", "fused"): 2.8583e9,
+               ("239a7b5e36619c63", "3c4a90062d61487f", "fused"): 2.8442e9,
+               ("239a7b5e36619c63", "3c4a90062d61487f", "separate-blhd"): 2.9109e9}
 
 
 # The same for the profiling stage-1 kernel (full HunyuanVideo launch), keyed by
 # the sha256 prefix of its source.
-PROF_NCU_TRAFFIC = {"5732be8477404d60": 1.488e9}
+PROF_NCU_TRAFFIC = {"5732be8477404d60": 1.488e9, "a5d1bd300122e4a1": 1.4840e9}
 
 
 def prof_source_key():
@@ -545,6 +548,10 @@ def run_ours(args, wl, rank, world, local):
     # partition of svg_head_shard, as svg_sparse_3d_attn_shard runs it: views
     # of the block, no copies), or with --shard replicas runs its own call
     shard_heads = world > 1 and args.shard == "heads"
+    tl = args.tensor_layout
+    if shard_heads and tl != "bhld":
+        raise SystemExit("--tensor-layout blhd runs one call per rank: use --shard replicas for N > 1")
+    lk = {"layout": tl}  # every call of the step on the same tensor layout
     job_wl = wl
     if shard_heads:
         import dataclasses
@@ -559,6 +566,8 @@ def run_ours(args, wl, rank, world, local):
     else:
         q, k, v = synth.make_qkv(wl, seed=rank, device=dev)
         rows_np = synth.sample_rows(wl.L, wl.S, rank)
+    if tl == "blhd":  # [B, L, H, d]: the same values, heads inside the token axis
+        q, k, v = (t.transpose(1, 2).contiguous() for t in (q, k, v))
     rows = torch.from_numpy(rows_np).to(dev)
     N, F = wl.N, wl.F
     o = torch.empty_like(q)
@@ -567,7 +576,7 @@ def run_ours(args, wl, rank, world, local):
     mse = torch.empty(wl.B, wl.H, 2, dtype=torch.float32, device=dev)
     label = torch.empty(wl.B, wl.H, dtype=torch.int8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    shape = svg.make_shape(q, N, F)
+    shape = svg.make_shape(q, N, F, layout=tl)
     prof_ws = svg.alloc_workspace(svg.svg_profile_workspace_size(shape, wl.S), dev)
 
     mixed = wl.name.startswith("mixed")
@@ -594,22 +603,22 @@ def run_ours(args, wl, rank, world, local):
             if e:
                 e["attn"][0].record(stream)
             svg.svg_mixed_attn_fused(q, k, v, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
-                                     status=status)
+                                     status=status, **lk)
             if e:
                 e["attn"][1].record(stream)
             return
         if e:
             e["permute"][0].record(stream)
-        svg.svg_permute_qkv(q, k, v, N, F, md_label, out=(qp, kp, vp))
+        svg.svg_permute_qkv(q, k, v, N, F, md_label, out=(qp, kp, vp), **lk)
         if e:
             e["permute"][1].record(stream)
             e["attn"][0].record(stream)
         svg.svg_mixed_attn(q, k, v, qp, kp, vp, mode, N, F, prm["window"], prm["md_half"], prm["stripe"], o=o,
-                           op=op, status=status)
+                           op=op, status=status, **lk)
         if e:
             e["attn"][1].record(stream)
             e["unpermute"][0].record(stream)
-        svg.svg_unpermute(op, N, F, md_label, out=o)
+        svg.svg_unpermute(op, N, F, md_label, out=o, **lk)
         if e:
             e["unpermute"][1].record(stream)
 
@@ -618,27 +627,27 @@ def run_ours(args, wl, rank, world, local):
             return step_mixed(e)
         if e:
             e["profile"][0].record(stream)
-        svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws)
+        svg.svg_profile_heads(q, k, v, N, F, wl.a1, wl.a2, rows, mse=mse, label=label, workspace=prof_ws, **lk)
         if fused:
             if e:
                 e["profile"][1].record(stream)
                 e["attn"][0].record(stream)
-            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status)
+            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status, **lk)
             if e:
                 e["attn"][1].record(stream)
             return
         if e:
             e["profile"][1].record(stream)
             e["permute"][0].record(stream)
-        svg.svg_permute_qkv(q, k, v, N, F, label, out=(qp, kp, vp))
+        svg.svg_permute_qkv(q, k, v, N, F, label, out=(qp, kp, vp), **lk)
         if e:
             e["permute"][1].record(stream)
             e["attn"][0].record(stream)
-        svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status)
+        svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status, **lk)
         if e:
             e["attn"][1].record(stream)
             e["unpermute"][0].record(stream)
-        svg.svg_unpermute(op, N, F, label, out=o)
+        svg.svg_unpermute(op, N, F, label, out=o, **lk)
         if e:
             e["unpermute"][1].record(stream)
 
@@ -683,13 +692,13 @@ def run_ours(args, wl, rank, world, local):
     dense_ms = None
     if not args.no_dense:
         od = torch.empty_like(q)
-        svg.svg_dense_attn(q, k, v, N, F, o=od)
+        svg.svg_dense_attn(q, k, v, N, F, o=od, **lk)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 2
         a.record(stream)
         for _ in range(reps):
-            svg.svg_dense_attn(q, k, v, N, F, o=od)
+            svg.svg_dense_attn(q, k, v, N, F, o=od, **lk)
         b.record(stream)
         torch.cuda.synchronize()
         dense_ms = a.elapsed_time(b) / reps
@@ -705,7 +714,7 @@ def run_ours(args, wl, rank, world, local):
 
         def search():
             svg.svg_mode_search(q, k, v, N, F, rows, prm["window"], prm["md_half"], prm["stripe"], loss=ms_loss,
-                                mode=ms_mode, workspace=ms_ws)
+                                mode=ms_mode, workspace=ms_ws, **lk)
 
         search()
         torch.cuda.synchronize()
@@ -726,7 +735,7 @@ def run_ours(args, wl, rank, world, local):
 
     # end to end through the public call with host buffers
     e2e = None
-    if not args.no_e2e and not mixed:
+    if not args.no_e2e and not mixed and tl == "bhld":  # the host-buffer call takes [B, H, L, d]
         # host tensors (page-locked); the call pipelines its own copies
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
@@ -771,8 +780,8 @@ def run_ours(args, wl, rank, world, local):
     if not mixed and n_temporal and not args.no_configs:
         if fused:
             qp, kp, vp, op = (torch.empty_like(q) for _ in range(4))
-        t_perm = time_calls(lambda: svg.svg_permute_qkv(q, k, v, N, F, label, out=(qp, kp, vp)), 5, stream)
-        t_unperm = time_calls(lambda: svg.svg_unpermute(op, N, F, label, out=o), 5, stream)
+        t_perm = time_calls(lambda: svg.svg_permute_qkv(q, k, v, N, F, label, out=(qp, kp, vp), **lk), 5, stream)
+        t_unperm = time_calls(lambda: svg.svg_unpermute(op, N, F, label, out=o, **lk), 5, stream)
         layout_kernels = {
             "permute_ms": t_perm, "permute_gbs": perm_bytes / (t_perm * 1e-3) / 1e9,
             "permute_frac_hbm": perm_bytes / (t_perm * 1e-3) / 1e9 / hbm,
@@ -793,7 +802,7 @@ def run_ours(args, wl, rank, world, local):
                             "traffic": PROF_NCU_TRAFFIC.get(prof_source_key()) if wl.name == "hunyuan" else None,
                             "algorithmic_work": f"{prof_bytes:.4e} bytes/launch = K and V of every head once"}
     configs = None
-    if not args.no_configs and rank == 0 and world == 1 and wl.name == "hunyuan":
+    if not args.no_configs and rank == 0 and world == 1 and wl.name == "hunyuan" and tl == "bhld":
         configs = []
         qp = kp = vp = op = None
         torch.cuda.empty_cache()
@@ -809,7 +818,7 @@ def run_ours(args, wl, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not mixed:
-        qkv64 = head_f64(wl, q, k, v)
+        qkv64 = head_f64(wl, *((t.transpose(1, 2) for t in (q, k, v)) if tl == "blhd" else (q, k, v)))
         ms, desc, _ = oracle_sample(wl, qkv64, rows_np, labels_np, n_prof_rows=wl.S, n_attn_rows=1024)
         cpu = {"value": ms, "unit": "ms/call", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
 
@@ -818,7 +827,8 @@ def run_ours(args, wl, rank, world, local):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False,
         "scaling": "strong" if shard_heads else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(job_wl, world, "heads" if shard_heads else "replicas"),
+        "config": dict(config_dict(job_wl, world, "heads" if shard_heads else "replicas"),
+                       tensor_layout="[B, L, H, d]" if tl == "blhd" else "[B, H, L, d]"),
         "effective_tflops": attn_tflops, "effective_tflops_call": flops / (step_ms * 1e-3) / 1e12,
         "frac_bf16_peak": attn_tflops / peak,
         "speedup_vs_dense": (dense_ms / step_ms) if dense_ms else None,
@@ -840,7 +850,8 @@ def run_ours(args, wl, rank, world, local):
                      "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "peak_sustained": peak_sus, "frac_sustained": attn_tflops / peak_sus,
                      "traffic": args.traffic if args.traffic is not None else (
-                         NCU_TRAFFIC.get(attn_source_key() + ("fused" if fused else "separate",))
+                         NCU_TRAFFIC.get(attn_source_key() + (("fused" if fused else "separate")
+                                                               + ("" if tl == "bhld" else "-blhd"),))
                          if wl.name == "hunyuan" else None),
                      "algorithmic_work": f"{flops:.4e} flops/launch = 4*d*unmasked pairs"},
         "roofline_profile": roofline_profile,
@@ -873,6 +884,9 @@ def main():
     ap.add_argument("--layout", choices=["auto", "fused", "separate"], default="auto",
                     help="temporal heads' layout transformation fused into attention, or as separate kernels; "
                          "auto = the whole call's own choice")
+    ap.add_argument("--tensor-layout", choices=["bhld", "blhd"], default="bhld",
+                    help="q, k, v, o as [B, H, L, d] or [B, L, H, d] (the whole call then takes the separate plan; "
+                         "no host-buffer e2e, which takes [B, H, L, d])")
     ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per chunk of the host-buffer call")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

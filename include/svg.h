@@ -88,7 +88,14 @@ typedef enum svg_status {
   SVG_ERR_WORKSPACE = 5    /* workspace smaller than the size query says   */
 } svg_status;
 
-typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1 } svg_dtype;
+/* Element type of the Q/K/V/O tensors and the arithmetic of attention:
+ * SVG_BF16  bf16 tensors, tcgen05 kind::f16 products, fp32 softmax and
+ *           accumulation, bf16 output;
+ * SVG_FP32  fp32 tensors, fp32 arithmetic on the CUDA cores (the exact path);
+ * SVG_TF32  fp32 tensors, attention products on the tcgen05 tensor cores in
+ *           tf32 (kind::tf32: 10-bit mantissas), fp32 softmax, accumulation
+ *           and output; profiling, permutation and labels as SVG_FP32. */
+typedef enum svg_dtype { SVG_BF16 = 0, SVG_FP32 = 1, SVG_TF32 = 2 } svg_dtype;
 
 #define SVG_SPATIAL 0
 #define SVG_TEMPORAL 1

@@ -81,7 +81,7 @@ int full_call_chunk(const svg_shape* s, int S) {
 
 SlotLayout slot_layout(const svg_shape* s, int S, int hc, bool fused) {
   SlotLayout l{};
-  const size_t es = s->dtype == SVG_FP32 ? 4 : 2;
+  const size_t es = s->dtype == SVG_BF16 ? 2 : 4;
   l.tensor = align256(static_cast<size_t>(hc) * s->N * s->F * s->d * es);
   ProfileLayout pl;
   if (!profile_layout(1, hc, s->N * s->F, s->d, s->dtype, S, &pl, 0, full_call_chunk(s, S))) pl.total = 0;
@@ -129,7 +129,7 @@ SVG_API svg_status svg_sparse_3d_attn_host(const svg_shape* shape, const void* q
   const int hc = heads_per_chunk < BH ? heads_per_chunk : BH;
   const bool fused = whole_call_fused(shape, a2);
   const SlotLayout lay = slot_layout(shape, S, hc, fused);
-  const size_t es = shape->dtype == SVG_FP32 ? 4 : 2;
+  const size_t es = shape->dtype == SVG_BF16 ? 2 : 4;
   const size_t head_bytes = static_cast<size_t>(shape->N) * shape->F * shape->d * es;
 
   PipeResources* r = nullptr;

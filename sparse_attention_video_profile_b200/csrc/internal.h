@@ -145,6 +145,9 @@ bool fused_layout_preferred(int N, int F, int a);
 // band.
 bool whole_call_fused(const svg_shape* s, int a2);
 svg_status launch_attn_simt(const BandAttnArgs& a, cudaStream_t stream);
+// fp32 tensors on the tensor cores in tf32 (attn_tf32.cu): bands with or
+// without labels (no modes, fused layout or SVG2 mode).
+svg_status launch_attn_tf32(const BandAttnArgs& a, cudaStream_t stream);
 // Tile shape of the tcgen05 kernel (rows of Q per tile, keys per tile).
 constexpr int kAttnBq = 128;
 constexpr int kAttnBk = 128;

@@ -288,7 +288,8 @@ svg_status launch_stage1_f32(const ProfParams& p, cudaStream_t stream) {
   return cuda_check(cudaGetLastError(), "fp32 profile launch");
 }
 
-int row_block(int /*d*/, int dtype) { return dtype == SVG_FP32 ? 4 : 128; }
+// fp32 and tf32 tensors profile alike (fp32 on the CUDA cores)
+int row_block(int /*d*/, int dtype) { return dtype == SVG_BF16 ? 128 : 4; }
 
 }  // namespace
 
@@ -297,7 +298,7 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
   const int rb = row_block(d, dtype);
   ProfileLayout lay{};
   lay.S_pad = (S + rb - 1) / rb * rb;
-  if (dtype == SVG_FP32) {
+  if (dtype != SVG_BF16) {
     lay.n_chunks = 1;
     lay.chunk = L;
   } else if (chunk_len > 0) {

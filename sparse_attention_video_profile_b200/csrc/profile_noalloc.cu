@@ -58,12 +58,13 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
   if (shape->B < 1 || shape->H < 1 || shape->N < 1 || shape->F < 1 || shape->d < 1)
     return fail(SVG_ERR_INVALID_ARG, "B, H, N, F, d must be >= 1");
   if (static_cast<long long>(shape->N) * shape->F > (1LL << 30)) return fail(SVG_ERR_INVALID_ARG, "L too large");
-  if (shape->dtype != SVG_BF16 && shape->dtype != SVG_FP32) return fail(SVG_ERR_INVALID_ARG, "unknown dtype");
+  if (shape->dtype != SVG_BF16 && shape->dtype != SVG_FP32 && shape->dtype != SVG_TF32)
+    return fail(SVG_ERR_INVALID_ARG, "unknown dtype");
   if (shape->layout != SVG_LAYOUT_BHLD && shape->layout != SVG_LAYOUT_BLHD)
     return fail(SVG_ERR_INVALID_ARG, "unknown layout");
   if (!(shape->scale >= 0.f) || isinf(shape->scale)) return fail(SVG_ERR_INVALID_ARG, "bad scale");
   if ((shape->dtype == SVG_BF16 && shape->d != 64 && shape->d != 128) ||
-      (shape->dtype == SVG_FP32 && shape->d != 32 && shape->d != 64 && shape->d != 128))
+      (shape->dtype != SVG_BF16 && shape->d != 32 && shape->d != 64 && shape->d != 128))
     return fail(SVG_ERR_UNSUPPORTED, "unsupported head dim %d for this dtype", shape->d);
   for (const void* t : {q, k, v})
     if (t == nullptr || (reinterpret_cast<uintptr_t>(t) & 15u) != 0)

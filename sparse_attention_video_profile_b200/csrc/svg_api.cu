@@ -30,7 +30,7 @@ __device__ int g_internal_status;
 
 namespace {
 
-size_t elem_size(int dtype) { return dtype == SVG_FP32 ? 4 : 2; }
+size_t elem_size(int dtype) { return dtype == SVG_BF16 ? 2 : 4; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -40,14 +40,15 @@ svg_status check_shape(const svg_shape* s) {
     return fail(SVG_ERR_INVALID_ARG, "B, H, N, F, d must be >= 1 (got %d %d %d %d %d)", s->B, s->H, s->N, s->F, s->d);
   if (static_cast<long long>(s->N) * s->F > (1LL << 30))
     return fail(SVG_ERR_INVALID_ARG, "L = N*F = %lld is too large", static_cast<long long>(s->N) * s->F);
-  if (s->dtype != SVG_BF16 && s->dtype != SVG_FP32) return fail(SVG_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+  if (s->dtype != SVG_BF16 && s->dtype != SVG_FP32 && s->dtype != SVG_TF32)
+    return fail(SVG_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
   if (s->layout != SVG_LAYOUT_BHLD && s->layout != SVG_LAYOUT_BLHD)
     return fail(SVG_ERR_INVALID_ARG, "unknown layout %d", s->layout);
   if (!(s->scale >= 0.f) || isinf(s->scale)) return fail(SVG_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (s->dtype == SVG_BF16 && s->d != 64 && s->d != 128)
     return fail(SVG_ERR_UNSUPPORTED, "bf16 supports d in {64, 128}, got %d", s->d);
-  if (s->dtype == SVG_FP32 && s->d != 32 && s->d != 64 && s->d != 128)
-    return fail(SVG_ERR_UNSUPPORTED, "fp32 supports d in {32, 64, 128}, got %d", s->d);
+  if (s->dtype != SVG_BF16 && s->d != 32 && s->d != 64 && s->d != 128)
+    return fail(SVG_ERR_UNSUPPORTED, "fp32 / tf32 support d in {32, 64, 128}, got %d", s->d);
   return SVG_OK;
 }
 
@@ -146,6 +147,7 @@ svg_status run_attention(const svg_shape* s, const HeadStrides& hs, const HeadSt
   svg_status st = status_word(status_dev, &a.status, stream);
   if (st != SVG_OK) return st;
   if (s->dtype == SVG_BF16) return launch_attn_sm100(a, stream);
+  if (s->dtype == SVG_TF32) return launch_attn_tf32(a, stream);
   return launch_attn_simt(a, stream);
 }
 
@@ -185,6 +187,12 @@ svg_status svg_attn_tile(int32_t dtype, int32_t d, int32_t* Bq, int32_t* Bk) {
   if (dtype == SVG_FP32) {  // one row at a time, 32 keys per step
     *Bq = 1;
     *Bk = 32;
+    return SVG_OK;
+  }
+  if (dtype == SVG_TF32) {  // 128-row query tiles, 128-key tiles
+    if (d != 32 && d != 64 && d != 128) return fail(SVG_ERR_UNSUPPORTED, "tf32 supports d in {32, 64, 128}");
+    *Bq = kAttnBq;
+    *Bk = kAttnBk;
     return SVG_OK;
   }
   return fail(SVG_ERR_INVALID_ARG, "unknown dtype %d", dtype);
@@ -237,7 +245,7 @@ size_t svg_workspace_size(const svg_shape* shape, int32_t n_temporal_heads_max) 
   const size_t prof = svg_profile_workspace_size(shape, L < 128 ? L : 128);
   if (prof == 0) return 0;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-  const size_t elt = shape->dtype == SVG_FP32 ? 4 : 2;
+  const size_t elt = elem_size(shape->dtype);
   const size_t tensor = al(static_cast<size_t>(shape->B) * shape->H * L * shape->d * elt);
   return al(prof) + (n_temporal_heads_max > 0 ? 4 * tensor : 0);
 }

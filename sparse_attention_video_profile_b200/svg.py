@@ -27,6 +27,7 @@ LIB_PATH = os.environ.get("SVG_LIB") or os.path.join(os.path.dirname(os.path.abs
 SVG_OK = 0
 SVG_BF16 = 0
 SVG_FP32 = 1
+SVG_TF32 = 2
 SPATIAL = 0
 TEMPORAL = 1
 SVG_DEV_TIMEOUT = 0x1
@@ -141,9 +142,11 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
 
 
-def make_shape(x: torch.Tensor, N: int, F: int, scale: float = 0.0, layout: str = "bhld") -> svg_shape:
+def make_shape(x: torch.Tensor, N: int, F: int, scale: float = 0.0, layout: str = "bhld",
+               tf32: bool = False) -> svg_shape:
     """The svg_shape of a q/k/v tensor: [B, H, L, d] (layout "bhld") or
-    [B, L, H, d] ("blhd")."""
+    [B, L, H, d] ("blhd").  tf32=True (float32 tensors only) runs attention
+    on the tensor cores in tf32 (SVG_TF32) instead of fp32 on the CUDA cores."""
     if layout not in LAYOUTS:
         raise ValueError(f"layout must be one of {sorted(LAYOUTS)}, got {layout!r}")
     if x.dim() != 4:
@@ -154,7 +157,12 @@ def make_shape(x: torch.Tensor, N: int, F: int, scale: float = 0.0, layout: str 
         B, L, H, d = x.shape
     if L != N * F:
         raise ValueError(f"L = {L} but N*F = {N * F}")
-    return svg_shape(B, H, N, F, d, _dtype_code(x), float(scale), LAYOUTS[layout])
+    code = _dtype_code(x)
+    if tf32:
+        if code != SVG_FP32:
+            raise TypeError("tf32=True takes float32 tensors")
+        code = SVG_TF32
+    return svg_shape(B, H, N, F, d, code, float(scale), LAYOUTS[layout])
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -289,10 +297,10 @@ def svg_unpermute(xp, N: int, F: int, label=None, *, out=None, layout: str = "bh
 
 
 def svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N: int, F: int, a1: int, a2: int, *, o=None, op=None,
-                          status=None, scale: float = 0.0, layout: str = "bhld", stream=None):
+                          status=None, scale: float = 0.0, layout: str = "bhld", tf32: bool = False, stream=None):
     """Returns (o, op): spatial heads' output in o, temporal heads' in op."""
     _same(q, k, v, qp, kp, vp)
-    shape = make_shape(q, N, F, scale, layout)
+    shape = make_shape(q, N, F, scale, layout, tf32=tf32)
     if o is None:
         o = torch.empty_like(q)
     if op is None:
@@ -316,9 +324,9 @@ def svg_block_sparse_attn_fused(q, k, v, label, N: int, F: int, a1: int, a2: int
 
 
 def svg_banded_attn(q, k, v, N: int, F: int, G: int, a: int, *, o=None, status=None, scale: float = 0.0,
-                    layout: str = "bhld", stream=None):
+                    layout: str = "bhld", tf32: bool = False, stream=None):
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale, layout)
+    shape = make_shape(q, N, F, scale, layout, tf32=tf32)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_banded_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), G, a, _ptr(status),
@@ -327,9 +335,9 @@ def svg_banded_attn(q, k, v, N: int, F: int, G: int, a: int, *, o=None, status=N
 
 
 def svg_dense_attn(q, k, v, N: int, F: int, *, o=None, status=None, scale: float = 0.0, layout: str = "bhld",
-                   stream=None):
+                   tf32: bool = False, stream=None):
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale, layout)
+    shape = make_shape(q, N, F, scale, layout, tf32=tf32)
     if o is None:
         o = torch.empty_like(q)
     _check(lib.svg_dense_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(status),
@@ -339,10 +347,10 @@ def svg_dense_attn(q, k, v, N: int, F: int, *, o=None, status=None, scale: float
 
 def svg_sparse_3d_attn(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, *, o=None, mse=None,
                        label=None, workspace=None, status=None, scale: float = 0.0, layout: str = "bhld",
-                       stream=None):
+                       tf32: bool = False, stream=None):
     """One whole sparse 3D-attention call.  Returns (o, mse, label)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale, layout)
+    shape = make_shape(q, N, F, scale, layout, tf32=tf32)
     S = rows.numel()
     if o is None:
         o = torch.empty_like(q)
@@ -402,13 +410,13 @@ def gather_output(o: torch.Tensor, n_heads: int, rank: int, world: int, layout: 
 
 def svg_sparse_3d_attn_shard(q, k, v, N: int, F: int, a1: int, a2: int, rows: torch.Tensor, rank: int, world: int, *,
                              o=None, mse=None, label=None, workspace=None, status=None, scale: float = 0.0,
-                             layout: str = "bhld", stream=None, gather: bool = False, group=None):
+                             layout: str = "bhld", tf32: bool = False, stream=None, gather: bool = False, group=None):
     """This rank's block of heads of one whole call (q, k, v are the full
     tensors).  Returns (o, mse, label) full-size; only this rank's heads are
     written unless gather=True, which then fills the rest from the other
     ranks (torch.distributed must be initialised)."""
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale, layout)
+    shape = make_shape(q, N, F, scale, layout, tf32=tf32)
     S = rows.numel()
     if o is None:
         o = torch.empty_like(q)
@@ -474,7 +482,7 @@ def svg_mixed_3d_attn(q, k, v, mode, N: int, F: int, window: int, md_half: int, 
 
 def svg_sparse_3d_attn_host(q, k, v, N: int, F: int, a1: int, a2: int, rows, *, o=None, mse=None, label=None,
                             heads_per_chunk: int = 4, workspace=None, status=None, scale: float = 0.0,
-                            device=None, stream=None):
+                            device=None, tf32: bool = False, stream=None):
     """svg_sparse_3d_attn on host (CPU) tensors, copies overlapped with the
     kernels.  q, k, v (and o) should be pinned.  Returns (o, mse, label) as
     host tensors, valid after `stream` (the current stream) synchronises."""
@@ -482,7 +490,7 @@ def svg_sparse_3d_attn_host(q, k, v, N: int, F: int, a1: int, a2: int, rows, *, 
         if t.device.type != "cpu":
             raise ValueError("svg_sparse_3d_attn_host takes host tensors")
     _same(q, k, v)
-    shape = make_shape(q, N, F, scale)
+    shape = make_shape(q, N, F, scale, tf32=tf32)
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     rows = rows.to(torch.int32).contiguous()
     if o is None:
@@ -604,15 +612,16 @@ class SparseAttention3D:
     workspace between calls (svg_sparse_3d_attn: profiling, then attention
     with the layout transformation fused in or as separate passes)."""
 
-    def __init__(self, N: int, F: int, a1: int, a2: int, scale: float = 0.0, layout: str = "bhld"):
-        self.N, self.F, self.a1, self.a2, self.scale, self.layout = N, F, a1, a2, scale, layout
+    def __init__(self, N: int, F: int, a1: int, a2: int, scale: float = 0.0, layout: str = "bhld",
+                 tf32: bool = False):
+        self.N, self.F, self.a1, self.a2, self.scale, self.layout, self.tf32 = N, F, a1, a2, scale, layout, tf32
         self._ws = None
 
     def __call__(self, q, k, v, rows, *, o=None, mse=None, label=None, status=None, stream=None):
-        shape = make_shape(q, self.N, self.F, self.scale, self.layout)
+        shape = make_shape(q, self.N, self.F, self.scale, self.layout, self.tf32)
         need = svg_sparse_3d_attn_workspace_size(shape, self.a2, rows.numel())
         if self._ws is None or self._ws.numel() < need or self._ws.device != q.device:
             self._ws = alloc_workspace(need, q.device)
         return svg_sparse_3d_attn(q, k, v, self.N, self.F, self.a1, self.a2, rows, o=o, mse=mse, label=label,
                                   workspace=self._ws, status=status, scale=self.scale, layout=self.layout,
-                                  stream=stream)
+                                  tf32=self.tf32, stream=stream)

@@ -143,6 +143,29 @@ def test_layout_validation_and_sizes():
     assert svg.svg_sparse_3d_attn_plan(svg.svg_shape(1, 24, 33, 3600, 128, svg.SVG_BF16, 0.0), 281)[2] is True
 
 
+def test_tf32_dtype_host_side():
+    """SVG_TF32: fp32 tensors (4-byte workspaces, the fp32 profiling layout),
+    128 x 128 attention tiles, d in {32, 64, 128}; the binding takes it for
+    float32 tensors only."""
+    import torch
+    assert svg.svg_attn_tile(svg.SVG_TF32, 64) == (128, 128)
+    f = svg.svg_shape(2, 3, 5, 40, 64, svg.SVG_FP32, 0.0)
+    t = svg.svg_shape(2, 3, 5, 40, 64, svg.SVG_TF32, 0.0)
+    assert svg.svg_profile_workspace_size(t, 32) == svg.svg_profile_workspace_size(f, 32) > 0
+    assert svg.svg_sparse_3d_attn_workspace_size(t, 4, 32) == svg.svg_sparse_3d_attn_workspace_size(f, 4, 32) > 0
+    assert svg.svg_workspace_size(t, 2) == svg.svg_workspace_size(f, 2)
+    assert svg.svg_sparse_3d_attn_plan(t, 4)[2] is False  # fp32 tensors always permute
+    p = ctypes.c_void_p(1 << 20)
+    bad = svg.svg_shape(1, 2, 4, 64, 96, svg.SVG_TF32, 0.0)
+    assert svg.lib.svg_dense_attn(ctypes.byref(bad), p, p, p, p, None, None) == 2
+    bad = svg.svg_shape(1, 2, 4, 64, 64, 3, 0.0)
+    assert svg.lib.svg_dense_attn(ctypes.byref(bad), p, p, p, p, None, None) == 1
+    x = torch.empty(1, 2, 20, 64)
+    assert svg.make_shape(x, 4, 5, tf32=True).dtype == svg.SVG_TF32
+    with pytest.raises(TypeError):
+        svg.make_shape(x.to(torch.bfloat16), 4, 5, tf32=True)
+
+
 def test_make_shape_reads_either_layout():
     import torch
     x = torch.empty(2, 3, 5 * 7, 64, dtype=torch.bfloat16)  # [B, H, L, d]

@@ -1,6 +1,7 @@
 """The range-checked build (libsvg_debug.so, svg_debug_checks() == 1) on the
 tiny and small shapes: every tensor-core kernel path -- banded and fused
-attention, mixed patterns, the SVG2 cluster-pair mode, k-means, profiling --
+attention, mixed patterns, the SVG2 cluster-pair mode, k-means, profiling,
+the tf32 attention of fp32 tensors --
 runs with its global indices checked, and must report no SVG_DEV_BOUNDS and
 still match the fp64 oracle.  This stands in for a memory checker: an index
 outside its buffer is recorded in the status word and the access skipped,
@@ -154,3 +155,19 @@ def test_profile_and_mode_search_checked(dsvg):
     assert torch.all(label >= 0) and torch.all(torch.isfinite(mse))
     assert torch.all(mode >= 0) and torch.all(torch.isfinite(loss))
     np.testing.assert_array_equal(label.cpu().numpy(), synth.head_kinds(wl, 4))
+
+
+@pytest.mark.parametrize("d", [32, 128])
+def test_tf32_checked(dsvg, d):
+    """fp32 tensors in tf32, with labels (token-major copies) and ragged L."""
+    N, F = 5, 61
+    g = torch.Generator(device=DEV)
+    g.manual_seed(70 + d)
+    q, k, v = (torch.randn(2, 3, N * F, d, generator=g, device=DEV) for _ in range(3))
+    rows = torch.from_numpy(synth.sample_rows(N * F, 32, 7)).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, mse, label = dsvg.svg_sparse_3d_attn(q, k, v, N, F, 2, 9, rows, status=status, tf32=True)
+    no_bounds(status, "tf32")
+    ref = oracle.sparse_attention(f64(q), f64(k), f64(v), label.cpu().numpy(), N, F, 2, 9)
+    got = f64(o)
+    assert np.max(np.abs(got - ref)) <= 1e-2 and np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 4e-3

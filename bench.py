@@ -64,6 +64,9 @@ def attn_source_key():
 # kernels one bf16 profiling call launches: tcgen05 stage 1, row combine, per-head finalize
 PROFILE_LAUNCHES = 3
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# dense tf32 / bf16 tensor throughput, nominal (1.1 / 2.25 PFLOP/s per B200)
+TF32_PER_BF16 = 1.1 / 2.25
+TF32_PEAK_NOTE = " x 1.1/2.25 (nominal tf32 / bf16 ratio)"
 
 
 def load_peaks():
@@ -552,6 +555,10 @@ def run_ours(args, wl, rank, world, local):
     if shard_heads and tl != "bhld":
         raise SystemExit("--tensor-layout blhd runs one call per rank: use --shard replicas for N > 1")
     lk = {"layout": tl}  # every call of the step on the same tensor layout
+    tf32 = args.precision == "tf32"
+    ak = dict(lk, tf32=True) if tf32 else lk  # attention calls: fp32 tensors through the tf32 tensor cores
+    if tf32 and (shard_heads or wl.name.startswith("mixed")):
+        raise SystemExit("--precision tf32 runs the spatial / temporal call on one GPU (or replicas)")
     job_wl = wl
     if shard_heads:
         import dataclasses
@@ -568,6 +575,9 @@ def run_ours(args, wl, rank, world, local):
         rows_np = synth.sample_rows(wl.L, wl.S, rank)
     if tl == "blhd":  # [B, L, H, d]: the same values, heads inside the token axis
         q, k, v = (t.transpose(1, 2).contiguous() for t in (q, k, v))
+    if tf32:  # the same values as fp32 tensors
+        q, k, v = (t.float().contiguous() for t in (q, k, v))
+    es = q.element_size()
     rows = torch.from_numpy(rows_np).to(dev)
     N, F = wl.N, wl.F
     o = torch.empty_like(q)
@@ -576,7 +586,7 @@ def run_ours(args, wl, rank, world, local):
     mse = torch.empty(wl.B, wl.H, 2, dtype=torch.float32, device=dev)
     label = torch.empty(wl.B, wl.H, dtype=torch.int8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    shape = svg.make_shape(q, N, F, layout=tl)
+    shape = svg.make_shape(q, N, F, layout=tl, tf32=tf32)
     prof_ws = svg.alloc_workspace(svg.svg_profile_workspace_size(shape, wl.S), dev)
 
     mixed = wl.name.startswith("mixed")
@@ -632,7 +642,7 @@ def run_ours(args, wl, rank, world, local):
             if e:
                 e["profile"][1].record(stream)
                 e["attn"][0].record(stream)
-            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status, **lk)
+            svg.svg_block_sparse_attn_fused(q, k, v, label, N, F, wl.a1, wl.a2, o=o, status=status, **ak)
             if e:
                 e["attn"][1].record(stream)
             return
@@ -643,7 +653,7 @@ def run_ours(args, wl, rank, world, local):
         if e:
             e["permute"][1].record(stream)
             e["attn"][0].record(stream)
-        svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status, **lk)
+        svg.svg_block_sparse_attn(q, k, v, qp, kp, vp, label, N, F, wl.a1, wl.a2, o=o, op=op, status=status, **ak)
         if e:
             e["attn"][1].record(stream)
             e["unpermute"][0].record(stream)
@@ -692,13 +702,13 @@ def run_ours(args, wl, rank, world, local):
     dense_ms = None
     if not args.no_dense:
         od = torch.empty_like(q)
-        svg.svg_dense_attn(q, k, v, N, F, o=od, **lk)
+        svg.svg_dense_attn(q, k, v, N, F, o=od, **ak)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 2
         a.record(stream)
         for _ in range(reps):
-            svg.svg_dense_attn(q, k, v, N, F, o=od, **lk)
+            svg.svg_dense_attn(q, k, v, N, F, o=od, **ak)
         b.record(stream)
         torch.cuda.synchronize()
         dense_ms = a.elapsed_time(b) / reps
@@ -747,7 +757,8 @@ def run_ours(args, wl, rank, world, local):
 
         def e2e_step():
             svg.svg_sparse_3d_attn_host(qh, kh, vh, N, F, wl.a1, wl.a2, rowsh, o=oh, mse=mseh, label=labh,
-                                        heads_per_chunk=args.e2e_chunk, workspace=ws_host_call, status=status)
+                                        heads_per_chunk=args.e2e_chunk, workspace=ws_host_call, status=status,
+                                        tf32=tf32)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -770,8 +781,10 @@ def run_ours(args, wl, rank, world, local):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     attn_tflops = flops / (kern_ms["attn"] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    perm_bytes = 2 * 3 * n_temporal * wl.B * wl.L * wl.d * 2
-    unperm_bytes = 2 * n_temporal * wl.B * wl.L * wl.d * 2
+    if tf32:  # dense tf32 runs at the nominal tf32 / bf16 ratio of the bf16 rate
+        peak *= TF32_PER_BF16
+    perm_bytes = 2 * 3 * n_temporal * wl.B * wl.L * wl.d * es
+    unperm_bytes = 2 * n_temporal * wl.B * wl.L * wl.d * es
 
     # the layout-transformation kernels on this call's labels, timed on their
     # own after the timed region (when the call fuses the layout they are not
@@ -791,7 +804,7 @@ def run_ours(args, wl, rank, world, local):
             "note": "svg_permute_qkv / svg_unpermute on this call's temporal heads, 2 warm + 5 timed calls each"}
         if fused:
             qp = kp = vp = op = None
-    prof_bytes = 2 * wl.B * wl.H * wl.L * wl.d * 2  # K and V read once
+    prof_bytes = 2 * wl.B * wl.H * wl.L * wl.d * es  # K and V read once
     roofline_profile = None
     if not mixed:
         prof_gbs = prof_bytes / (kern_ms["profile"] * 1e-3) / 1e9
@@ -802,7 +815,7 @@ def run_ours(args, wl, rank, world, local):
                             "traffic": PROF_NCU_TRAFFIC.get(prof_source_key()) if wl.name == "hunyuan" else None,
                             "algorithmic_work": f"{prof_bytes:.4e} bytes/launch = K and V of every head once"}
     configs = None
-    if not args.no_configs and rank == 0 and world == 1 and wl.name == "hunyuan" and tl == "bhld":
+    if not args.no_configs and rank == 0 and world == 1 and wl.name == "hunyuan" and tl == "bhld" and not tf32:
         configs = []
         qp = kp = vp = op = None
         torch.cuda.empty_cache()
@@ -815,6 +828,8 @@ def run_ours(args, wl, rank, world, local):
         torch.cuda.empty_cache()
     # the seconds-long power-capped figure, shown beside the burst one
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if tf32:
+        peak_sus *= TF32_PER_BF16
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not mixed:
@@ -826,7 +841,7 @@ def run_ours(args, wl, rank, world, local):
         "metric": METRIC, "value": value, "unit": "ms/call", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False,
         "scaling": "strong" if shard_heads else "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "tf32" if tf32 else "bf16", "data": "synthetic",
         "config": dict(config_dict(job_wl, world, "heads" if shard_heads else "replicas"),
                        tensor_layout="[B, L, H, d]" if tl == "blhd" else "[B, H, L, d]"),
         "effective_tflops": attn_tflops, "effective_tflops_call": flops / (step_ms * 1e-3) / 1e12,
@@ -846,12 +861,15 @@ def run_ours(args, wl, rank, world, local):
         "layout_kernels": layout_kernels,
         "temporal_heads": n_temporal,
         "density": pairs / (wl.B * wl.H * float(wl.L) * wl.L),
-        "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<128>", "achieved": attn_tflops, "peak": peak,
-                     "peak_kind": f"{peak_kind} bf16_tflops (burst)", "unit": "TFLOP/s", "frac": attn_tflops / peak,
+        "roofline": {"bound": "tensor", "kernel": f"{'attn_tf32_kernel' if tf32 else 'attn_sm100_kernel'}<{wl.d}>",
+                     "achieved": attn_tflops, "peak": peak,
+                     "peak_kind": f"{peak_kind} bf16_tflops (burst)" + (TF32_PEAK_NOTE if tf32 else ""),
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "peak_sustained": peak_sus, "frac_sustained": attn_tflops / peak_sus,
                      "traffic": args.traffic if args.traffic is not None else (
                          NCU_TRAFFIC.get(attn_source_key() + (("fused" if fused else "separate")
-                                                               + ("" if tl == "bhld" else "-blhd"),))
+                                                               + ("" if tl == "bhld" else "-blhd")
+                                                               + ("-tf32" if tf32 else ""),))
                          if wl.name == "hunyuan" else None),
                      "algorithmic_work": f"{flops:.4e} flops/launch = 4*d*unmasked pairs"},
         "roofline_profile": roofline_profile,
@@ -887,6 +905,9 @@ def main():
     ap.add_argument("--tensor-layout", choices=["bhld", "blhd"], default="bhld",
                     help="q, k, v, o as [B, H, L, d] or [B, L, H, d] (the whole call then takes the separate plan; "
                          "no host-buffer e2e, which takes [B, H, L, d])")
+    ap.add_argument("--precision", choices=["bf16", "tf32"], default="bf16",
+                    help="tf32: the same inputs as fp32 tensors, attention on the tensor cores in tf32 (SVG_TF32; "
+                         "profiling in fp32 on the CUDA cores)")
     ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per chunk of the host-buffer call")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

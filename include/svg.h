@@ -60,7 +60,7 @@
  *             can clear each other's bits: pass a word of your own to rely
  *             on them.  svg_last_error() gives a message for the last
  *             failing call on this host thread.
- *   Support.  bf16: d in {64, 128}.  fp32: d in {32, 64, 128}.  a1 >= 1,
+ *   Support.  bf16: d in {64, 128}.  fp32 and tf32: d in {32, 64, 128}.  a1 >= 1,
  *             a2 >= 1 (a1 >= N or a2 >= F keep every pair of that kind).
  */
 #ifndef SVG_H_
@@ -257,8 +257,7 @@ SVG_API svg_status svg_profile_heads(const svg_shape* shape, const void* q, cons
  * writes every byte it later reads.  Calls whose kernels overlap on the GPU,
  * for example on two streams, race on the array: serialise them.
  * Limits: shapes whose partial results cannot fit the array even with one
- * key chunk (bf16), or at all (fp32, which always uses one chunk), return
- * SVG_ERR_WORKSPACE before anything is enqueued.  The call allocates and
+ * key chunk return SVG_ERR_WORKSPACE before anything is enqueued.  The call allocates and
  * frees nothing.  Arguments are otherwise as for svg_profile_heads.
  */
 #define SVG_PROFILE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)

@@ -169,10 +169,11 @@ struct ProfileLayout {
 inline size_t profile_status_offset(const ProfileLayout& lay) { return lay.o_bytes + lay.ml_bytes + lay.part_bytes; }
 
 // Workspace layout of the profiling kernels.  max_chunks > 0 caps the number
-// of key chunks (fewer chunks need less workspace); chunk_len > 0 (bf16)
-// fixes the keys per chunk instead of choosing them for the head count, so a
-// call on a subset of heads splits the keys, and rounds, exactly as a call on
-// all of them; fp32 always uses one chunk.
+// of key chunks (fewer chunks need less workspace); chunk_len > 0 fixes the
+// keys per chunk instead of choosing them for the head count, so a call on a
+// subset of heads splits the keys, and rounds, exactly as a call on all of
+// them.  bf16 chunks are whole 128-key tiles, fp32 chunks (CUDA cores)
+// multiples of 32 keys, at least 1024 unless the sequence is shorter.
 bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout* out, int max_chunks = 0,
                     int chunk_len = 0);
 

@@ -42,15 +42,21 @@ struct ProfParams {
   float sl2;
 };
 
-// fp32 stage 1: one warp per (head, sampled row), all keys, chunk count 1.
+// fp32 stage 1: one warp per (head, sampled row, key chunk); the chunk
+// partials go to the same workspace layout as the bf16 stage 1's.  The four
+// rows of a block share each 32-key step's K and V rows, loaded once into
+// shared memory with coalesced reads (K rows padded by one word, so lane j
+// reading key j's column c hits bank (j + c) mod 32).
 template <int D>
 __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
   constexpr int PER = D / 32;
   __shared__ float sq[4][D];
+  __shared__ float sK[32][D + 1];
+  __shared__ float sV[32][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = blockIdx.x * 4 + warp;
-  const int bh = blockIdx.y;
-  if (s >= p.S_pad) return;
+  const int s = blockIdx.x * 4 + warp;  // < S_pad: S_pad is a multiple of the block's 4 rows
+  const int bh = blockIdx.y, ch = blockIdx.z;
+  const int y_begin = ch * p.chunk, y_end = min(p.L, y_begin + p.chunk);
   const long long hoff = p.hs.head(bh), sl = p.hs.sl;
   const float* q = static_cast<const float*>(p.q) + hoff;
   const float* k = static_cast<const float*>(p.k) + hoff;
@@ -67,15 +73,22 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
 #pragma unroll
     for (int t = 0; t < PER; ++t) acc[vv][t] = 0.f;
   }
-  for (int y0 = 0; y0 < p.L; y0 += 32) {
+  for (int y0 = y_begin; y0 < y_end; y0 += 32) {
+    __syncthreads();  // the previous step's rows are no longer read
+    for (int e = threadIdx.x; e < 32 * D; e += 128) {
+      const int r = e / D, c = e - r * D;
+      const bool in = y0 + r < y_end;
+      sK[r][c] = in ? k[(y0 + r) * sl + c] : 0.f;
+      sV[r][c] = in ? v[(y0 + r) * sl + c] : 0.f;
+    }
+    __syncthreads();
     const int y = y0 + lane;
     float sc = -INFINITY;
     int iy = -1, jy = -1;
-    if (y < p.L) {
-      const float* kr = k + y * sl;
+    if (y < y_end) {
       float dot = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < D; ++c) dot = fmaf(sq[warp][c], kr[c], dot);
+      for (int c = 0; c < D; ++c) dot = fmaf(sq[warp][c], sK[lane][c], dot);
       sc = dot;
       iy = y / p.F;
       jy = y % p.F;
@@ -83,7 +96,7 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
     float pv[3];
 #pragma unroll
     for (int vv = 0; vv < 3; ++vv) {
-      bool ok = y < p.L;
+      bool ok = y < y_end;
       if (vv == 1) ok = ok && abs(ir - iy) < p.a1;
       if (vv == 2) ok = ok && abs(jr - jy) < p.a2;
       const float sv = ok ? sc : -INFINITY;
@@ -102,12 +115,11 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
       for (int t = 0; t < PER; ++t) acc[vv][t] *= alpha;
       pv[vv] = pp;
     }
-    const int nvalid = min(32, p.L - y0);
+    const int nvalid = min(32, y_end - y0);
     for (int jj = 0; jj < nvalid; ++jj) {
-      const float* vr = v + (y0 + jj) * sl;
       float vals[PER];
 #pragma unroll
-      for (int t = 0; t < PER; ++t) vals[t] = vr[lane + 32 * t];
+      for (int t = 0; t < PER; ++t) vals[t] = sV[jj][lane + 32 * t];
 #pragma unroll
       for (int vv = 0; vv < 3; ++vv) {
         const float pj = __shfl_sync(0xffffffffu, pv[vv], jj);
@@ -118,7 +130,7 @@ __global__ void __launch_bounds__(128) profile_simt_kernel(const ProfParams p) {
   }
 #pragma unroll
   for (int vv = 0; vv < 3; ++vv) {
-    const size_t base = (static_cast<size_t>(bh) * 3 + vv) * p.S_pad + s;  // nch == 1
+    const size_t base = ((static_cast<size_t>(bh) * p.nch + ch) * 3 + vv) * p.S_pad + s;
 #pragma unroll
     for (int t = 0; t < PER; ++t) p.ws_o[base * D + lane + 32 * t] = acc[vv][t];
     if (lane == 0) {
@@ -283,7 +295,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 template <int D>
 svg_status launch_stage1_f32(const ProfParams& p, cudaStream_t stream) {
-  dim3 grid((p.S_pad + 3) / 4, p.BH);
+  if (p.nch > 65535) return fail(SVG_ERR_UNSUPPORTED, "%d key chunks exceed the grid limit", p.nch);
+  dim3 grid((p.S_pad + 3) / 4, p.BH, p.nch);
   profile_simt_kernel<D><<<grid, 128, 0, stream>>>(p);
   return cuda_check(cudaGetLastError(), "fp32 profile launch");
 }
@@ -299,8 +312,24 @@ bool profile_layout(int B, int H, int L, int d, int dtype, int S, ProfileLayout*
   ProfileLayout lay{};
   lay.S_pad = (S + rb - 1) / rb * rb;
   if (dtype != SVG_BF16) {
-    lay.n_chunks = 1;
-    lay.chunk = L;
+    // fp32 (CUDA cores): enough key chunks for about 16 blocks of 4 rows per
+    // SM, each chunk at least 1024 keys; chunk_len, when given, fixes it
+    long long chunk;
+    if (chunk_len > 0) {
+      chunk = (static_cast<long long>(chunk_len) + 31) / 32 * 32;
+    } else {
+      const long long blocks = static_cast<long long>(B) * H * (lay.S_pad / 4);
+      long long nch = (148LL * 16 + blocks - 1) / blocks;
+      long long most = (L + 1023) / 1024;
+      if (most > 65535) most = 65535;  // grid z
+      if (nch > most) nch = most;
+      if (max_chunks > 0 && nch > max_chunks) nch = max_chunks;
+      if (nch < 1) nch = 1;
+      chunk = ((L + nch - 1) / nch + 31) / 32 * 32;
+    }
+    if (chunk > L) chunk = L;
+    lay.chunk = static_cast<int>(chunk);
+    lay.n_chunks = static_cast<int>((L + chunk - 1) / chunk);
   } else if (chunk_len > 0) {
     long long chunk = (static_cast<long long>(chunk_len) + kKT - 1) / kKT * kKT;
     if (chunk > L) chunk = (L + kKT - 1) / kKT * kKT;

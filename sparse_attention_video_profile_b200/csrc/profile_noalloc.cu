@@ -78,16 +78,16 @@ extern "C" SVG_API svg_status svg_profile_heads_noalloc(const svg_shape* shape, 
   profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay);
   constexpr size_t kMax = SVG_PROFILE_NOALLOC_SCRATCH_BYTES;
   if (lay.total > kMax) {
-    // Fewer, longer key chunks need less scratch (bf16 path; fp32 uses one chunk).
+    // Fewer, longer key chunks need less scratch.
     ProfileLayout one;
     profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &one, 1);
     const size_t per_chunk = one.o_bytes + one.ml_bytes;  // bytes that scale with the chunk count
     const long long fit = static_cast<long long>((kMax - one.part_bytes - one.status_bytes - 512) / per_chunk);
-    if (shape->dtype != SVG_BF16 || one.total > kMax || fit < 1)
+    if (one.total > kMax || fit < 1)
       return fail(SVG_ERR_WORKSPACE,
                   "profiling this shape needs at least %zu bytes of scratch, more than the %zu-byte static "
                   "array of svg_profile_heads_noalloc; use svg_profile_heads with a workspace",
-                  shape->dtype != SVG_BF16 ? lay.total : one.total, kMax);
+                  one.total, kMax);
     profile_layout(shape->B, shape->H, L, shape->d, shape->dtype, S, &lay, static_cast<int>(fit));
     if (lay.total > kMax) return fail(SVG_ERR_WORKSPACE, "scratch layout does not fit the static array");
   }

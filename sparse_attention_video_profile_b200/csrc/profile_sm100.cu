@@ -7,22 +7,27 @@
 // one chunk of keys, computes three online-softmax attention states at once:
 // unmasked (d), spatial |i_x - i_y| < a1 (s) and temporal |j_x - j_y| < a2
 // (t).  Per 128-key tile:
-//   S = Q K^T                       one tcgen05.mma group into TMEM
-//   P_d, P_s (bf16) written over S  -> O_d += P_d V, O_s += P_s V
-//   P_t written over P_d once P_d V has read it -> O_t += P_t V
+//   S_k = Q K_k^T                     one tcgen05.mma group into TMEM
+//   P_d, P_s, P_t (bf16) in shared memory -> O_v += P_v V_k, v = d, s, t
 // The three variants share one softmax reference, the running max over all
 // kept keys, so each key needs one exponential: P_s and P_t are P_d
 // restricted to the spatial and temporal masks (the normalisation of each
 // variant divides the reference out again).
-// The three P V products read P straight from TMEM (A-from-TMEM form).  The
-// partial (max, sum, unnormalised output) triples of every row and variant
-// go to the workspace; the combine kernels merge the chunks.
+// TMEM holds S and the three accumulators (all 512 columns at d = 128), so
+// there is one S buffer; P goes to shared memory instead (three 32 KB
+// K-major tiles, the A operands of the P V products), which frees S as soon
+// as the softmax has read it.  The tensor cores then compute S_{k+1} while
+// the softmax works on tile k, and the products of tile k follow; the
+// softmax waits for the products of tile k-1 only before it overwrites P.
+// The partial (max, sum, unnormalised output) triples of every row and
+// variant go to the workspace; the combine kernels merge the chunks.
 // TMEM: S [0,128), O_d [128,128+D), O_s [128+D,128+2D), O_t [128+2D,128+3D).
 //
 // Warps 0-7: two threads per sampled row, one per 64-key half of each tile
 // (Q gather, masks, three softmaxes, epilogue); the halves exchange their
 // maxima through shared memory once per tile.  Warp 8: TMA producer of K and
-// V.  Warp 9: MMA issuer.
+// V (the ring is short, so it also prefetches tiles further ahead into L2).
+// Warp 9: MMA issuer.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -55,8 +60,11 @@ struct PCfg {
   static constexpr int HALVES = D / 64;
   static constexpr int HALF_BYTES = 128 * 128;
   static constexpr int TILE_BYTES = 128 * D * 2;
-  static constexpr int NS = (D == 128) ? 5 : 8;
-  static constexpr int SMEM_BAR = TILE_BYTES + NS * TILE_BYTES;
+  static constexpr int P_BYTES = 128 * 128 * 2;  // one P tile: 128 rows x 128 keys, two 64-key halves
+  static constexpr int NS = (D == 128) ? 2 : 6;
+  static constexpr int PF = 4;                   // ring entries prefetched into L2 ahead of their load
+  static constexpr int SMEM_P = TILE_BYTES + NS * TILE_BYTES;
+  static constexpr int SMEM_BAR = SMEM_P + 3 * P_BYTES;
   static constexpr int SMEM_X = SMEM_BAR + 512;  // row-max exchange [2][2][128] + final sums [5][128] (fp32)
   static constexpr int SMEM_BYTES = SMEM_X + 5120 + 1024;
   // 10 warps: softmax 0-7 (warp w: rows 32 (w & 3) .. +31, key columns
@@ -64,7 +72,16 @@ struct PCfg {
   static constexpr int THREADS = 320;
   static constexpr uint32_t COL_S = 0;
   static constexpr uint32_t col_o(int v) { return 128u + D * v; }
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
+
+// Prefetch of a 4D tile into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
 
 // Pairs (of 8) of each half row's exponentials computed by the FMA-pipe
 // polynomial instead of the MUFU ex2 unit.
@@ -164,17 +181,16 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + C::TILE_BYTES;
+  uint8_t* sP = smem + C::SMEM_P;               // [3] P_d, P_s, P_t (bf16, K-major, 128-byte swizzle)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
   uint64_t* bar_q = bars;                       // 128 arrivals: Q gathered
   uint64_t* bar_full = bars + 1;                // [NS]
   uint64_t* bar_empty = bars + 1 + C::NS;       // [NS]
-  uint64_t* bar_s = bars + 1 + 2 * C::NS;       // S ready
-  uint64_t* bar_p01 = bar_s + 1;                // 256 arrivals: P_d, P_s written
-  uint64_t* bar_o01 = bar_s + 2;                // P_d V, P_s V done
-  uint64_t* bar_pt = bar_s + 3;                 // 256 arrivals: P_t written
-  uint64_t* bar_ot = bar_s + 4;                 // P_t V done
-  uint64_t* bar_od = bar_s + 5;                 // P_d V done (P_t may overwrite P_d)
-  uint64_t* bar_x = bar_s + 6;                  // [4] 64 arrivals: the two halves of 32 rows exchanged
+  uint64_t* bar_s = bars + 1 + 2 * C::NS;       // S_k ready (and every earlier product done)
+  uint64_t* bar_sfree = bar_s + 1;              // 256 arrivals: S_k read, its columns free
+  uint64_t* bar_p = bar_s + 2;                  // 256 arrivals: P_d, P_s, P_t of tile k written
+  uint64_t* bar_pv = bar_s + 3;                 // the three P V products of tile k done
+  uint64_t* bar_x = bar_s + 4;                  // [4] 64 arrivals: the two halves of 32 rows exchanged
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_x + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xm = reinterpret_cast<float*>(smem + C::SMEM_X);  // [2 parity][2 half][128 rows] half-row maxima
@@ -195,11 +211,9 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(bar_s, 1);
-    mbar_init(bar_p01, 256);
-    mbar_init(bar_o01, 1);
-    mbar_init(bar_pt, 256);
-    mbar_init(bar_ot, 1);
-    mbar_init(bar_od, 1);
+    mbar_init(bar_sfree, 256);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_pv, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&bar_x[q], 64);
     fence_barrier_init();
   }
@@ -218,20 +232,44 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
     const int th = p.hs.tma_h(bh), tb = p.hs.tma_b(bh);
+    // entry n of the ring: K_0, then K_{k+1} ahead of V_k (the order the MMA
+    // warp consumes them): K_0, K_1, V_0, K_2, V_1, ..., K_{nk-1}, V_{nk-2}, V_{nk-1}
+    auto entry_tile = [&](int n, bool& is_v) {
+      if (n == 0) {
+        is_v = false;
+        return 0;
+      }
+      if ((n & 1) && (n + 1) / 2 < nk) {
+        is_v = false;
+        return (n + 1) / 2;
+      }
+      is_v = true;
+      return (n & 1) ? nk - 1 : n / 2 - 1;
+    };
+    auto prefetch = [&](int n) {
+      bool is_v;
+      const int t = entry_tile(n, is_v);
+#pragma unroll
+      for (int h = 0; h < C::HALVES; ++h)
+        tma_prefetch_l2_4d(is_v ? &p.tm_v : &p.tm_k, h * 64, (kt0 + t) * 128, th, tb);
+    };
+    for (int n = 0; n < min(C::PF, 2 * nk); ++n) prefetch(n);
     for (int n = 0; n < 2 * nk; ++n) {
       const int slot = n % C::NS;
+      if (n + C::PF < 2 * nk) prefetch(n + C::PF);  // on its way to L2 while n waits for its slot
       if (!mbar_wait(&bar_empty[slot], ((n / C::NS) & 1) ^ 1, p.wait_ns)) {
         *abort_flag = 1;
         atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
         break;
       }
-      const CUtensorMap* tm = (n & 1) ? &p.tm_v : &p.tm_k;
-      in_range((kt0 + (n >> 1)) * 128, p.L, p.status);
+      bool is_v;
+      const int t = entry_tile(n, is_v);
+      in_range((kt0 + t) * 128, p.L, p.status);
       mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
       for (int h = 0; h < C::HALVES; ++h)
-        tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, tm, &bar_full[slot], h * 64,
-                    (kt0 + (n >> 1)) * 128, th, tb);
+        tma_load_4d(sRing + slot * C::TILE_BYTES + h * C::HALF_BYTES, is_v ? &p.tm_v : &p.tm_k, &bar_full[slot],
+                    h * 64, (kt0 + t) * 128, th, tb);
     }
   } else if (run && warp == 9) {
     // ------------------------------------------------ MMA issuer
@@ -243,42 +281,53 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dk = smem_desc_sw128(ring_base, 16, 1024);
     const uint64_t dv = smem_desc_sw128(ring_base, C::HALF_BYTES, 1024);
-    auto pv = [&](int v, uint32_t pcol, int slot, bool acc) {
+    const uint64_t dp = smem_desc_sw128(smem_u32(sP), 16, 1024);
+    // O_v += P_v V: A = P_v (K-major in shared memory), B = V (MN-major)
+    auto pv = [&](int v, int slot, bool acc) {
+      const uint64_t a = dp + static_cast<uint64_t>((v * C::P_BYTES) >> 4);
       const uint64_t b = dv + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        umma_ts_warp(tmem + C::col_o(v), tmem + pcol + kk * 8, b + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t aoff = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
+        umma_ss_warp(tmem + C::col_o(v), a + aoff, b + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
                      (acc || kk > 0) ? 1u : 0u);
+      }
     };
-    bool ok = warp_wait_p(bar_q, 0, p.wait_ns);
-    for (int k = 0; ok && k < nk; ++k) {
-      const int nK = 2 * k, nV = 2 * k + 1;
-      const int slotK = nK % C::NS, slotV = nV % C::NS;
-      ok = warp_wait_p(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const uint64_t b = dk + static_cast<uint64_t>((slotK * C::TILE_BYTES) >> 4);
+    // S_k = Q K_k^T into the S columns
+    auto qk = [&](int slot) {
+      const uint64_t b = dk + static_cast<uint64_t>((slot * C::TILE_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
-          umma_ss_warp(tmem + C::COL_S, dq + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::HALF_BYTES + (kk & 3) * 32) >> 4);
+        umma_ss_warp(tmem + C::COL_S, dq + off, b + off, idesc_qk, kk > 0 ? 1u : 0u);
       }
       umma_commit_warp(bar_s);
-      umma_commit_warp(&bar_empty[slotK]);
-      ok = warp_wait_p(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns) && warp_wait_p(bar_p01, k & 1, p.wait_ns);
+      umma_commit_warp(&bar_empty[slot]);
+    };
+    // Ring entries (the producer's order): K_0 is entry 0, K_{k+1} entry
+    // 2k + 1, V_k entry 2k + 2 (the last V entry 2 nk - 1).  S_{k+1} goes in
+    // as soon as the softmax has read S_k, ahead of the products of tile k.
+    bool ok = warp_wait_p(bar_q, 0, p.wait_ns) && warp_wait_p(&bar_full[0], 0, p.wait_ns);
+    if (ok) {
+      tc_fence_after();
+      qk(0);
+    }
+    for (int k = 0; ok && k < nk; ++k) {
+      if (k + 1 < nk) {
+        const int nK = 2 * k + 1, slotK = nK % C::NS;
+        ok = warp_wait_p(bar_sfree, k & 1, p.wait_ns) && warp_wait_p(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+        qk(slotK);
+      }
+      const int nV = (k + 1 < nk) ? 2 * k + 2 : 2 * nk - 1, slotV = nV % C::NS;
+      ok = warp_wait_p(bar_p, k & 1, p.wait_ns) && warp_wait_p(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      pv(0, C::COL_S, slotV, k > 0);  // O_d += P_d V
-      umma_commit_warp(bar_od);
-      pv(1, C::COL_S + 64, slotV, k > 0);  // O_s += P_s V
-      umma_commit_warp(bar_o01);
-      ok = warp_wait_p(bar_pt, k & 1, p.wait_ns);
-      if (!ok) break;
-      tc_fence_after();
-      pv(2, C::COL_S, slotV, k > 0);  // O_t += P_t V
-      umma_commit_warp(bar_ot);
+      pv(0, slotV, k > 0);  // O_d += P_d V
+      pv(1, slotV, k > 0);  // O_s += P_s V
+      pv(2, slotV, k > 0);  // O_t += P_t V
+      umma_commit_warp(bar_pv);
       umma_commit_warp(&bar_empty[slotV]);
     }
     if (!ok && lane == 0) {
@@ -346,6 +395,8 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       tmem_wait_ld();
       reg_fence32(sr[0]);
       reg_fence32(sr[1]);
+      tc_fence_before();
+      mbar_arrive(bar_sfree);  // S_{k+1} may overwrite the columns
       float s[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
@@ -389,18 +440,14 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
         m3 = fmax3f(m3, s[c + 6], s[c + 7]);
       }
       const float mh = fmaxf(fmax3f(m0, m1, m2), m3);
-      // The row's maximum over the whole tile, from both halves.  The
-      // exchange also orders both halves' score loads before either half's P
-      // stores, which overwrite score columns the other half reads.
+      // The row's maximum over the whole tile, from both halves.
       float* xk = xm + (k & 1) * 256;
       xk[h * 128 + r] = mh;
-      tc_fence_before();
       mbar_arrive(&bar_x[q]);
       if (!warp_wait_p(&bar_x[q], k & 1, p.wait_ns)) {
         ok = false;
         break;
       }
-      tc_fence_after();
       const float m_new = fmax3f(m_ref, mh, xk[(h ^ 1) * 128 + r]);
       float alpha = 1.f;
       bool resc = false;
@@ -437,44 +484,39 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       float wsum[2];
       pack_plain(s, pkd, wsum);
       l_d = l_d * alpha + (wsum[0] + wsum[1]);
-      __syncwarp();
-      tmem_st32(tS + h * 32, pkd);  // P_d: packed columns [0, 64)
-      l_s = l_s * alpha + pack_variant(pkd, wsum, ms, pk);
-      __syncwarp();
-      tmem_st32(tS + 64 + h * 32, pk);  // P_s: packed columns [64, 128)
-      // both halves of a row take the same decision (same reference)
-      const bool any_resc = k > 0 && __any_sync(0xffffffffu, resc);
-      if (any_resc) {
-        if (!warp_wait_p(bar_o01, (k - 1) & 1, p.wait_ns)) {
+      // the products of tile k-1 read P and add into O: wait for them before
+      // overwriting P or rescaling O (bar_s of this tile already covers the
+      // products of tile k-2, so the barrier is never two phases behind)
+      if (k > 0) {
+        if (!warp_wait_p(bar_pv, (k - 1) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
+      }
+      // this half row = 64 keys = one 128-byte row of a swizzled 64-key block
+      uint8_t* prow = sP + h * C::HALF_BYTES + r * 128;
+      auto store_p = [&](int v, const uint32_t(&w)[32]) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + v * C::P_BYTES + ((c ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      };
+      store_p(0, pkd);
+      l_s = l_s * alpha + pack_variant(pkd, wsum, ms, pk);
+      store_p(1, pk);
+      l_t = l_t * alpha + pack_variant(pkd, wsum, mt, pk);
+      store_p(2, pk);
+      // both halves of a row take the same decision (same reference)
+      if (k > 0 && __any_sync(0xffffffffu, resc)) {
         rescale_o_half<D>(tO + C::col_o(0), alpha);
         rescale_o_half<D>(tO + C::col_o(1), alpha);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p01);
-      l_t = l_t * alpha + pack_variant(pkd, wsum, mt, pk);
-      // P_t goes over P_d once P_d V has read it (P_s V may still run)
-      if (!warp_wait_p(bar_od, k & 1, p.wait_ns)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st32(tS + h * 32, pk);
-      if (any_resc) {
-        if (!warp_wait_p(bar_ot, (k - 1) & 1, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         rescale_o_half<D>(tO + C::col_o(2), alpha);
+        tmem_wait_st();
       }
-      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // P visible to the tensor cores
       tc_fence_before();
-      mbar_arrive(bar_pt);
+      mbar_arrive(bar_p);
     }
     // the first half of each row collects the second half's sums and counts
     if (ok) {
@@ -499,7 +541,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
       // row max): report it rather than return a wrong label.
       if ((inband_s > 0 && !(l_s > 0.f)) || (inband_t > 0 && !(l_t > 0.f))) atomicOr(p.status, SVG_DEV_RANGE);
     }
-    if (ok && warp_wait_p(bar_ot, (nk - 1) & 1, p.wait_ns)) {
+    if (ok && warp_wait_p(bar_pv, (nk - 1) & 1, p.wait_ns)) {
       tc_fence_after();
 #pragma unroll
       for (int v = 0; v < 3; ++v) {

@@ -7,9 +7,11 @@
 // G = N, a = a2), so a query row keeps one key interval [lo, hi).
 //
 // One CTA per (head, 128-row query tile), one key tile of 128 rows at a time:
-//   S = Q K^T          D/8 tcgen05.mma kind::tf32 (K = 8) into TMEM
-//   P = exp2(S - m)    fp32 softmax, P rounded to tf32 and written over S
-//   O += P V           16 tcgen05.mma kind::tf32 with A = P from TMEM
+//   S_k = Q K_k^T      D/8 tcgen05.mma kind::tf32 (K = 8) into TMEM
+//   P = exp2(S - m)    fp32 softmax, P rounded to tf32 and written over S_k
+//   O += P V_k         16 tcgen05.mma kind::tf32 with A = P from TMEM
+// Two S buffers: S_{k+1} is computed while the softmax works on S_k, and
+// P_k V_k follows.
 // Q, K and V stay fp32 in memory; the tensor cores read their top 19 bits
 // (tf32), the softmax, the row sums and the accumulators are fp32.  P is
 // rounded to tf32 before both its row sum and the product, so each output row
@@ -21,10 +23,9 @@
 // CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, descriptor layout 1: 4-row atoms of
 // 512 bytes).  Warps 0-3 own the query rows
 // (thread t = row t = TMEM lane t), warp 4 issues the TMA loads of a ring of
-// K and V tiles, warp 5 the MMAs.  TMEM: S / P in columns [0, 128), O in
-// [128, 128 + D).  The tile's S waits for the previous P V (one S buffer);
-// fp32 tensors are the small configurations, so the kernel keeps one simple
-// pipeline instead of the bf16 kernel's two query tiles per CTA.
+// K and V tiles (in the order the MMAs take them: K_0, K_1, V_0, K_2, V_1,
+// ...), warp 5 the MMAs.  TMEM: S / P of even tiles in columns [0, 128), of
+// odd tiles in [128, 256), O in [256, 256 + D).
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -36,13 +37,17 @@ struct TCfg {
   static constexpr int BLOCKS = D / 32;                  // 32-column (128-byte) blocks per row
   static constexpr int BLK_BYTES = 128 * 128;            // one block of 128 rows
   static constexpr int TILE_BYTES = BLOCKS * BLK_BYTES;  // 128 rows x D fp32
-  static constexpr int NS = (D == 128) ? 2 : (D == 64) ? 4 : 6;  // K / V ring slots
+  // K / V ring slots; the shared memory also keeps a second CTA (which would
+  // wait for the 512 TMEM columns) off the SM
+  static constexpr int NS = (D == 128) ? 2 : (D == 64) ? 4 : 8;
   static constexpr int SMEM_BAR = TILE_BYTES * (1 + NS);
   static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers; 1024-byte alignment slack
   static constexpr int THREADS = 192;
-  static constexpr int TMEM_COLS = 256;
-  static_assert(128 + D <= TMEM_COLS, "S and O must fit the TMEM allocation");
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t COL_O = 256;
+  static_assert(COL_O + D <= TMEM_COLS, "two S buffers and O must fit the TMEM allocation");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(2 * SMEM_BYTES > 228 * 1024, "one CTA per SM");
 };
 
 struct Tf32Params {
@@ -119,10 +124,10 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
   uint64_t* bar_q = bars;
   uint64_t* bar_full = bars + 1;             // [NS] K or V tile landed
   uint64_t* bar_empty = bars + 1 + C::NS;    // [NS] slot read by the MMAs
-  uint64_t* bar_s = bars + 1 + 2 * C::NS;    // S of the current key tile ready
-  uint64_t* bar_p = bar_s + 1;               // P written (128 arrivals)
-  uint64_t* bar_o = bar_p + 1;               // the last P V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_o + 1);
+  uint64_t* bar_s = bars + 1 + 2 * C::NS;    // [2] S of tile k ready in buffer k & 1
+  uint64_t* bar_p = bar_s + 2;               // P_k written (128 arrivals)
+  uint64_t* bar_pv = bar_p + 1;              // P_k V_k done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_pv + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -146,9 +151,10 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
       mbar_init(&bar_full[s], 1);
       mbar_init(&bar_empty[s], 1);
     }
-    mbar_init(bar_s, 1);
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
     mbar_init(bar_p, 128);
-    mbar_init(bar_o, 1);
+    mbar_init(bar_pv, 1);
     fence_barrier_init();
   }
   if (warp == 5) {
@@ -181,8 +187,11 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
         atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
         break;
       }
-      const CUtensorMap* tm = (n & 1) ? tv : tk;
-      const int row = (kt0 + (n >> 1)) * 128;
+      // entry n: K_0; K_{k+1} at 2k + 1; V_k at 2k + 2 (the last V at 2 nk - 1)
+      const bool is_v = n > 0 && !((n & 1) && (n + 1) / 2 < nk);
+      const int t = n == 0 ? 0 : !is_v ? (n + 1) / 2 : (n & 1) ? nk - 1 : n / 2 - 1;
+      const CUtensorMap* tm = is_v ? tv : tk;
+      const int row = (kt0 + t) * 128;
       in_range(row, L, p.status);
       mbar_arrive_expect_tx(&bar_full[slot], C::TILE_BYTES);
 #pragma unroll
@@ -195,34 +204,46 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
     constexpr uint32_t idesc_pv = idesc_tf32(128, D, 1);
     const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
     const uint32_t ring = smem_u32(sRing);
-    bool ok = wait_all(bar_q, 0, p.wait_ns);
-    for (int k = 0; ok && k < nk; ++k) {
-      const int nK = 2 * k, nV = 2 * k + 1;
-      const int slotK = nK % C::NS, slotV = nV % C::NS;
-      ok = wait_all(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
-      if (!ok) break;
-      tc_fence_after();
-      // S = Q K^T: K = 8 columns (32 bytes) per instruction inside a
-      // 128-byte block, then the next block
-      const uint64_t dk = smem_desc_sw128(ring + slotK * C::TILE_BYTES, 16, 1024);
+    // S_j = Q K_j^T into buffer j & 1: K = 8 columns (32 bytes) per
+    // instruction inside a 128-byte block, then the next block
+    auto qk = [&](int j, int slot) {
+      const uint64_t dk = smem_desc_sw128(ring + slot * C::TILE_BYTES, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 8; ++kk) {
         const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::BLK_BYTES + (kk & 3) * 32) >> 4);
-        ss_tf32(tmem, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+        ss_tf32(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
       }
-      umma_commit_warp(bar_s);  // also tells the softmax the previous P V is done
-      umma_commit_warp(&bar_empty[slotK]);
+      umma_commit_warp(&bar_s[j & 1]);
+      umma_commit_warp(&bar_empty[slot]);
+    };
+    bool ok = wait_all(bar_q, 0, p.wait_ns) && wait_all(&bar_full[0], 0, p.wait_ns);
+    if (ok) {
+      tc_fence_after();
+      qk(0, 0);
+    }
+    for (int k = 0; ok && k < nk; ++k) {
+      // S_{k+1} goes into the other buffer, whose last reader (P_{k-1} V_{k-1})
+      // was issued before it
+      if (k + 1 < nk) {
+        const int nK = 2 * k + 1, slotK = nK % C::NS;
+        ok = wait_all(&bar_full[slotK], (nK / C::NS) & 1, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+        qk(k + 1, slotK);
+      }
+      const int nV = (k + 1 < nk) ? 2 * k + 2 : 2 * nk - 1, slotV = nV % C::NS;
       ok = wait_all(bar_p, k & 1, p.wait_ns) && wait_all(&bar_full[slotV], (nV / C::NS) & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      // O += P V: V MN-major (its 32-column blocks one BLK_BYTES apart, 4-row
-      // atoms 512 bytes apart), 8 keys (two atoms, 1024 bytes) per instruction
+      // O += P_k V_k: V MN-major (its 32-column blocks one BLK_BYTES apart,
+      // 4-row atoms 512 bytes apart), 8 keys (two atoms, 1024 bytes) per
+      // instruction
       const uint64_t dv = smem_desc_sw128_32b(ring + slotV * C::TILE_BYTES, C::BLK_BYTES, 512);
 #pragma unroll
       for (int kk = 0; kk < 128 / 8; ++kk)
-        ts_tf32(tmem + 128, tmem + kk * 8, dv + static_cast<uint64_t>((kk * 1024) >> 4), idesc_pv,
-                (k > 0 || kk > 0) ? 1u : 0u);
-      if (k + 1 == nk) umma_commit_warp(bar_o);
+        ts_tf32(tmem + C::COL_O, tmem + (k & 1) * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 1024) >> 4),
+                idesc_pv, (k > 0 || kk > 0) ? 1u : 0u);
+      umma_commit_warp(bar_pv);
       umma_commit_warp(&bar_empty[slotV]);
     }
     if (!ok && lane == 0) {
@@ -244,12 +265,13 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
     float m = -INFINITY, l = 0.f;
     bool ok = run;
     for (int k = 0; ok && k < nk; ++k) {
-      ok = wait_all(bar_s, k & 1, p.wait_ns);
+      const uint32_t tS = trow + (k & 1) * 128;
+      ok = wait_all(&bar_s[k & 1], (k >> 1) & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       uint32_t v[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(trow + c * 32, *reinterpret_cast<uint32_t(*)[32]>(v + c * 32));
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(v + c * 32));
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v + c * 32));  // no use before the wait
@@ -263,19 +285,26 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
         mx = fmaxf(mx, sv);
       }
       const float m_new = fmaxf(m, mx);
-      // O holds P V of the earlier tiles (complete: the commit behind bar_s
-      // covers it); rescale it when this row's reference grew
+      // O holds P V of the earlier tiles once P_{k-1} V_{k-1} is done.  Waiting
+      // for it every tile also keeps this tile's P arrival behind the MMA
+      // warp's wait for the previous one (no two bar_p phases in flight).
+      if (k > 0) {
+        ok = wait_all(bar_pv, (k - 1) & 1, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // rescale O when this row's reference grew
       const float alpha = (m_new == -INFINITY || m == m_new) ? 1.f : ex2_approx(m - m_new);
       if (__any_sync(0xffffffffu, k > 0 && alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
-          tmem_ld32(trow + 128 + c * 32, ov);
+          tmem_ld32(trow + C::COL_O + c * 32, ov);
           tmem_wait_ld();
           reg_fence32(ov);
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(trow + 128 + c * 32, ov);
+          tmem_st32(trow + C::COL_O + c * 32, ov);
         }
       }
       float sum = 0.f;
@@ -289,12 +318,12 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
       l = l * alpha + sum;
       m = m_new;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st32(trow + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(v + c * 32));
+      for (int c = 0; c < 4; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(v + c * 32));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
     }
-    if (ok) ok = wait_all(bar_o, 0, p.wait_ns);
+    if (ok) ok = wait_all(bar_pv, (nk - 1) & 1, p.wait_ns);
     if (ok) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -303,7 +332,7 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
-        tmem_ld32(trow + 128 + c * 32, ov);
+        tmem_ld32(trow + C::COL_O + c * 32, ov);
         tmem_wait_ld();
         reg_fence32(ov);
         if (store_ok) {

@@ -22,9 +22,11 @@
 // tf32 needs the 128-byte swizzle of 32-byte chunks (TMA
 // CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, descriptor layout 1: 4-row atoms of
 // 512 bytes).  Warps 0-3 own the query rows
-// (thread t = row t = TMEM lane t), warp 4 issues the TMA loads of a ring of
+// (two threads per row: warps w and w + 4 take keys [0, 64) and [64, 128) of
+// row 32 (w & 3) + lane = TMEM lane, and exchange their maxima once per tile
+// through shared memory), warp 8 issues the TMA loads of a ring of
 // K and V tiles (in the order the MMAs take them: K_0, K_1, V_0, K_2, V_1,
-// ...), warp 5 the MMAs.  TMEM: S / P of even tiles in columns [0, 128), of
+// ...), warp 9 the MMAs.  TMEM: S / P of even tiles in columns [0, 128), of
 // odd tiles in [128, 256), O in [256, 256 + D).
 #include "internal.h"
 #include "sm100.cuh"
@@ -41,8 +43,9 @@ struct TCfg {
   // wait for the 512 TMEM columns) off the SM
   static constexpr int NS = (D == 128) ? 2 : (D == 64) ? 4 : 8;
   static constexpr int SMEM_BAR = TILE_BYTES * (1 + NS);
-  static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers; 1024-byte alignment slack
-  static constexpr int THREADS = 192;
+  static constexpr int SMEM_X = SMEM_BAR + 256;               // half-row maxima [2][2][128], sums [2][128]
+  static constexpr int SMEM_BYTES = SMEM_X + 3072 + 1024;     // 1024-byte alignment slack
+  static constexpr int THREADS = 320;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 256;
   static_assert(COL_O + D <= TMEM_COLS, "two S buffers and O must fit the TMEM allocation");
@@ -114,7 +117,7 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, uint64_
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant__ Tf32Params p) {
+__global__ void __launch_bounds__(320, 1) attn_tf32_kernel(const __grid_constant__ Tf32Params p) {
   using C = TCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -127,7 +130,8 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
   uint64_t* bar_s = bars + 1 + 2 * C::NS;    // [2] S of tile k ready in buffer k & 1
   uint64_t* bar_p = bar_s + 2;               // P_k written (128 arrivals)
   uint64_t* bar_pv = bar_p + 1;              // P_k V_k done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_pv + 1);
+  uint64_t* bar_x = bar_pv + 1;              // [4] 64 arrivals: the two halves of 32 rows exchanged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_x + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -153,11 +157,12 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
     }
     mbar_init(&bar_s[0], 1);
     mbar_init(&bar_s[1], 1);
-    mbar_init(bar_p, 128);
+    mbar_init(bar_p, 256);
     mbar_init(bar_pv, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bar_x[q], 64);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
   const uint32_t tmem = *tmem_slot;
   const bool run = (*abort_flag == 0) && nk > 0;
 
-  if (run && warp == 4 && lane == 0) {
+  if (run && warp == 8 && lane == 0) {
     // ------------------------------------------------ TMA producer
     const CUtensorMap* tq = lab ? &p.tm_qp : &p.tm_q;
     const CUtensorMap* tk = lab ? &p.tm_kp : &p.tm_k;
@@ -198,7 +203,7 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
       for (int b = 0; b < C::BLOCKS; ++b)
         tma_load_4d(sRing + slot * C::TILE_BYTES + b * C::BLK_BYTES, tm, &bar_full[slot], b * 32, row, th, tb);
     }
-  } else if (run && warp == 5) {
+  } else if (run && warp == 9) {
     // ------------------------------------------------ MMA issuer (whole warp; one elected lane issues)
     constexpr uint32_t idesc_qk = idesc_tf32(128, 128, 0);
     constexpr uint32_t idesc_pv = idesc_tf32(128, D, 1);
@@ -250,9 +255,10 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
       *abort_flag = 1;
       atomicOr(p.status, static_cast<int>(SVG_DEV_TIMEOUT));
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------ rows: softmax and epilogue
-    const int r = threadIdx.x;  // query row of the tile = TMEM lane
+    const int q = warp & 3, h = warp >> 2;  // lane quarter; key half [64 h, 64 h + 64) of every tile
+    const int r = q * 32 + lane;             // query row of the tile = TMEM lane
     const int x = q0 + r;
     const bool row_ok = x < L;
     int lo = 0, hi = 0;
@@ -261,30 +267,39 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
       lo = static_cast<int>(max(0LL, (g - a + 1) * G));
       hi = static_cast<int>(min(static_cast<long long>(L), (g + a) * G));
     }
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float* xm = reinterpret_cast<float*>(smem + C::SMEM_X);  // [2 parity][2 half][128 rows]
+    float* fin = xm + 512;                                     // [2 half][128 rows] row sums
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tO = trow + C::COL_O + h * (D / 2);  // this half's output columns
     float m = -INFINITY, l = 0.f;
     bool ok = run;
     for (int k = 0; ok && k < nk; ++k) {
-      const uint32_t tS = trow + (k & 1) * 128;
+      const uint32_t tS = trow + (k & 1) * 128 + h * 64;
       ok = wait_all(&bar_s[k & 1], (k >> 1) & 1, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(v + c * 32));
+      uint32_t v[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
       tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v + c * 32));  // no use before the wait
-      const int y0 = (kt0 + k) * 128;
+      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v));  // no use before the wait
+      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      const int y0 = (kt0 + k) * 128 + h * 64;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < 64; ++c) {
         const int y = y0 + c;
         const float sv = (y >= lo && y < hi) ? __uint_as_float(v[c]) * p.sl2 : -INFINITY;
         v[c] = __float_as_uint(sv);
         mx = fmaxf(mx, sv);
       }
-      const float m_new = fmaxf(m, mx);
+      // the row's maximum over the whole tile, from both halves
+      float* xk = xm + (k & 1) * 256;
+      xk[h * 128 + r] = mx;
+      mbar_arrive(&bar_x[q]);
+      ok = wait_all(&bar_x[q], k & 1, p.wait_ns);
+      if (!ok) break;
+      const float m_new = fmaxf(m, fmaxf(mx, xk[(h ^ 1) * 128 + r]));
       // O holds P V of the earlier tiles once P_{k-1} V_{k-1} is done.  Waiting
       // for it every tile also keeps this tile's P arrival behind the MMA
       // warp's wait for the previous one (no two bar_p phases in flight).
@@ -293,23 +308,24 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
         if (!ok) break;
         tc_fence_after();
       }
-      // rescale O when this row's reference grew
+      // rescale this half of O when the row's reference grew (both halves
+      // take the same decision: same m, same m_new)
       const float alpha = (m_new == -INFINITY || m == m_new) ? 1.f : ex2_approx(m - m_new);
       if (__any_sync(0xffffffffu, k > 0 && alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(trow + C::COL_O + c * 32, ov);
+          uint32_t ov[16];
+          tmem_ld16(tO + c * 16, ov);
           tmem_wait_ld();
-          reg_fence32(ov);
+          reg_fence16(ov);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(trow + C::COL_O + c * 32, ov);
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st16(tO + c * 16, ov);
         }
       }
       float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < 64; ++c) {
         const float sv = __uint_as_float(v[c]);
         const float pr = (m_new == -INFINITY) ? 0.f : ex2_approx(sv - m_new);  // masked: exp2(-inf) = 0
         v[c] = to_tf32(pr);
@@ -317,28 +333,35 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
       }
       l = l * alpha + sum;
       m = m_new;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(v + c * 32));
+      tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(v));
+      tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(v + 32));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
     }
+    // the row sum of both halves
+    if (ok) {
+      fin[h * 128 + r] = l;
+      mbar_arrive(&bar_x[q]);
+      ok = wait_all(&bar_x[q], nk & 1, p.wait_ns);
+    }
     if (ok) ok = wait_all(bar_pv, (nk - 1) & 1, p.wait_ns);
     if (ok) {
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lt = fin[r] + fin[128 + r];
+      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       const bool store_ok = row_ok && in_range(x, L, p.status) && in_range(bh, p.BH, p.status);
-      float* out = (lab ? p.op : p.o) + st.head(store_ok ? bh : 0) + (store_ok ? x : 0) * st.sl;
+      float* out = (lab ? p.op : p.o) + st.head(store_ok ? bh : 0) + (store_ok ? x : 0) * st.sl + h * (D / 2);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(trow + C::COL_O + c * 32, ov);
+        uint32_t ov[16];
+        tmem_ld16(tO + c * 16, ov);
         tmem_wait_ld();
-        reg_fence32(ov);
+        reg_fence16(ov);
         if (store_ok) {
-          float4* dst = reinterpret_cast<float4*>(out + c * 32);
+          float4* dst = reinterpret_cast<float4*>(out + c * 16);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
+          for (int e = 0; e < 4; ++e)
             dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l, __uint_as_float(ov[4 * e + 1]) * inv_l,
                                  __uint_as_float(ov[4 * e + 2]) * inv_l, __uint_as_float(ov[4 * e + 3]) * inv_l);
         }
@@ -351,7 +374,7 @@ __global__ void __launch_bounds__(192, 1) attn_tf32_kernel(const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

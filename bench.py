@@ -47,7 +47,8 @@ NCU_TRAFFIC = {("645b18066bbc1e1a", "d2f4abb45748fc0c", "fused"): 2.8525e9,
 
 # The same for the profiling stage-1 kernel (full HunyuanVideo launch), keyed by
 # the sha256 prefix of its source.
-PROF_NCU_TRAFFIC = {"5732be8477404d60": 1.488e9, "a5d1bd300122e4a1": 1.4840e9, "cabba81d0b39bcb9": 1.4901e9}
+PROF_NCU_TRAFFIC = {"5732be8477404d60": 1.488e9, "a5d1bd300122e4a1": 1.4840e9, "cabba81d0b39bcb9": 1.4901e9,
+                    "cfcfb262609a7c06": 1.4874e9}
 
 
 def prof_source_key():

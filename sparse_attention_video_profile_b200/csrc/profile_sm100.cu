@@ -381,6 +381,9 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
     // One softmax reference (the running max over all kept keys of the row)
     // serves the three variants: P_s and P_t are P_d restricted to their masks.
     float m_ref = -INFINITY, l_d = 0.f, l_s = 0.f, l_t = 0.f;
+    // in-frame position of this half's first key, carried from tile to tile
+    // (one division here instead of one per tile)
+    int j0h = ((kt0 * 128 + h * 64) % p.F);
     int inband_s = 0, inband_t = 0;
     bool ok = true;
     for (int k = 0; k < nk; ++k) {
@@ -412,7 +415,7 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
         if (p.kind[v] == kMaskPositionBand) {
           const int a = p.par[v];
           int c = 0;
-          int j0 = kbase % p.F;
+          int j0 = j0h;
           while (c < nv) {  // one frame segment per pass: keys c .. c + (F - j0) - 1
             const int seg_end = min(nv, c + (p.F - j0));
             const int lo = max(c, c + (jr - a + 1 - j0));
@@ -425,6 +428,8 @@ __global__ void __launch_bounds__(320, 1) profile_sm100_kernel(const __grid_cons
           set_range64(mv, max(lo_v[v] - kbase, 0), min(hi_v[v] - kbase, nv));
         }
       }
+      j0h += 128;  // the next tile's first key of this half
+      if (j0h >= p.F) j0h = (p.F >= 128) ? j0h - p.F : j0h % p.F;
       // keys past the chunk end get weight 0 in every variant
       if (nv < 64) {
 #pragma unroll

@@ -21,8 +21,6 @@ import oracle
 from sparse_attention_video_profile_b200 import svg
 from test_gpu_parity import DEV, check_profile, f64, profile_bounds
 
-pytestmark = pytest.mark.gpu
-
 TOLS = {"bf16": (2e-2, 1e-2), "fp32": (1e-4, 1e-5), "tf32": (1e-2, 4e-3)}
 N_CASES = 20
 
@@ -50,6 +48,7 @@ def _id(c):
     return "{kind}-B{B}H{H}N{N}F{F}d{d}-a{a1},{a2}-S{S}-{layout}".format(**c)
 
 
+@pytest.mark.gpu
 @pytest.mark.parametrize("case", CASES, ids=_id)
 def test_whole_call_random_shapes(case):
     c = case

@@ -294,6 +294,26 @@ def test_sparse_3d_attn_end_to_end(name):
     assert_close(f64(o), ref, q.dtype, name)
 
 
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_sparse_3d_attn_literal_embedding_scale(name):
+    """The whole call on the literal reading of the synthetic heads
+    (embeddings N(0, 1) / sqrt(d), where the labels invert): profiling within
+    the bound, labels as the oracle's, output within the bar."""
+    wl = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(wl, seed=0, device=DEV, emb_std=wl.d ** -0.5)
+    rows_np = synth.sample_rows(wl.L, wl.S, 0)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, mse, label = svg.svg_sparse_3d_attn(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows, status=status)
+    sync_ok(status)
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    ref_mse, ref_label = oracle.profile_heads(qn, kn, vn, wl.N, wl.F, wl.a1, wl.a2, rows_np)
+    check_profile(mse, label, ref_mse, ref_label,
+                  profile_bounds(qn, kn, vn, wl.N, wl.F, wl.a1, wl.a2, rows_np, fp32=q.dtype == torch.float32))
+    ref = oracle.sparse_attention(qn, kn, vn, label.cpu().numpy(), wl.N, wl.F, wl.a1, wl.a2)
+    assert_close(f64(o), ref, q.dtype, name + " (literal embedding scale)")
+
+
 def test_full_bands_equal_dense():
     wl = synth.WORKLOADS["small"]
     q, k, v = synth.make_qkv(wl, seed=2, device=DEV)

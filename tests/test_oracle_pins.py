@@ -300,6 +300,19 @@ def test_synthetic_heads_get_their_constructed_labels(name):
     assert np.all(gap > 0.2)
 
 
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_literal_embedding_scale_inverts_the_labels(name):
+    """The literal reading of the synthetic heads (embeddings N(0, 1) / sqrt(d))
+    gives each head the opposite label: its in-band logit boost, about
+    w^2 / sqrt(d), is too small to concentrate the softmax in its band.  This is
+    why the default scale is d^(-1/4) (boost about w^2)."""
+    wl = synth.WORKLOADS[name]
+    q, k, v = (synth.round_bf16_to_f64(t) for t in synth.make_qkv(wl, seed=0, emb_std=wl.d ** -0.5))
+    rows = synth.sample_rows(wl.L, wl.S, 0)
+    mse, label = oracle.profile_heads(q, k, v, wl.N, wl.F, wl.a1, wl.a2, rows)
+    np.testing.assert_array_equal(label, 1 - synth.head_kinds(wl, 0))
+
+
 # ------------------------------------------------------------ block list pin
 
 def _banded_tile_ranges(L, G, a, Bq, Bk, qb):

@@ -22,7 +22,7 @@ from sparse_attention_video_profile_b200 import svg
 from test_gpu_parity import DEV, check_profile, f64, profile_bounds
 
 TOLS = {"bf16": (2e-2, 1e-2), "fp32": (1e-4, 1e-5), "tf32": (1e-2, 4e-3)}
-N_CASES = 20
+N_CASES = 40
 
 
 def draw_case(i):
